@@ -1,0 +1,538 @@
+"""Benchmark of the InPlace-ABN layer (training forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole layer over one batch: iabn_forward (x -> z in
+place), iabn_backward (dz -> dx in place, dgamma, dbeta) and
+iabn_update_running_stats, on the ResNet-trunk workload: NHWC bf16 storage,
+N=64 C=256 H=W=56, leaky-ReLU 0.01.  Inputs are synthetic (seeded, same value
+recipe as the tests) and restored before every step (the layer is in place);
+the L2 cache is flushed (a 2x-L2 write) before every forward and every
+backward call, outside the timed events.
+
+Metric: GB/s of compulsory traffic, 5*E*s bytes per step (the forward reads x
+and writes z; the backward reads z and dz and writes dx), divided by the
+device time of the three calls (CUDA events on the launching stream).  Under
+torchrun (N > 1) every rank runs its own replica (no cross-GPU statistics):
+value = N * bytes / max-over-ranks time ("weak" scaling).
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
+oracle (test infrastructure) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elements/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_hbm_gbs():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads and the CPU baseline")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz, self.error = [], set(), None, None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(pynvml, device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # no NVML: report why
+            self.nv, self.error = None, repr(e)
+
+    @staticmethod
+    def _handle(pynvml, idx):
+        import torch
+        try:
+            p = torch.cuda.get_device_properties(idx)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for b, name in self.REASONS.items():
+            if bits & b:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception as e:
+                self.error = repr(e)
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.nv is not None:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+               "samples": len(self.samples)}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+# ------------------------------------------------------------------ inputs
+
+def device_inputs(sp, seed, gen_device):
+    """Synthetic layer inputs drawn on the device (same recipe as the tests:
+    mu_c ~ U(-2,2), sigma_c ~ U(0.5,3), x = mu + sigma*N(0,1) (Student-t(3)
+    for the segmentation workload), gamma = +-U(lo,1.5), beta ~ N(0, 0.1),
+    dz ~ N(0,1))."""
+    import torch
+    import workloads as wl
+    g = torch.Generator(device=gen_device).manual_seed(seed)
+    n, c, h, w = sp.shape
+    dev = gen_device
+    mu = torch.rand(c, generator=g, device=dev, dtype=torch.float32) * 4 - 2
+    sig = torch.rand(c, generator=g, device=dev) * 2.5 + 0.5
+    sign = torch.where(torch.rand(c, generator=g, device=dev) < 0.5, -1.0, 1.0)
+    gamma = sign * (torch.rand(c, generator=g, device=dev) * (1.5 - sp.gamma_lo) + sp.gamma_lo)
+    beta = torch.randn(c, generator=g, device=dev) * (0.1 ** 0.5)
+    shape_l = (n, h, w, c) if sp.layout == wl.NHWC else (n, c, h, w)
+    bshape = (1, 1, 1, c) if sp.layout == wl.NHWC else (1, c, 1, 1)
+    if sp.x_dist == "student_t3":
+        z = torch.randn(shape_l, generator=g, device=dev)
+        chi = sum(torch.randn(shape_l, generator=g, device=dev) ** 2 for _ in range(3))
+        e = z / torch.sqrt(chi / 3.0)
+    else:
+        e = torch.randn(shape_l, generator=g, device=dev)
+    x = (mu.view(bshape) + sig.view(bshape) * e).to(wl.torch_dtype(sp.dtype)).reshape(-1)
+    dz = torch.randn(shape_l, generator=g, device=dev).to(wl.torch_dtype(sp.dtype)).reshape(-1)
+    return x, dz, gamma.contiguous(), beta.contiguous()
+
+
+class Layer:
+    """Device buffers of one layer plus its pristine inputs."""
+
+    def __init__(self, sp, seed, device):
+        import torch
+        import place_batchnorm_activation_b200 as iabn
+        self.iabn, self.sp = iabn, sp
+        self.x0, self.dz0, self.gamma, self.beta = device_inputs(sp, seed, device)
+        self.x = self.x0.clone()
+        self.dz = self.dz0.clone()
+        c = sp.c
+        self.mean = torch.empty(c, device=device)
+        self.var = torch.empty(c, device=device)
+        self.dgamma = torch.empty(c, device=device)
+        self.dbeta = torch.empty(c, device=device)
+        self.rmean = torch.zeros(c, device=device)
+        self.rvar = torch.ones(c, device=device)
+        self.ws = iabn.new_workspace(sp.shape, sp.layout, sp.dtype, device=device)
+        self.bytes = 5 * sp.numel * sp.itemsize
+
+    def restore(self):
+        self.x.copy_(self.x0)
+        self.dz.copy_(self.dz0)
+
+    def fwd(self):
+        sp = self.sp
+        self.iabn.forward(self.x, self.gamma, self.beta, self.mean, self.var, self.ws,
+                          shape=sp.shape, layout=sp.layout, eps=sp.eps, act=sp.act,
+                          act_param=sp.act_param)
+
+    def bwd(self):
+        sp = self.sp
+        self.iabn.backward(self.x, self.dz, self.gamma, self.beta, self.var, self.dgamma,
+                           self.dbeta, self.ws, shape=sp.shape, layout=sp.layout, eps=sp.eps,
+                           act=sp.act, act_param=sp.act_param)
+
+    def run(self):
+        self.iabn.update_running_stats(self.mean, self.var, self.rmean, self.rvar,
+                                       count=self.sp.per_channel, momentum=self.sp.momentum)
+
+
+def timed_layer_steps(layer, flush, steps, warmup, dist_barrier=None, sampler=None):
+    """Warm-up, then `steps` timed steps; returns per-step event times (ms) of
+    fwd, bwd and the running-stat update, and the launch count in between."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(warmup):
+        layer.restore()
+        flush.zero_()
+        layer.fwd()
+        flush.zero_()
+        layer.bwd()
+        layer.run()
+    records = [(ev(), ev(), ev(), ev(), ev(), ev()) for _ in range(steps)]
+    if dist_barrier:
+        dist_barrier()
+    torch.cuda.synchronize()
+    l0 = layer.iabn.iabn_kernel_launches()
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        t0 = time.perf_counter()
+        for r in records:
+            layer.restore()
+            flush.zero_()
+            r[0].record()
+            layer.fwd()
+            r[1].record()
+            flush.zero_()
+            r[2].record()
+            layer.bwd()
+            r[3].record()
+            r[4].record()
+            layer.run()
+            r[5].record()
+        if dist_barrier:
+            dist_barrier()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    launches = layer.iabn.iabn_kernel_launches() - l0
+    f = [r[0].elapsed_time(r[1]) for r in records]
+    b = [r[2].elapsed_time(r[3]) for r in records]
+    u = [r[4].elapsed_time(r[5]) for r in records]
+    return f, b, u, launches, wall
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def e2e_steps(layer, steps, warmup):
+    """Through the public API with host buffers: pinned host x, dz -> device,
+    forward, backward, running stats, z and dx (and dgamma, dbeta) -> host.
+    Returns per-step ms and bytes moved each way."""
+    import torch
+    hx = layer.x0.cpu().pin_memory()
+    hdz = layer.dz0.cpu().pin_memory()
+    hz = torch.empty_like(hx).pin_memory()
+    hdx = torch.empty_like(hdz).pin_memory()
+    hg = torch.empty_like(layer.dgamma, device="cpu").pin_memory()
+    hb = torch.empty_like(layer.dbeta, device="cpu").pin_memory()
+
+    def step():
+        layer.x.copy_(hx, non_blocking=True)
+        layer.dz.copy_(hdz, non_blocking=True)
+        layer.fwd()
+        layer.bwd()
+        layer.run()
+        hz.copy_(layer.x, non_blocking=True)
+        hdx.copy_(layer.dz, non_blocking=True)
+        hg.copy_(layer.dgamma, non_blocking=True)
+        hb.copy_(layer.dbeta, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in times]
+    h2d = hx.numel() * hx.element_size() + hdz.numel() * hdz.element_size()
+    d2h = (hz.numel() * hz.element_size() + hdx.numel() * hdx.element_size()
+           + hg.numel() * 4 + hb.numel() * 4)
+    return ms, h2d, d2h
+
+
+# -------------------------------------------------------- other workloads
+
+def bench_other_workloads(flush, steps, warmup, hbm_peak, device):
+    """Workloads 2-4 of the layer's benchmark set, same protocol (L2 flushed
+    before every call).  The layer sweep chains 16 layers (x_{l+1} is a
+    subsampled, channel-cycled copy of z_l, made outside the timed events),
+    forward l = 0..15 then backward l = 15..0 with a fresh dz per layer."""
+    import torch
+    import workloads as wl
+    out = {}
+    for wid in (2, 3):
+        sp = wl.spec(wid)
+        L = Layer(sp, sp.seed, device)
+        f, b, u, _, _ = timed_layer_steps(L, flush, steps, warmup)
+        tf, tb = statistics.median(f), statistics.median(b)
+        gbs = L.bytes / ((tf + tb) * 1e-3) / 1e9
+        out[sp.name] = {"fwd_us": round(tf * 1e3, 2), "bwd_us": round(tb * 1e3, 2),
+                        "gbs": round(gbs, 1), "frac_measured_hbm": round(gbs / hbm_peak, 4),
+                        "frac_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                        "elements_per_s": sp.numel / ((tf + tb) * 1e-3)}
+        del L
+        torch.cuda.empty_cache()
+    # layer sweep
+    layers = []
+    for l in range(len(wl.SWEEP_SHAPES)):
+        sp = wl.spec(4, l)
+        layers.append(Layer(sp, sp.seed, device))
+    base0 = layers[0].x0.clone()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def one_pass(rec):
+        layers[0].x.copy_(base0)
+        for l, L in enumerate(layers):
+            if l > 0:
+                a, b = layers[l - 1], L
+                za = a.x.view(a.sp.n, a.sp.h, a.sp.w, a.sp.c)
+                r = a.sp.h // b.sp.h
+                idx = torch.arange(b.sp.c, device=device) % a.sp.c
+                b.x.copy_(za[:, ::r, ::r, :][..., idx].reshape(-1))
+            flush.zero_()
+            rec[2 * l][0].record()
+            L.fwd()
+            rec[2 * l][1].record()
+        for l in range(len(layers) - 1, -1, -1):
+            L = layers[l]
+            L.dz.copy_(L.dz0)
+            flush.zero_()
+            rec[2 * l + 1][0].record()
+            L.bwd()
+            rec[2 * l + 1][1].record()
+
+    for _ in range(warmup):
+        one_pass([(ev(), ev()) for _ in range(2 * len(layers))])
+    torch.cuda.synchronize()
+    totals = []
+    for _ in range(max(3, steps // 4)):
+        rec = [(ev(), ev()) for _ in range(2 * len(layers))]
+        one_pass(rec)
+        torch.cuda.synchronize()
+        totals.append(sum(a.elapsed_time(b) for a, b in rec))
+    t = statistics.median(totals)
+    total_bytes = sum(L.bytes for L in layers)
+    gbs = total_bytes / (t * 1e-3) / 1e9
+    out["layer_sweep"] = {"sum_of_32_calls_us": round(t * 1e3, 2), "gbs": round(gbs, 1),
+                          "frac_measured_hbm": round(gbs / hbm_peak, 4),
+                          "frac_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                          "elements_per_s": sum(L.sp.numel for L in layers) / (t * 1e-3),
+                          "dz": "fresh N(0,1) per layer"}
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------ CPU (oracle)
+
+def oracle_pass(sp_sample):
+    """One forward + backward + running update of the oracle on a sample."""
+    import numpy as np
+    import oracle
+    import workloads as wl
+    inp = wl.draw(sp_sample)
+    g, b = inp.gamma.astype(np.float64), inp.beta.astype(np.float64)
+    eps, p = float(np.float32(sp_sample.eps)), float(np.float32(sp_sample.act_param))
+    t0 = time.perf_counter()
+    fw = oracle.forward(sp_sample.shape, sp_sample.layout, inp.x64, g, b, eps, sp_sample.act, p)
+    z = oracle.round_to(fw["z"], sp_sample.dtype)
+    bw = oracle.backward_inplace(sp_sample.shape, sp_sample.layout, z, inp.dz64, g, b,
+                                 fw["var"], eps, sp_sample.act, p)
+    oracle.round_to(bw["dx"], sp_sample.dtype)
+    oracle.running_update(sp_sample.per_channel, fw["mean"], fw["var"], 0.1,
+                          inp.running_mean, inp.running_var)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(batch: int):
+    import workloads as wl
+    sp = wl.spec(1).with_(n=batch)
+    t = oracle_pass(sp)
+    gbs = 5 * sp.numel * sp.itemsize / t / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"resnet_trunk workload with N={batch} instead of 64 "
+                      f"({sp.numel} elements), one fwd+bwd+running update, "
+                      f"single-threaded fp64 C oracle, {t:.2f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import workloads as wl
+    sp = wl.spec(1).with_(n=1)
+    for _ in range(args.warmup):
+        oracle_pass(sp)
+    times = [oracle_pass(sp) for _ in range(args.steps)]
+    t = statistics.mean(times)
+    gbs = 5 * sp.numel * sp.itemsize / t / 1e9
+    line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "resnet_trunk NHWC bf16 N=64 C=256 H=W=56 leaky_relu 0.01, "
+                                   "fwd+bwd+running stats; each step a bounded sample N=1",
+                       "sample_elements": sp.numel},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"N=1 slice of the resnet_trunk workload "
+                                       f"({sp.numel} elements) per step"},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- main
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+    import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    barrier = None
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        barrier = dist.barrier
+
+    hbm_peak, peak_kind = measured_hbm_gbs()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device=device)
+    sp = wl.spec(1)
+    layer = Layer(sp, sp.seed + 1000 * rank, device)
+
+    sampler = ClockSampler(local)
+    f, b, u, launches, wall = timed_layer_steps(layer, flush, args.steps, args.warmup,
+                                                barrier, sampler)
+    t_step = [x + y + z for x, y, z in zip(f, b, u)]
+    mean_ms = statistics.mean(t_step)
+    t_max = mean_ms
+    if world > 1:
+        tt = torch.tensor([mean_ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    value = world * layer.bytes / (t_max * 1e-3) / 1e9
+    fwd_us, bwd_us = statistics.mean(f) * 1e3, statistics.mean(b) * 1e3
+
+    # e2e through host buffers
+    e_ms, h2d, d2h = e2e_steps(layer, max(3, args.steps // 10), 2)
+    e_mean = statistics.mean(e_ms)
+    e_max = e_mean
+    if world > 1:
+        tt = torch.tensor([e_mean], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_max = float(tt.item())
+    e2e_value = world * layer.bytes / (e_max * 1e-3) / 1e9
+
+    extra = {}
+    if not args.no_extra and world == 1:
+        extra = bench_other_workloads(flush, max(5, args.steps // 5), 3, hbm_peak, device)
+
+    if rank == 0:
+        bwd_bytes = 3 * sp.numel * sp.itemsize
+        achieved = bwd_bytes / (bwd_us * 1e-6) / 1e9
+        fwd_achieved = 2 * sp.numel * sp.itemsize / (fwd_us * 1e-6) / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "resnet_trunk: NHWC, bf16 storage, N=64 C=256 H=W=56, "
+                                   "leaky_relu 0.01, eps 1e-5, fwd+bwd+running stats",
+                       "storage_dtype": "bf16", "elements": sp.numel,
+                       "compulsory_bytes_per_step": layer.bytes,
+                       "l2": "flushed (2x L2 write) before every fwd and every bwd call",
+                       "inputs": "restored from pristine device copies before each step",
+                       "parallelism": f"replicas x{world} (no cross-GPU statistics)",
+                       "plan": os.environ.get("IABN_FORCE_PLAN", "auto")},
+            "elements_per_s": world * sp.numel / (t_max * 1e-3),
+            "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
+            "running_update_us": round(statistics.mean(u) * 1e3, 2),
+            "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
+            "frac_of_measured_hbm": round(value / world / hbm_peak, 4),
+            "roofline": {"bound": "hbm", "kernel": "backward (iabn_backward)",
+                         "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": bwd_bytes},
+            "roofline_fwd": {"bound": "hbm", "achieved": round(fwd_achieved, 1),
+                             "peak": hbm_peak, "unit": "GB/s",
+                             "frac": round(fwd_achieved / hbm_peak, 4),
+                             "algorithmic_bytes_per_launch": 2 * sp.numel * sp.itemsize},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e_max, 3)},
+            "gpu_launches": int(launches),
+            "clocks": sampler.summary(),
+            "timed_wall_s": round(wall, 4),
+        }
+        if extra:
+            line["workloads"] = extra
+        if not args.no_extra and world == 1:
+            line["cpu_baseline"] = cpu_baseline(32)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,158 @@
+/*
+ * iabn.h -- C ABI of libiabn.so: In-Place Activated BatchNorm (InPlace-ABN)
+ * for NVIDIA B200 (sm_100a), training mode, one GPU.
+ *
+ * The layer fuses batch normalisation and an invertible activation and keeps
+ * a single buffer: the forward overwrites its input x with the activated
+ * output z; the backward recovers what it needs from z alone by inverting
+ * the activation and the scale-and-shift, and overwrites the incoming
+ * gradient dz with dx.
+ *
+ * Sources (web pages about the method; cited by title and section):
+ *   [ABN] "In-Place Activated BatchNorm for Memory-Optimized Training of
+ *         DNNs" (Rota Bulo, Porzi, Kontschieder; CVPR 2018), the
+ *         section-by-section summary on paperlayer.ai: section 3 "In-Place
+ *         Activated Batch Normalization" -- bullets "INPLACE-ABN" (one buffer,
+ *         invertible activation and scale-and-shift), "Batch Normalization
+ *         Review" (empirical mean and variance, learnable gamma and beta),
+ *         "INPLACE-ABN II" (gradients written in terms of y); section 4
+ *         "Experimental setup" (leaky-ReLU, slope 0.01).  The abstract (same
+ *         title, codewithpapers.app and app.cochat.ai pages) calls it a single
+ *         plugin layer for existing frameworks.
+ *   [BN]  Ioffe & Szegedy, "Batch Normalization ...", cited in that paper's
+ *         reference list: batch statistics and the BN backward.
+ *
+ * Conventions for every call
+ *   - Every pointer argument except `stream` is a DEVICE pointer to memory
+ *     owned by the caller.  The library allocates nothing and keeps no state
+ *     between calls other than per-device launch settings.
+ *   - All calls are asynchronous and ordered on `stream` (a cudaStream_t;
+ *     NULL means the legacy default stream), except iabn_get_device_status.
+ *   - Arguments are checked on the host before anything is launched; a
+ *     rejected call launches nothing and returns the error.
+ *   - Element (n, c, h, w) of a tensor lives at ((n*C + c)*H + h)*W + w for
+ *     IABN_NCHW and ((n*H + h)*W + w)*C + c for IABN_NHWC.  M = N*H*W is the
+ *     number of values per channel.
+ *   - Activation tensors (x/z, dz/dx) use the storage type `dtype`; gamma,
+ *     beta, statistics and parameter gradients are always float32 [C].  All
+ *     arithmetic is float32 (statistics combined in float64), with one
+ *     round-to-nearest-even into the storage type per written element.
+ *   - Activation tensors must start on a 16-byte boundary
+ *     (IABN_ERR_MISALIGNED otherwise).
+ *   - One workspace may serve only one call in flight at a time.  It must be
+ *     zero-filled once before its first use; each call leaves it reusable.
+ *     Its size is given by iabn_workspace_size and depends only on the
+ *     descriptor.
+ *   - Errors found on the device never trap: they set a sticky status word
+ *     in the workspace that iabn_get_device_status reads.
+ */
+#ifndef IABN_H
+#define IABN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    IABN_OK = 0,
+    IABN_ERR_INVALID_ARG = 1,    /* null pointer, bad dimension, M < 2, bad parameter */
+    IABN_ERR_UNSUPPORTED = 2,    /* valid but not supported (e.g. sizes beyond int64) */
+    IABN_ERR_MISALIGNED = 3,     /* an activation tensor is not 16-byte aligned */
+    IABN_ERR_WORKSPACE = 4,      /* workspace missing or smaller than iabn_workspace_size */
+    IABN_ERR_CUDA = 5,           /* a CUDA runtime call failed (launch, copy, ...) */
+    IABN_ERR_TIMEOUT = 6,        /* device: a bounded wait inside a kernel ran out */
+    IABN_ERR_SINGULAR_GAMMA = 7  /* device: |gamma_c| < FLT_MIN in a backward call */
+} iabn_status;
+
+typedef enum { IABN_NCHW = 0, IABN_NHWC = 1 } iabn_layout;
+typedef enum { IABN_F32 = 0, IABN_BF16 = 1, IABN_F16 = 2 } iabn_dtype;
+
+/* The activation phi.  The positive branch is taken iff its argument is > 0.
+ *   IABN_ACT_LEAKY_RELU: phi(y) = y (y > 0), a*y otherwise; act_param = a > 0.
+ *   IABN_ACT_ELU:        phi(y) = y (y > 0), alpha*(e^y - 1) otherwise;
+ *                        act_param = alpha > 0.
+ *   IABN_ACT_IDENTITY:   phi(y) = y (plain batch normalisation); act_param unused. */
+typedef enum { IABN_ACT_LEAKY_RELU = 0, IABN_ACT_ELU = 1, IABN_ACT_IDENTITY = 2 } iabn_act;
+
+/* Tensor descriptor: logical shape N x C x H x W, memory layout and storage
+ * type (iabn_layout / iabn_dtype values). */
+typedef struct {
+    int64_t n, c, h, w;
+    int32_t layout;
+    int32_t dtype;
+} iabn_desc;
+
+/* Bytes of workspace the forward and backward calls need for descriptor `d`
+ * (a multiple of 256).  Returns 0 if the descriptor is invalid.  Host-only. */
+size_t iabn_workspace_size(const iabn_desc* d);
+
+/* Forward, training mode ([ABN] section 3, "Batch Normalization Review" and
+ * "INPLACE-ABN"; [BN] Algorithm 1).
+ *   mean_c = (1/M) sum x,  var_c = (1/M) sum (x - mean_c)^2   (biased),
+ *   xhat = (x - mean_c) / sqrt(var_c + eps),  y = gamma_c*xhat + beta_c,
+ *   z = phi(y), written over x_inout.
+ * x_inout   [N,C,H,W] in `d->layout`/`d->dtype`: x on entry, z on return.
+ * gamma, beta [C] float32 (gamma may be negative; it must be nonzero for the
+ *           backward to be defined).
+ * eps >= 0.
+ * save_mean, save_var [C] float32, written: the batch mean and the biased
+ *           variance; iabn_backward and iabn_update_running_stats take them.
+ * workspace, ws_bytes: scratch of at least iabn_workspace_size(d) bytes.
+ * stream:   cudaStream_t the work is ordered on. */
+iabn_status iabn_forward(const iabn_desc* d, void* x_inout,
+                         const float* gamma, const float* beta, float eps,
+                         int32_t act, float act_param,
+                         float* save_mean, float* save_var,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward from the stored output only ([ABN] section 3, "INPLACE-ABN" and
+ * "INPLACE-ABN II"; appendix "Derivation of Gradient dL").
+ *   y = phi^-1(z); dy = dz * phi'(y) (phi' read from z);
+ *   xhat = (y - beta_c)/gamma_c;  rstd = 1/sqrt(save_var_c + eps);
+ *   dbeta_c = sum dy,  dgamma_c = sum dy*xhat,
+ *   dx = gamma_c*rstd*(dy - dbeta_c/M - xhat*dgamma_c/M), written over dz.
+ * ELU inverse: with t = z/alpha, y = log1p(t) when 1 + t > 2^-24, else
+ *   y = ln(2^-24); its slope is max(z + alpha, 0).
+ * z         [N,C,H,W]: exactly the tensor iabn_forward produced (not modified).
+ * dz_inout  [N,C,H,W]: dL/dz on entry, dL/dx on return.  Must not alias z.
+ * gamma, beta, save_var, eps, act, act_param: as passed to / returned by the
+ *           forward call.
+ * dgamma, dbeta [C] float32: written (not accumulated).
+ * A channel with |gamma_c| < FLT_MIN gets NaN in dx, dgamma_c, dbeta_c and
+ * sets IABN_ERR_SINGULAR_GAMMA in the workspace status word. */
+iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz_inout,
+                          const float* gamma, const float* beta,
+                          const float* save_var, float eps,
+                          int32_t act, float act_param,
+                          float* dgamma, float* dbeta,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* Running statistics ([BN] Algorithm 2 uses the unbiased variance for
+ * inference; the momentum form is the usual framework convention):
+ *   running_mean <- (1 - momentum)*running_mean + momentum*save_mean,
+ *   running_var  <- (1 - momentum)*running_var + momentum*save_var*count/(count - 1).
+ * c: number of channels; count: M of the forward call (>= 2);
+ * momentum in [0, 1].  running_mean, running_var [C] float32, updated in place. */
+iabn_status iabn_update_running_stats(int64_t c, int64_t count,
+                                      const float* save_mean, const float* save_var,
+                                      float* running_mean, float* running_var,
+                                      float momentum, void* stream);
+
+/* Synchronises `stream`, reads the workspace's sticky device status and
+ * clears it (resetting the workspace's control block for reuse).  Returns
+ * IABN_OK, IABN_ERR_TIMEOUT, IABN_ERR_SINGULAR_GAMMA (the most severe
+ * condition seen since the last read), or IABN_ERR_CUDA if the stream or a
+ * copy failed. */
+iabn_status iabn_get_device_status(void* workspace, void* stream);
+
+/* Diagnostics: the number of kernels this library has launched in this
+ * process so far (all devices, all threads).  Host-only; never fails. */
+uint64_t iabn_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* IABN_H */

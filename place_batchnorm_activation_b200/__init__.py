@@ -1,0 +1,199 @@
+"""Python binding of libiabn.so -- In-Place Activated BatchNorm on B200.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels
+of libiabn.so (declared in include/iabn.h).  PyTorch is used for device
+memory and streams.  There is no CPU fallback: if the library is missing or
+no GPU is present, calls raise.
+
+Two levels:
+  * ``iabn_forward``, ``iabn_backward``, ``iabn_update_running_stats``,
+    ``iabn_workspace_size``, ``iabn_get_device_status``: the C entry points
+    with the same names and arguments (raw device pointers as ints).
+  * ``forward``, ``backward``, ``update_running_stats``, ``workspace_size``,
+    ``get_device_status``: the same calls taking torch tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libiabn.so")
+
+# enums of include/iabn.h
+IABN_OK = 0
+IABN_ERR_INVALID_ARG = 1
+IABN_ERR_UNSUPPORTED = 2
+IABN_ERR_MISALIGNED = 3
+IABN_ERR_WORKSPACE = 4
+IABN_ERR_CUDA = 5
+IABN_ERR_TIMEOUT = 6
+IABN_ERR_SINGULAR_GAMMA = 7
+STATUS_NAMES = {0: "IABN_OK", 1: "IABN_ERR_INVALID_ARG", 2: "IABN_ERR_UNSUPPORTED",
+                3: "IABN_ERR_MISALIGNED", 4: "IABN_ERR_WORKSPACE", 5: "IABN_ERR_CUDA",
+                6: "IABN_ERR_TIMEOUT", 7: "IABN_ERR_SINGULAR_GAMMA"}
+
+IABN_NCHW, IABN_NHWC = 0, 1
+IABN_F32, IABN_BF16, IABN_F16 = 0, 1, 2
+IABN_ACT_LEAKY_RELU, IABN_ACT_ELU, IABN_ACT_IDENTITY = 0, 1, 2
+
+# Symbols include/iabn.h declares (checked by the tests).
+EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_backward",
+           "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches")
+
+
+class IabnDesc(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("c", ctypes.c_int64), ("h", ctypes.c_int64),
+                ("w", ctypes.c_int64), ("layout", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class IabnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libiabn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "place_batchnorm_activation_b200._build.build()")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, f32, i32, i64 = ctypes.c_void_p, ctypes.c_float, ctypes.c_int32, ctypes.c_int64
+            pd = ctypes.POINTER(IabnDesc)
+            L.iabn_workspace_size.argtypes = [pd]
+            L.iabn_workspace_size.restype = ctypes.c_size_t
+            L.iabn_forward.argtypes = [pd, vp, vp, vp, f32, i32, f32, vp, vp, vp,
+                                       ctypes.c_size_t, vp]
+            L.iabn_forward.restype = i32
+            L.iabn_backward.argtypes = [pd, vp, vp, vp, vp, vp, f32, i32, f32, vp, vp, vp,
+                                        ctypes.c_size_t, vp]
+            L.iabn_backward.restype = i32
+            L.iabn_update_running_stats.argtypes = [i64, i64, vp, vp, vp, vp, f32, vp]
+            L.iabn_update_running_stats.restype = i32
+            L.iabn_get_device_status.argtypes = [vp, vp]
+            L.iabn_get_device_status.restype = i32
+            L.iabn_kernel_launches.argtypes = []
+            L.iabn_kernel_launches.restype = ctypes.c_uint64
+            _lib = L
+    return _lib
+
+
+def make_desc(shape, layout: int, dtype: int) -> IabnDesc:
+    n, c, h, w = (int(v) for v in shape)
+    return IabnDesc(n, c, h, w, int(layout), int(dtype))
+
+
+# -------------------------------------------------------------- raw C calls
+
+def iabn_workspace_size(desc: IabnDesc) -> int:
+    return int(lib().iabn_workspace_size(ctypes.byref(desc)))
+
+
+def iabn_forward(desc, x_inout, gamma, beta, eps, act, act_param, save_mean, save_var,
+                 workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_forward(ctypes.byref(desc), x_inout, gamma, beta, eps, act,
+                                  act_param, save_mean, save_var, workspace, ws_bytes, stream))
+
+
+def iabn_backward(desc, z, dz_inout, gamma, beta, save_var, eps, act, act_param, dgamma,
+                  dbeta, workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_backward(ctypes.byref(desc), z, dz_inout, gamma, beta, save_var,
+                                   eps, act, act_param, dgamma, dbeta, workspace, ws_bytes,
+                                   stream))
+
+
+def iabn_update_running_stats(c, count, save_mean, save_var, running_mean, running_var,
+                              momentum, stream) -> int:
+    return int(lib().iabn_update_running_stats(c, count, save_mean, save_var, running_mean,
+                                               running_var, momentum, stream))
+
+
+def iabn_get_device_status(workspace, stream) -> int:
+    return int(lib().iabn_get_device_status(workspace, stream))
+
+
+def iabn_kernel_launches() -> int:
+    return int(lib().iabn_kernel_launches())
+
+
+# ---------------------------------------------------------- tensor helpers
+
+def _dtype_code(t) -> int:
+    import torch
+    try:
+        return {torch.float32: IABN_F32, torch.bfloat16: IABN_BF16,
+                torch.float16: IABN_F16}[t.dtype]
+    except KeyError:
+        raise IabnError(IABN_ERR_INVALID_ARG, f"unsupported storage dtype {t.dtype}") from None
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    if not t.is_cuda:
+        raise IabnError(IABN_ERR_INVALID_ARG, "tensor is not on a CUDA device")
+    if not t.is_contiguous():
+        raise IabnError(IABN_ERR_INVALID_ARG, "tensor is not contiguous")
+    return int(t.data_ptr())
+
+
+def _ok(status: int, what: str) -> None:
+    if status != IABN_OK:
+        raise IabnError(status, what)
+
+
+def workspace_size(shape, layout: int, dtype: int) -> int:
+    return iabn_workspace_size(make_desc(shape, layout, dtype))
+
+
+def new_workspace(shape, layout: int, dtype: int, device=None):
+    """A zero-filled workspace tensor (uint8) for this descriptor."""
+    import torch
+    return torch.zeros(workspace_size(shape, layout, dtype), dtype=torch.uint8, device=device)
+
+
+def forward(x, gamma, beta, save_mean, save_var, workspace, *, shape, layout: int,
+            eps: float, act: int, act_param: float, stream=None) -> None:
+    """x (storage dtype, ``shape`` in ``layout``) is overwritten with z."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    _ok(iabn_forward(desc, _ptr(x), _ptr(gamma), _ptr(beta), float(eps), int(act),
+                     float(act_param), _ptr(save_mean), _ptr(save_var), _ptr(workspace),
+                     workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+        "iabn_forward")
+
+
+def backward(z, dz, gamma, beta, save_var, dgamma, dbeta, workspace, *, shape, layout: int,
+             eps: float, act: int, act_param: float, stream=None) -> None:
+    """dz is overwritten with dx; dgamma and dbeta are written."""
+    desc = make_desc(shape, layout, _dtype_code(z))
+    _ok(iabn_backward(desc, _ptr(z), _ptr(dz), _ptr(gamma), _ptr(beta), _ptr(save_var),
+                      float(eps), int(act), float(act_param), _ptr(dgamma), _ptr(dbeta),
+                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                      _stream_ptr(stream)), "iabn_backward")
+
+
+def update_running_stats(save_mean, save_var, running_mean, running_var, *, count: int,
+                         momentum: float, stream=None) -> None:
+    _ok(iabn_update_running_stats(save_mean.numel(), int(count), _ptr(save_mean),
+                                  _ptr(save_var), _ptr(running_mean), _ptr(running_var),
+                                  float(momentum), _stream_ptr(stream)),
+        "iabn_update_running_stats")
+
+
+def get_device_status(workspace, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the workspace's device status."""
+    return iabn_get_device_status(_ptr(workspace), _stream_ptr(stream))

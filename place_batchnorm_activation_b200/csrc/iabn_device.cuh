@@ -1,0 +1,202 @@
+// iabn_device.cuh -- device-side building blocks shared by the InPlace-ABN
+// kernels: storage types, the activation and its inverse, the workspace
+// control block, a bounded grid barrier and deterministic warp reductions.
+//
+// Method: "In-Place Activated BatchNorm for Memory-Optimized Training of
+// DNNs" (paperlayer.ai summary), section 3 "INPLACE-ABN" (invertible
+// activation and scale-and-shift) and section 4 "Experimental setup"
+// (leaky-ReLU slope 0.01).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace iabn {
+
+enum : int { kNCHW = 0, kNHWC = 1 };
+enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
+enum : int { kLeaky = 0, kElu = 1, kIdent = 2 };
+
+// Sticky status bits written by kernels into the workspace control block.
+constexpr uint32_t kStTimeout = 1u << 0;
+constexpr uint32_t kStSingular = 1u << 1;
+
+// First 256 bytes of every workspace.
+struct Control {
+    uint32_t status;     // sticky kSt* bits
+    uint32_t bar_count;  // grid-barrier arrivals in the current round (0 between rounds)
+    uint32_t bar_gen;    // grid-barrier generation, bumped once per completed round
+    uint32_t pad[61];
+};
+static_assert(sizeof(Control) == 256, "control block is 256 bytes");
+
+// Largest number of CTAs whose per-channel partials a workspace holds.
+constexpr int kMaxPartialBlocks = 256;
+
+// Default time budget of one bounded wait (grid barrier, mbarrier): 1 s.
+constexpr unsigned long long kWaitBudgetNs = 1000000000ull;
+
+// ------------------------------------------------------------ storage types
+
+template <int DT> struct Storage;
+template <> struct Storage<kF32> {
+    using T = float;
+    static __device__ __forceinline__ float load(const T* p) { return *p; }
+    static __device__ __forceinline__ void store(T* p, float v) { *p = v; }
+};
+template <> struct Storage<kBF16> {
+    using T = __nv_bfloat16;
+    static __device__ __forceinline__ float load(const T* p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void store(T* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+template <> struct Storage<kF16> {
+    using T = __half;
+    static __device__ __forceinline__ float load(const T* p) { return __half2float(*p); }
+    static __device__ __forceinline__ void store(T* p, float v) { *p = __float2half_rn(v); }
+};
+
+// ---------------------------------------------------------------- activation
+// phi and its inverse.  The positive branch is taken iff the argument is > 0,
+// so phi'(0) is the negative-branch slope.  For 16-bit storage the ELU uses
+// the fast exponential / logarithm intrinsics: their error (a few fp32 ulp)
+// is far below one storage ulp of z, which bounds what the inverse can
+// recover anyway.  For fp32 storage the accurate library functions are used.
+
+// ELU inverse floor: 1 + z/alpha is clamped at 2^-24, y = ln(2^-24).
+constexpr float kEluFloorU = 5.9604644775390625e-08f;   // 2^-24
+constexpr float kEluFloorY = -16.635532333438686f;      // ln(2^-24)
+
+template <int ACT, int DT>
+__device__ __forceinline__ float act_forward(float y, float p) {
+    if (ACT == kLeaky) return y > 0.f ? y : p * y;
+    if (ACT == kElu) {
+        if (y > 0.f) return y;
+        return DT == kF32 ? p * expm1f(y) : p * (__expf(y) - 1.f);
+    }
+    return y;
+}
+
+// From the stored z and the incoming dz: the pre-activation y and dy = dz*phi'(y).
+template <int ACT, int DT>
+__device__ __forceinline__ void act_backward(float z, float dz, float p, float inv_p,
+                                             float& y, float& dy) {
+    if (ACT == kLeaky) {
+        const bool pos = z > 0.f;
+        y = pos ? z : z * inv_p;
+        dy = pos ? dz : dz * p;
+    } else if (ACT == kElu) {
+        if (z > 0.f) {
+            y = z;
+            dy = dz;
+        } else {
+            const float t = z * inv_p;
+            const float u = 1.f + t;
+            if (u <= kEluFloorU) {
+                y = kEluFloorY;
+            } else {
+                y = DT == kF32 ? log1pf(t) : __logf(u);
+            }
+            dy = dz * fmaxf(z + p, 0.f);   // phi'(y) = alpha*e^y = z + alpha
+        }
+    } else {
+        y = z;
+        dy = dz;
+    }
+}
+
+// ------------------------------------------------------------ small helpers
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// Grid-wide barrier for a co-resident (cooperatively launched) grid, with a
+// time budget.  Central counter with a generation word: the last CTA to
+// arrive resets the counter and bumps the generation; the others wait for
+// the bump.  Returns false (after setting kStTimeout) if the budget ran out;
+// the caller must then skip the rest of its work.  Every thread of the CTA
+// must call it.
+__device__ __forceinline__ bool grid_barrier(Control* ctl, unsigned long long budget_ns) {
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        const uint32_t gen = ld_acquire_gpu(&ctl->bar_gen);
+        const uint32_t nblocks = gridDim.x * gridDim.y * gridDim.z;
+        __threadfence();
+        const uint32_t arrived = atom_add_acq_rel_gpu(&ctl->bar_count, 1u) + 1u;
+        if (arrived == nblocks) {
+            ctl->bar_count = 0u;
+            __threadfence();
+            st_release_gpu(&ctl->bar_gen, gen + 1u);
+        } else {
+            const unsigned long long t0 = global_ns();
+            unsigned int backoff = 32;
+            while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
+                if (global_ns() - t0 > budget_ns) {
+                    atomicOr(&ctl->status, kStTimeout);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(backoff);
+                if (backoff < 256) backoff <<= 1;
+            }
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+// Deterministic warp reductions (fixed shuffle-down tree; lane 0 holds the
+// result, which is then broadcast so every lane sees the same bits).
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+    return __shfl_sync(0xffffffffu, v, 0);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+    return __shfl_sync(0xffffffffu, v, 0);
+}
+
+// Chan et al. merge of two (count, mean, M2) summaries, in fp32.
+__device__ __forceinline__ void chan_merge(float& n, float& mean, float& m2,
+                                           float nb, float meanb, float m2b) {
+    const float nt = n + nb;
+    if (nb == 0.f) return;
+    if (n == 0.f) {
+        n = nb; mean = meanb; m2 = m2b;
+        return;
+    }
+    const float d = meanb - mean;
+    const float f = nb / nt;
+    mean = fmaf(d, f, mean);
+    m2 = m2 + m2b + d * d * n * f;
+    n = nt;
+}
+
+}  // namespace iabn

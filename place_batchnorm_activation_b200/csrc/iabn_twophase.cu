@@ -1,0 +1,477 @@
+// iabn_twophase.cu -- the split ("two-phase") plan of the InPlace-ABN layer:
+// separate launches for the per-block statistics, the per-channel finalize
+// and the elementwise apply.  It handles every shape, layout and alignment
+// and needs no co-resident grid; the resident plan (iabn_resident.cu) is the
+// fast path for the shapes it supports.
+//
+// Method: "In-Place Activated BatchNorm for Memory-Optimized Training of
+// DNNs" (paperlayer.ai summary), section 3: "Batch Normalization Review"
+// (per-channel batch mean and variance, gamma/beta), "INPLACE-ABN" (store
+// only z; invert the activation and the scale-and-shift in the backward),
+// "INPLACE-ABN II" (gradients in terms of y).
+//
+// Determinism: every reduction runs in a fixed order (fixed partition of the
+// rows/planes, fixed trees), so results are bitwise reproducible.
+#include "iabn_device.cuh"
+#include "iabn_internal.h"
+
+namespace iabn {
+
+// Partial-summary slots per channel of the NHWC split statistics.
+static inline int nhwc_row_blocks(int64_t R) {
+    return (int)(R < kMaxPartialBlocks ? R : kMaxPartialBlocks);
+}
+
+// ---------------------------------------------------------------- forward
+
+// NHWC: block (rb, cb) owns rows [rb*R/RB, (rb+1)*R/RB) and columns
+// [cb*W, cb*W + W).  Thread t reads column t % W of rows phase, phase + RP,
+// ... (coalesced along the channel dimension) with a running Welford update,
+// then the RP row phases of each column merge in a fixed tree.
+template <int DT>
+__global__ void __launch_bounds__(256)
+k_tp_stats_nhwc(const typename Storage<DT>::T* __restrict__ x, int64_t R, int64_t C, int RB,
+                double2* __restrict__ part) {
+    const int W = C < 256 ? (int)C : 256;
+    const int RP = 256 / W;
+    const int t = threadIdx.x;
+    const int lc = t % W, phase = t / W;
+    const int64_t col = (int64_t)blockIdx.y * W + lc;
+    const int64_t rb = blockIdx.x;
+    const int64_t r0 = rb * R / RB, r1 = (rb + 1) * R / RB;
+    float n = 0.f, mean = 0.f, m2 = 0.f;
+    if (phase < RP && col < C) {
+        for (int64_t r = r0 + phase; r < r1; r += RP) {
+            const float v = Storage<DT>::load(x + r * C + col);
+            n += 1.f;
+            const float d = v - mean;
+            mean += d / n;
+            m2 = fmaf(d, v - mean, m2);
+        }
+    }
+    __shared__ float sn[256], sm[256], sq[256];
+    sn[t] = n; sm[t] = mean; sq[t] = m2;
+    __syncthreads();
+    for (int s = 1; s < RP; s <<= 1) {
+        const bool act = phase < RP && (phase % (2 * s)) == 0 && phase + s < RP;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f;
+        if (act) {
+            a0 = sn[t]; a1 = sm[t]; a2 = sq[t];
+            const int o = t + s * W;
+            b0 = sn[o]; b1 = sm[o]; b2 = sq[o];
+            chan_merge(a0, a1, a2, b0, b1, b2);
+        }
+        __syncthreads();
+        if (act) { sn[t] = a0; sm[t] = a1; sq[t] = a2; }
+        __syncthreads();
+    }
+    if (phase == 0 && col < C) part[rb * C + col] = make_double2(sm[t], sq[t]);
+}
+
+// NCHW: one warp per (n, c) plane of HW contiguous values; lanes run Welford
+// over a strided share and merge in a fixed shuffle tree.  Partial slot of
+// plane (n, c) is n*C + c.
+template <int DT>
+__global__ void __launch_bounds__(256)
+k_tp_stats_nchw(const typename Storage<DT>::T* __restrict__ x, int64_t planes, int64_t HW,
+                double2* __restrict__ part) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t pl = gw; pl < planes; pl += nw) {
+        const typename Storage<DT>::T* src = x + pl * HW;
+        float n = 0.f, mean = 0.f, m2 = 0.f;
+        for (int64_t i = lane; i < HW; i += 32) {
+            const float v = Storage<DT>::load(src + i);
+            n += 1.f;
+            const float d = v - mean;
+            mean += d / n;
+            m2 = fmaf(d, v - mean, m2);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float b0 = __shfl_down_sync(0xffffffffu, n, o);
+            const float b1 = __shfl_down_sync(0xffffffffu, mean, o);
+            const float b2 = __shfl_down_sync(0xffffffffu, m2, o);
+            if (lane + o < 32) chan_merge(n, mean, m2, b0, b1, b2);
+        }
+        if (lane == 0) part[pl] = make_double2(mean, m2);
+    }
+}
+
+// Count of values behind partial k of a channel.
+__device__ __forceinline__ double partial_count(int layout, int64_t k, int64_t R, int RB,
+                                                int64_t HW) {
+    if (layout == kNHWC) return (double)((k + 1) * R / RB - k * R / RB);
+    return (double)HW;
+}
+
+// One warp per channel: combine the K partial summaries (count_k, mean_k,
+// M2_k) in fp64 with the parallel-axis identity
+//   mean = sum count_k mean_k / M,  M2 = sum (M2_k + count_k (mean_k - mean)^2),
+// then write the batch statistics and the apply coefficients.
+__global__ void __launch_bounds__(256)
+k_tp_finalize_fwd(const double2* __restrict__ part, int layout, int64_t C, int64_t K,
+                  int64_t R, int RB, int64_t HW, double M,
+                  const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                  float* __restrict__ save_mean, float* __restrict__ save_var,
+                  float4* __restrict__ coef) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t c = gw; c < C; c += nw) {
+        double s = 0.0;
+        for (int64_t k = lane; k < K; k += 32)
+            s += partial_count(layout, k, R, RB, HW) * part[k * C + c].x;
+        const double mean = warp_sum(s) / M;
+        double q = 0.0;
+        for (int64_t k = lane; k < K; k += 32) {
+            const double2 pk = part[k * C + c];
+            const double d = pk.x - mean;
+            q += pk.y + partial_count(layout, k, R, RB, HW) * d * d;
+        }
+        const double var = warp_sum(q) / M;
+        if (lane == 0) {
+            save_mean[c] = (float)mean;
+            save_var[c] = (float)var;
+            const double rstd = 1.0 / sqrt(var + (double)eps);
+            coef[c] = make_float4((float)mean, (float)((double)gamma[c] * rstd), beta[c], 0.f);
+        }
+    }
+}
+
+// Flat grid-stride apply; the channel of element i is tracked incrementally
+// (NHWC: i mod C; NCHW: (i div HW) mod C) so the loop has no division.
+template <int LAYOUT>
+struct ChannelWalker {
+    int64_t c, rem, sc, sr, sq, C, HW;
+    __device__ __forceinline__ void init(int64_t i, int64_t stride, int64_t C_, int64_t HW_) {
+        C = C_; HW = HW_;
+        if (LAYOUT == kNHWC) {
+            c = i % C; sc = stride % C;
+        } else {
+            rem = i % HW; c = (i / HW) % C; sr = stride % HW; sq = (stride / HW) % C;
+        }
+    }
+    __device__ __forceinline__ void advance() {
+        if (LAYOUT == kNHWC) {
+            c += sc;
+            if (c >= C) c -= C;
+        } else {
+            rem += sr;
+            int64_t carry = 0;
+            if (rem >= HW) { rem -= HW; carry = 1; }
+            c += sq + carry;
+            if (c >= C) c -= C;
+        }
+    }
+};
+
+template <int DT, int ACT, int LAYOUT>
+__global__ void __launch_bounds__(256)
+k_tp_apply_fwd(typename Storage<DT>::T* __restrict__ x, int64_t E, int64_t C, int64_t HW,
+               const float4* __restrict__ coef, float p) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= E) return;
+    ChannelWalker<LAYOUT> w;
+    w.init(i, stride, C, HW);
+    for (; i < E; i += stride) {
+        const float4 k = __ldg(coef + w.c);
+        const float v = Storage<DT>::load(x + i);
+        const float y = fmaf(v - k.x, k.y, k.z);
+        Storage<DT>::store(x + i, act_forward<ACT, DT>(y, p));
+        w.advance();
+    }
+}
+
+// --------------------------------------------------------------- backward
+
+// Per-channel sums S1 = sum dy and S2 = sum dy*xhat, xhat = (y - beta)/gamma
+// recovered from z.  Same partition and merge order as the statistics.
+template <int DT, int ACT>
+__global__ void __launch_bounds__(256)
+k_tp_reduce_nhwc(const typename Storage<DT>::T* __restrict__ z,
+                 const typename Storage<DT>::T* __restrict__ dz, int64_t R, int64_t C, int RB,
+                 const float* __restrict__ gamma, const float* __restrict__ beta, float p,
+                 float inv_p, double2* __restrict__ part) {
+    const int W = C < 256 ? (int)C : 256;
+    const int RP = 256 / W;
+    const int t = threadIdx.x;
+    const int lc = t % W, phase = t / W;
+    const int64_t col = (int64_t)blockIdx.y * W + lc;
+    const int64_t rb = blockIdx.x;
+    const int64_t r0 = rb * R / RB, r1 = (rb + 1) * R / RB;
+    float s1 = 0.f, s2 = 0.f;
+    if (phase < RP && col < C) {
+        const float ig = 1.f / gamma[col];
+        const float nb = -beta[col] * ig;
+        for (int64_t r = r0 + phase; r < r1; r += RP) {
+            const int64_t k = r * C + col;
+            float y, dy;
+            act_backward<ACT, DT>(Storage<DT>::load(z + k), Storage<DT>::load(dz + k), p, inv_p,
+                                  y, dy);
+            s1 += dy;
+            s2 = fmaf(dy, fmaf(y, ig, nb), s2);
+        }
+    }
+    __shared__ float a[256], b[256];
+    a[t] = s1; b[t] = s2;
+    __syncthreads();
+    for (int s = 1; s < RP; s <<= 1) {
+        const bool act = phase < RP && (phase % (2 * s)) == 0 && phase + s < RP;
+        float u = 0.f, v = 0.f;
+        if (act) { u = a[t] + a[t + s * W]; v = b[t] + b[t + s * W]; }
+        __syncthreads();
+        if (act) { a[t] = u; b[t] = v; }
+        __syncthreads();
+    }
+    if (phase == 0 && col < C) part[rb * C + col] = make_double2(a[t], b[t]);
+}
+
+template <int DT, int ACT>
+__global__ void __launch_bounds__(256)
+k_tp_reduce_nchw(const typename Storage<DT>::T* __restrict__ z,
+                 const typename Storage<DT>::T* __restrict__ dz, int64_t planes, int64_t C,
+                 int64_t HW, const float* __restrict__ gamma, const float* __restrict__ beta,
+                 float p, float inv_p, double2* __restrict__ part) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t pl = gw; pl < planes; pl += nw) {
+        const int64_t c = pl % C;
+        const float ig = 1.f / gamma[c];
+        const float nb = -beta[c] * ig;
+        float s1 = 0.f, s2 = 0.f;
+        for (int64_t i = lane; i < HW; i += 32) {
+            const int64_t k = pl * HW + i;
+            float y, dy;
+            act_backward<ACT, DT>(Storage<DT>::load(z + k), Storage<DT>::load(dz + k), p, inv_p,
+                                  y, dy);
+            s1 += dy;
+            s2 = fmaf(dy, fmaf(y, ig, nb), s2);
+        }
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        if (lane == 0) part[pl] = make_double2(s1, s2);
+    }
+}
+
+// One warp per channel: S1, S2 summed in fp64; dbeta = S1, dgamma = S2; the
+// apply coefficients express dx in terms of y (the "INPLACE-ABN II" form):
+//   dx = A*dy + B*y + Cc,  A = gamma*rstd,  B = -rstd*S2/M,
+//   Cc = -gamma*rstd*S1/M - B*beta.
+__global__ void __launch_bounds__(256)
+k_tp_finalize_bwd(const double2* __restrict__ part, int64_t C, int64_t K, double M,
+                  const float* __restrict__ gamma, const float* __restrict__ beta,
+                  const float* __restrict__ save_var, float eps, float* __restrict__ dgamma,
+                  float* __restrict__ dbeta, float4* __restrict__ coef,
+                  Control* __restrict__ ctl) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t c = gw; c < C; c += nw) {
+        double s1 = 0.0, s2 = 0.0;
+        for (int64_t k = lane; k < K; k += 32) {
+            const double2 pk = part[k * C + c];
+            s1 += pk.x;
+            s2 += pk.y;
+        }
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        if (lane == 0) {
+            const double g = gamma[c], b = beta[c];
+            const double rstd = 1.0 / sqrt((double)save_var[c] + (double)eps);
+            if (!(fabs(g) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN (or NaN)
+                atomicOr(&ctl->status, kStSingular);
+                dgamma[c] = __int_as_float(0x7fc00000);
+                dbeta[c] = __int_as_float(0x7fc00000);
+                coef[c] = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                      __int_as_float(0x7fc00000), 0.f);
+            } else {
+                dbeta[c] = (float)s1;
+                dgamma[c] = (float)s2;
+                const double A = g * rstd, B = -rstd * s2 / M;
+                const double Cc = -g * rstd * s1 / M - B * b;
+                coef[c] = make_float4((float)A, (float)B, (float)Cc, 0.f);
+            }
+        }
+    }
+}
+
+template <int DT, int ACT, int LAYOUT>
+__global__ void __launch_bounds__(256)
+k_tp_apply_bwd(const typename Storage<DT>::T* __restrict__ z, typename Storage<DT>::T* dz,
+               int64_t E, int64_t C, int64_t HW, const float4* __restrict__ coef, float p,
+               float inv_p) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= E) return;
+    ChannelWalker<LAYOUT> w;
+    w.init(i, stride, C, HW);
+    for (; i < E; i += stride) {
+        const float4 k = __ldg(coef + w.c);
+        float y, dy;
+        act_backward<ACT, DT>(Storage<DT>::load(z + i), Storage<DT>::load(dz + i), p, inv_p, y,
+                              dy);
+        Storage<DT>::store(dz + i, fmaf(k.x, dy, fmaf(k.y, y, k.z)));
+        w.advance();
+    }
+}
+
+// ------------------------------------------------------------ running stats
+
+__global__ void k_running_update(int64_t C, float unbias, const float* __restrict__ mean,
+                                 const float* __restrict__ var, float* __restrict__ rmean,
+                                 float* __restrict__ rvar, float m) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    rmean[c] = fmaf(m, mean[c], (1.f - m) * rmean[c]);
+    rvar[c] = fmaf(m, var[c] * unbias, (1.f - m) * rvar[c]);
+}
+
+// ------------------------------------------------------------ host launch
+
+static int grid_for(int64_t work, int per_block, int cap) {
+    int64_t g = (work + per_block - 1) / per_block;
+    if (g < 1) g = 1;
+    if (g > cap) g = cap;
+    return (int)g;
+}
+
+template <int DT, int ACT, int LAYOUT>
+static cudaError_t fwd_apply(const Geom& g, void* x, const float4* coef, float p,
+                             cudaStream_t s, int sms) {
+    using T = typename Storage<DT>::T;
+    k_tp_apply_fwd<DT, ACT, LAYOUT><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
+        static_cast<T*>(x), g.E, g.C, g.HW, coef, p);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <int DT>
+static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Workspace& w,
+                                   cudaStream_t s, int sms) {
+    using T = typename Storage<DT>::T;
+    const T* x = static_cast<const T*>(a.x);
+    int64_t K;
+    int RB = 1;
+    if (g.layout == kNHWC) {
+        RB = nhwc_row_blocks(g.R);
+        const int W = g.C < 256 ? (int)g.C : 256;
+        dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
+        k_tp_stats_nhwc<DT><<<grid, 256, 0, s>>>(x, g.R, g.C, RB, w.part);
+        K = RB;
+        count_launches(1);
+    } else {
+        const int64_t planes = g.N * g.C;
+        k_tp_stats_nchw<DT><<<grid_for(planes, 8, sms * 16), 256, 0, s>>>(x, planes, g.HW,
+                                                                          w.part);
+        K = g.N;
+        count_launches(1);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_tp_finalize_fwd<<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
+        w.part, g.layout, g.C, K, g.R, RB, g.HW, (double)g.M, a.gamma, a.beta, a.eps,
+        a.save_mean, a.save_var, w.coef);
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    void* xm = a.x;
+    const float p = a.act_param;
+    if (g.layout == kNHWC) {
+        switch (a.act) {
+        case kLeaky: return fwd_apply<DT, kLeaky, kNHWC>(g, xm, w.coef, p, s, sms);
+        case kElu: return fwd_apply<DT, kElu, kNHWC>(g, xm, w.coef, p, s, sms);
+        default: return fwd_apply<DT, kIdent, kNHWC>(g, xm, w.coef, p, s, sms);
+        }
+    }
+    switch (a.act) {
+    case kLeaky: return fwd_apply<DT, kLeaky, kNCHW>(g, xm, w.coef, p, s, sms);
+    case kElu: return fwd_apply<DT, kElu, kNCHW>(g, xm, w.coef, p, s, sms);
+    default: return fwd_apply<DT, kIdent, kNCHW>(g, xm, w.coef, p, s, sms);
+    }
+}
+
+cudaError_t forward_twophase(const Geom& g, const FwdArgs& a, const Workspace& w,
+                             cudaStream_t s, int sms) {
+    switch (g.dtype) {
+    case kF32: return fwd_twophase_dt<kF32>(g, a, w, s, sms);
+    case kBF16: return fwd_twophase_dt<kBF16>(g, a, w, s, sms);
+    default: return fwd_twophase_dt<kF16>(g, a, w, s, sms);
+    }
+}
+
+template <int DT, int ACT>
+static cudaError_t bwd_twophase_act(const Geom& g, const BwdArgs& a, const Workspace& w,
+                                    cudaStream_t s, int sms) {
+    using T = typename Storage<DT>::T;
+    const T* z = static_cast<const T*>(a.z);
+    T* dz = static_cast<T*>(a.dz);
+    const float p = a.act_param;
+    const float inv_p = ACT == kIdent ? 1.f : 1.f / p;
+    int64_t K;
+    if (g.layout == kNHWC) {
+        const int RB = nhwc_row_blocks(g.R);
+        const int W = g.C < 256 ? (int)g.C : 256;
+        dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
+        k_tp_reduce_nhwc<DT, ACT><<<grid, 256, 0, s>>>(z, dz, g.R, g.C, RB, a.gamma, a.beta, p,
+                                                       inv_p, w.part);
+        K = RB;
+        count_launches(1);
+    } else {
+        const int64_t planes = g.N * g.C;
+        k_tp_reduce_nchw<DT, ACT><<<grid_for(planes, 8, sms * 16), 256, 0, s>>>(
+            z, dz, planes, g.C, g.HW, a.gamma, a.beta, p, inv_p, w.part);
+        K = g.N;
+        count_launches(1);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_tp_finalize_bwd<<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
+        w.part, g.C, K, (double)g.M, a.gamma, a.beta, a.save_var, a.eps, a.dgamma, a.dbeta,
+        w.coef, w.ctl);
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int grid = grid_for(g.E, 256, sms * 8);
+    if (g.layout == kNHWC)
+        k_tp_apply_bwd<DT, ACT, kNHWC><<<grid, 256, 0, s>>>(z, dz, g.E, g.C, g.HW, w.coef, p,
+                                                            inv_p);
+    else
+        k_tp_apply_bwd<DT, ACT, kNCHW><<<grid, 256, 0, s>>>(z, dz, g.E, g.C, g.HW, w.coef, p,
+                                                            inv_p);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <int DT>
+static cudaError_t bwd_twophase_dt(const Geom& g, const BwdArgs& a, const Workspace& w,
+                                   cudaStream_t s, int sms) {
+    switch (a.act) {
+    case kLeaky: return bwd_twophase_act<DT, kLeaky>(g, a, w, s, sms);
+    case kElu: return bwd_twophase_act<DT, kElu>(g, a, w, s, sms);
+    default: return bwd_twophase_act<DT, kIdent>(g, a, w, s, sms);
+    }
+}
+
+cudaError_t backward_twophase(const Geom& g, const BwdArgs& a, const Workspace& w,
+                              cudaStream_t s, int sms) {
+    switch (g.dtype) {
+    case kF32: return bwd_twophase_dt<kF32>(g, a, w, s, sms);
+    case kBF16: return bwd_twophase_dt<kBF16>(g, a, w, s, sms);
+    default: return bwd_twophase_dt<kF16>(g, a, w, s, sms);
+    }
+}
+
+cudaError_t running_update(int64_t C, int64_t count, const float* mean, const float* var,
+                           float* rmean, float* rvar, float momentum, cudaStream_t s) {
+    const float unbias = (float)((double)count / (double)(count - 1));
+    k_running_update<<<(unsigned)((C + 255) / 256), 256, 0, s>>>(C, unbias, mean, var, rmean,
+                                                                  rvar, momentum);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace iabn

@@ -1,0 +1,168 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element, for every workload at full size and
+for edge shapes, under both launch plans.
+
+Forward: z (storage type), batch mean and biased variance.
+Backward (stage-separated): both sides start from the oracle's own rounded z
+and fp32 variance, so a one-ulp rounding flip in the forward is not blamed on
+the backward.  End to end: the GPU forward feeds the GPU backward; the
+oracle's chain feeds the oracle; same tolerance.
+Tolerances: fp32 rel 1e-5 / abs 1e-6; bf16, fp16 rel 2e-2 / abs 1e-2 (dx
+relative to the size of its terms, see gpu_util).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+from gpu_util import PLANS, TOL, GpuLayer, compare, forced_plan, oracle_expect, \
+    oracle_sweep_inputs
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+_cache = {}
+
+
+def expect_for(workload):
+    if workload not in _cache:
+        inp = wl.draw(wl.spec(workload))
+        _cache[workload] = (inp, oracle_expect(inp))
+    return _cache[workload]
+
+
+def check_layer(inp, exp, plan, *, running=False, e2e=True):
+    sp = inp.spec
+    tol = TOL[sp.dtype]
+    with forced_plan(plan):
+        L = GpuLayer(inp)
+        # forward
+        L.forward()
+        if running:
+            L.running()
+        torch.cuda.synchronize()
+        compare(L.host(L.x), exp["z"], sp.dtype, f"{sp.name} z")
+        compare(L.mean.cpu().numpy(), exp["mean"], tol, f"{sp.name} mean")
+        compare(L.var.cpu().numpy(), exp["var"], tol, f"{sp.name} var")
+        if running:
+            compare(L.rmean.cpu().numpy(), exp["running_mean"], tol, f"{sp.name} running_mean")
+            compare(L.rvar.cpu().numpy(), exp["running_var"], tol, f"{sp.name} running_var")
+        if e2e:
+            # end to end: GPU z and GPU variance feed the GPU backward
+            L.backward()
+            torch.cuda.synchronize()
+            compare(L.host(L.dz), exp["dx"], sp.dtype, f"{sp.name} e2e dx", exp["dx_scale"])
+            compare(L.dgamma.cpu().numpy(), exp["dgamma"], tol, f"{sp.name} e2e dgamma")
+            compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} e2e dbeta")
+        # stage-separated backward from the oracle's z and variance
+        z = L.load_z(exp["z"])
+        L.reset_dz()
+        var32 = torch.from_numpy(exp["var32"].astype(np.float32)).cuda()
+        L.backward(z=z, var=var32)
+        torch.cuda.synchronize()
+        compare(L.host(L.dz), exp["dx"], sp.dtype, f"{sp.name} dx", exp["dx_scale"])
+        compare(L.dgamma.cpu().numpy(), exp["dgamma"], tol, f"{sp.name} dgamma")
+        compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} dbeta")
+        # z is read-only for the backward
+        np.testing.assert_array_equal(L.host(L.x), exp["z"])
+        assert L.status() == 0
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("workload", [0, 1, 2, 3])
+def test_workload_parity(workload, plan):
+    inp, exp = expect_for(workload)
+    check_layer(inp, exp, plan, running=(workload == 1))
+
+
+@pytest.mark.parametrize("plan", PLANS)
+def test_layer_sweep_parity(plan):
+    """All 16 layers of the layer sweep (full size), each from the oracle's
+    chained input."""
+    for inp, exp in oracle_sweep_inputs():
+        check_layer(inp, exp, plan, e2e=False)
+
+
+EDGE = [
+    # (n, c, h, w, layout, dtype, act, param)
+    (3, 1, 5, 7, wl.NCHW, wl.F32, wl.LEAKY_RELU, 0.01),
+    (3, 1, 5, 7, wl.NHWC, wl.BF16, wl.ELU, 1.0),
+    (2, 3, 4, 5, wl.NHWC, wl.F32, wl.ELU, 0.5),
+    (2, 3, 4, 5, wl.NCHW, wl.F16, wl.LEAKY_RELU, 0.2),
+    (5, 6, 1, 1, wl.NCHW, wl.F32, wl.IDENTITY, 0.0),
+    (5, 6, 1, 1, wl.NHWC, wl.F16, wl.LEAKY_RELU, 0.01),
+    (1, 4, 1, 2, wl.NHWC, wl.F32, wl.LEAKY_RELU, 0.01),
+    (1, 4, 2, 1, wl.NCHW, wl.BF16, wl.ELU, 1.0),
+    (4, 12, 3, 3, wl.NHWC, wl.BF16, wl.LEAKY_RELU, 0.01),
+    (4, 12, 3, 3, wl.NCHW, wl.F32, wl.ELU, 1.0),
+    (2, 16, 7, 7, wl.NCHW, wl.F16, wl.ELU, 1.0),
+    (2, 16, 7, 7, wl.NHWC, wl.F32, wl.LEAKY_RELU, 0.01),
+    (7, 40, 9, 11, wl.NHWC, wl.F16, wl.ELU, 1.0),
+    (7, 40, 9, 11, wl.NCHW, wl.BF16, wl.LEAKY_RELU, 0.01),
+    (2, 300, 5, 5, wl.NHWC, wl.F32, wl.LEAKY_RELU, 0.01),
+    (2, 300, 5, 5, wl.NCHW, wl.F16, wl.IDENTITY, 0.0),
+    (1, 2, 1000, 37, wl.NCHW, wl.F32, wl.ELU, 1.0),
+    (1, 2, 1000, 37, wl.NHWC, wl.BF16, wl.LEAKY_RELU, 0.01),
+    (16, 24, 13, 13, wl.NHWC, wl.F32, wl.LEAKY_RELU, 0.01),
+    (16, 24, 13, 13, wl.NCHW, wl.F32, wl.ELU, 1.0),
+    (3, 8200, 2, 2, wl.NHWC, wl.BF16, wl.LEAKY_RELU, 0.01),
+    (32, 64, 31, 29, wl.NHWC, wl.F32, wl.ELU, 1.0),
+    (32, 64, 31, 29, wl.NCHW, wl.F32, wl.LEAKY_RELU, 0.01),
+]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("case", EDGE, ids=lambda c: "x".join(map(str, c[:4])) +
+                         f"-{'nhwc' if c[4] else 'nchw'}-{wl.DTYPE_NAMES[c[5]]}-"
+                         f"{wl.ACT_NAMES[c[6]]}")
+def test_edge_shapes(case, plan):
+    n, c, h, w, layout, dtype, act, p = case
+    sp = wl.LayerSpec("edge", n, c, h, w, layout, dtype, act, p, seed=777 + n * c + h * w)
+    inp = wl.draw(sp)
+    check_layer(inp, oracle_expect(inp), plan, running=True)
+
+
+@pytest.mark.parametrize("plan", PLANS)
+def test_deterministic(plan):
+    """Bitwise-identical outputs over repeated calls (fixed reduction order)."""
+    sp = wl.spec(1).with_(n=8)
+    inp = wl.draw(sp)
+    outs = []
+    with forced_plan(plan):
+        for _ in range(3):
+            L = GpuLayer(inp)
+            L.forward()
+            L.backward()
+            torch.cuda.synchronize()
+            outs.append([wl.torch_to_storage(L.x, sp.dtype), wl.torch_to_storage(L.dz, sp.dtype),
+                         L.mean.cpu().numpy(), L.var.cpu().numpy(), L.dgamma.cpu().numpy(),
+                         L.dbeta.cpu().numpy()])
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("plan", PLANS)
+def test_singular_gamma(plan):
+    sp = wl.LayerSpec("singular", 4, 6, 5, 5, wl.NHWC, wl.F32, wl.LEAKY_RELU, 0.01, seed=99)
+    inp = wl.draw(sp)
+    inp.gamma[2] = 0.0
+    exp = oracle_expect(inp)
+    with forced_plan(plan):
+        L = GpuLayer(inp)
+        L.forward()
+        torch.cuda.synchronize()
+        compare(L.host(L.x), exp["z"], sp.dtype, "z")
+        assert L.status() == 0
+        L.backward()
+        import place_batchnorm_activation_b200 as iabn
+        assert L.status() == iabn.IABN_ERR_SINGULAR_GAMMA
+        assert L.status() == 0          # read clears it
+        dx = wl.logical_view(L.host(L.dz), sp.shape, sp.layout)
+        assert np.isnan(dx[:, 2]).all()
+        assert np.isfinite(np.delete(dx, 2, axis=1)).all()
+        dg = L.dgamma.cpu().numpy()
+        assert np.isnan(dg[2]) and np.isfinite(np.delete(dg, 2)).all()
