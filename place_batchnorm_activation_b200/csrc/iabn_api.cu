@@ -4,10 +4,12 @@
 // Plan choice: the resident plan (one co-resident grid per call, data staged
 // through shared memory, grid-wide statistics) when the shape qualifies,
 // else the split two-phase plan.  IABN_FORCE_PLAN=twophase|resident in the
-// environment forces one (resident falls back to two-phase when the shape
-// does not qualify).
+// environment forces one (a shape the resident plan does not take still runs
+// two-phase; a resident launch that fails is then reported, not replaced).
+// IABN_DEBUG=1 prints CUDA errors to stderr.
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -114,7 +116,17 @@ static Plan forced_plan() {
 static iabn_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return IABN_OK;
     cudaGetLastError();   // clear a sticky launch error so later calls are not blamed
+    if (getenv("IABN_DEBUG")) fprintf(stderr, "iabn: CUDA error %d: %s\n", (int)e,
+                                      cudaGetErrorString(e));
     return IABN_ERR_CUDA;
+}
+
+// Launch-configuration errors after which nothing ran, so the two-phase plan
+// may run instead.
+static bool resident_declined(cudaError_t e) {
+    return e == cudaErrorNotSupported || e == cudaErrorCooperativeLaunchTooLarge ||
+           e == cudaErrorInvalidValue || e == cudaErrorLaunchOutOfResources ||
+           e == cudaErrorInvalidConfiguration;
 }
 
 }  // namespace iabn
@@ -148,8 +160,7 @@ extern "C" iabn_status iabn_forward(const iabn_desc* d, void* x_inout, const flo
     const Plan plan = forced_plan();
     if (plan != kTwoPhase && resident_supported(g)) {
         cudaError_t e = forward_resident(g, a, w, s);
-        if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge)
-            return from_cuda(e);
+        if (e == cudaSuccess || plan == kResident || !resident_declined(e)) return from_cuda(e);
         cudaGetLastError();
     }
     return from_cuda(forward_twophase(g, a, w, s, device_sms(dev)));
@@ -179,8 +190,7 @@ extern "C" iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz
     const Plan plan = forced_plan();
     if (plan != kTwoPhase && resident_supported(g)) {
         cudaError_t e = backward_resident(g, a, w, s);
-        if (e != cudaErrorNotSupported && e != cudaErrorCooperativeLaunchTooLarge)
-            return from_cuda(e);
+        if (e == cudaSuccess || plan == kResident || !resident_declined(e)) return from_cuda(e);
         cudaGetLastError();
     }
     return from_cuda(backward_twophase(g, a, w, s, device_sms(dev)));

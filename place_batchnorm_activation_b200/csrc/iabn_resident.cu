@@ -1,18 +1,206 @@
-// iabn_resident.cu -- resident plan (placeholder until the co-resident
-// kernels land): reports every shape as unsupported so the two-phase plan runs.
-#include "iabn_device.cuh"
-#include "iabn_internal.h"
+// iabn_resident.cu -- host side of the resident plan: which shapes qualify,
+// how a call is tiled over the SMs and their shared memory, and the launch.
+//
+// Shapes that qualify:
+//   NHWC: a row of C channels is a multiple of 16 bytes and at most 16 KiB
+//         (C % 8 == 0 and C <= 8192 for 16-bit storage; C % 4 == 0 and
+//         C <= 4096 for fp32).
+//   NCHW: with g = 16 / gcd(16, H*W*s) planes per unit every unit starts on a
+//         16-byte boundary; N*C must be a multiple of g and one unit must fit
+//         in 32 KiB.
+// Everything else runs the two-phase plan.
+//
+// Tuning knobs read from the environment (defaults in brackets):
+//   IABN_L2_HINTS [1]       L2 evict-last on tiles phase B reloads, evict-first
+//                           on the rest; 0 = no hints.
+//   IABN_TILE_KB  [16 / 8]  bytes per tensor per tile (forward / backward).
+//   IABN_RING     [5 / 4]   slots cycled by the stream (forward / backward).
+//   IABN_BARRIER_BUDGET_NS  [1e9] time budget of each bounded wait.
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "iabn_resident.cuh"
 
 namespace iabn {
 
-bool resident_supported(const Geom&) { return false; }
+namespace {
 
-cudaError_t forward_resident(const Geom&, const FwdArgs&, const Workspace&, cudaStream_t) {
-    return cudaErrorNotSupported;
+struct DeviceLimits {
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+DeviceLimits device_limits() {
+    static std::mutex mu;
+    static DeviceLimits cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceLimits{};
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceLimits& d = cache[dev];
+    if (d.sms == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            d.sms = v;
+        v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) ==
+            cudaSuccess)
+            d.smem_optin = v;
+    }
+    return d;
 }
 
-cudaError_t backward_resident(const Geom&, const BwdArgs&, const Workspace&, cudaStream_t) {
-    return cudaErrorNotSupported;
+long env_long(const char* name, long dflt) {
+    const char* s = getenv(name);
+    if (!s || !*s) return dflt;
+    char* end = nullptr;
+    const long v = strtol(s, &end, 10);
+    return (end && *end == 0) ? v : dflt;
+}
+
+int gcd_int(int64_t a, int64_t b) {
+    while (b) {
+        const int64_t t = a % b;
+        a = b;
+        b = t;
+    }
+    return (int)a;
+}
+
+int round_up_int(int v, int a) { return (v + a - 1) / a * a; }
+
+// Fills P for direction dir (0 forward, 1 backward); false if the shape does
+// not qualify or the device cannot hold the tiles.
+bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& cpt) {
+    if (dl.sms <= 0 || dl.smem_optin <= 0) return false;
+    const int s = g.esize;
+    const int NT = dir == 0 ? 1 : 2;
+    const int target = (int)env_long("IABN_TILE_KB", dir == 0 ? 16 : 8) * 1024;
+    if (target < 1024 || target > 65536) return false;
+    P = ResPlan{};
+    cpt = 1;
+    int scratch = 0;   // bytes of ring-slot scratch the per-CTA merge needs
+    if (g.layout == kNHWC) {
+        const int64_t rby = g.C * s;
+        if (rby % 16 != 0 || rby > 16384) return false;
+        P.VC = (int)(rby / 16);
+        cpt = P.VC > kResThreads ? 2 : 1;
+        P.RP = cpt == 1 ? kResThreads / P.VC : 1;
+        P.unit_bytes = (int)rby;
+        P.units = g.R;
+        int tr = target / (int)rby;
+        if (tr < 1) tr = 1;
+        if (P.RP > 1) tr = tr < P.RP ? P.RP : tr / P.RP * P.RP;
+        P.tile_units = tr;
+        P.g = 1;
+        P.L = 1;
+        if (cpt == 1 && P.RP > 1) scratch = kResThreads * (16 / s) * 8 + P.RP * 4;
+    } else {
+        const int64_t pb = g.HW * s;
+        const int gq = 16 / gcd_int(pb, 16);
+        if ((g.N * g.C) % gq != 0) return false;
+        if (gq * pb > 32768) return false;
+        if (g.HW > (1 << 30)) return false;
+        P.unit_bytes = (int)(gq * pb);
+        P.units = g.N * g.C / gq;
+        int tu = target / P.unit_bytes;
+        P.tile_units = tu < 1 ? 1 : tu;
+        P.g = gq;
+        int L = 1;
+        while (L < 32 && L * 8 < g.HW) L *= 2;
+        P.L = L;
+        P.VC = 1;
+        P.RP = 1;
+    }
+    P.tile_bytes = P.tile_units * P.unit_bytes;
+    P.half_bytes = round_up_int(P.tile_bytes, 128);
+    P.slot_bytes = P.half_bytes * NT;
+    const int budget = dl.smem_optin - 1024 - kBarBytes;
+    int nslots = budget / P.slot_bytes;
+    if (nslots > kMaxSlots) nslots = kMaxSlots;
+    int ring = (int)env_long("IABN_RING", dir == 0 ? 5 : 4);
+    if (ring < 3) ring = 3;
+    while (ring * P.slot_bytes < scratch) ++ring;
+    if (ring > nslots) return false;
+    P.nslots = nslots;
+    P.ring = ring;
+    P.smem_bytes = kBarBytes + nslots * P.slot_bytes;
+    P.G = (int)(P.units < dl.sms ? P.units : dl.sms);
+    if (P.G > kMaxPartialBlocks) P.G = kMaxPartialBlocks;
+    P.hints = env_long("IABN_L2_HINTS", 1) != 0 ? 1 : 0;
+    return true;
+}
+
+cudaError_t launch(const Geom& g, const ResArgs& a, int cpt, int act, int dir, int smem_optin,
+                   cudaStream_t s) {
+    switch (g.dtype) {
+    case kF32: return launch_resident_f32(a, g.layout, cpt, act, dir, smem_optin, s);
+    case kBF16: return launch_resident_bf16(a, g.layout, cpt, act, dir, smem_optin, s);
+    default: return launch_resident_f16(a, g.layout, cpt, act, dir, smem_optin, s);
+    }
+}
+
+ResArgs base_args(const Geom& g, const Workspace& w) {
+    ResArgs a;
+    a.N = g.N;
+    a.C = g.C;
+    a.HW = g.HW;
+    a.M = (double)g.M;
+    a.ctl = w.ctl;
+    a.part = w.part;
+    a.coef = w.coef;
+    const long b = env_long("IABN_BARRIER_BUDGET_NS", (long)kWaitBudgetNs);
+    a.budget_ns = b > 0 ? (unsigned long long)b : kWaitBudgetNs;
+    return a;
+}
+
+}  // namespace
+
+bool resident_supported(const Geom& g) {
+    const DeviceLimits dl = device_limits();
+    ResPlan P;
+    int cpt;
+    return make_plan(g, 0, dl, P, cpt) && make_plan(g, 1, dl, P, cpt);
+}
+
+cudaError_t forward_resident(const Geom& g, const FwdArgs& f, const Workspace& w,
+                             cudaStream_t s) {
+    const DeviceLimits dl = device_limits();
+    ResArgs a = base_args(g, w);
+    int cpt;
+    if (!make_plan(g, 0, dl, a.P, cpt)) return cudaErrorNotSupported;
+    a.src0 = static_cast<const unsigned char*>(f.x);
+    a.src1 = nullptr;
+    a.dst = static_cast<unsigned char*>(f.x);
+    a.gamma = f.gamma;
+    a.beta = f.beta;
+    a.var_in = nullptr;
+    a.out0 = f.save_mean;
+    a.out1 = f.save_var;
+    a.eps = f.eps;
+    a.p = f.act_param;
+    a.inv_p = f.act == kIdent ? 1.f : 1.f / f.act_param;
+    return launch(g, a, cpt, f.act, 0, dl.smem_optin, s);
+}
+
+cudaError_t backward_resident(const Geom& g, const BwdArgs& b, const Workspace& w,
+                              cudaStream_t s) {
+    const DeviceLimits dl = device_limits();
+    ResArgs a = base_args(g, w);
+    int cpt;
+    if (!make_plan(g, 1, dl, a.P, cpt)) return cudaErrorNotSupported;
+    a.src0 = static_cast<const unsigned char*>(b.z);
+    a.src1 = static_cast<const unsigned char*>(b.dz);
+    a.dst = static_cast<unsigned char*>(b.dz);
+    a.gamma = b.gamma;
+    a.beta = b.beta;
+    a.var_in = b.save_var;
+    a.out0 = b.dgamma;
+    a.out1 = b.dbeta;
+    a.eps = b.eps;
+    a.p = b.act_param;
+    a.inv_p = b.act == kIdent ? 1.f : 1.f / b.act_param;
+    return launch(g, a, cpt, b.act, 1, dl.smem_optin, s);
 }
 
 }  // namespace iabn

@@ -9,7 +9,11 @@ rms_c(dz)) is the size of the terms dx is the difference of
 (dx = gamma rstd (dy - mean dy - xhat mean(dy xhat))): with few values per
 channel those terms cancel almost completely (for M = 2, dx is
 eps/(var+eps) times them) and no fp32 evaluation can meet a bound relative
-to the tiny difference.
+to the tiny difference.  Likewise dgamma = sum dy*xhat and dbeta = sum dy
+are compared relative to max(|want|, sqrt(sum (dz*xhat)^2)) and
+max(|want|, sqrt(sum dz^2)) -- the root-sum-square of their terms (|phi'| <= 1)
+-- because a one-ulp difference in each stored z moves a near-cancelling sum
+by about that much times the storage rounding.
 """
 from __future__ import annotations
 
@@ -97,7 +101,7 @@ def oracle_expect(inp: wl.LayerInputs) -> dict:
     g = inp.gamma.astype(np.float64)
     b = inp.beta.astype(np.float64)
     eps, p = f32(sp.eps), f32(sp.act_param)
-    fw = oracle.forward(sp.shape, sp.layout, inp.x64, g, b, eps, sp.act, p)
+    fw = oracle.forward(sp.shape, sp.layout, inp.x64, g, b, eps, sp.act, p, want_xhat_y=True)
     z = oracle.round_to(fw["z"], sp.dtype)
     var32 = oracle.round_to(fw["var"], oracle.F32)
     bw = oracle.backward_inplace(sp.shape, sp.layout, z, inp.dz64, g, b, var32, eps, sp.act, p)
@@ -108,10 +112,13 @@ def oracle_expect(inp: wl.LayerInputs) -> dict:
     rms = np.sqrt((dzl ** 2).mean(axis=(0, 2, 3)))
     term = (np.abs(g) / np.sqrt(var32 + eps))[None, :, None, None] * (dzl + rms[None, :, None, None])
     dx_scale = wl._arrange(term, sp.layout)
+    xh = wl.logical_view(fw["xhat"], sp.shape, sp.layout)
+    dgamma_scale = np.sqrt(((dzl * xh) ** 2).sum(axis=(0, 2, 3)))
+    dbeta_scale = np.sqrt((dzl ** 2).sum(axis=(0, 2, 3)))
     return {"mean": fw["mean"], "var": fw["var"], "z": z, "var32": var32,
             "dx": oracle.round_to(bw["dx"], sp.dtype), "dx_scale": dx_scale,
-            "dgamma": bw["dgamma"], "dbeta": bw["dbeta"], "running_mean": rm,
-            "running_var": rv}
+            "dgamma": bw["dgamma"], "dbeta": bw["dbeta"], "dgamma_scale": dgamma_scale,
+            "dbeta_scale": dbeta_scale, "running_mean": rm, "running_var": rv}
 
 
 class GpuLayer:

@@ -55,8 +55,10 @@ def check_layer(inp, exp, plan, *, running=False, e2e=True):
             L.backward()
             torch.cuda.synchronize()
             compare(L.host(L.dz), exp["dx"], sp.dtype, f"{sp.name} e2e dx", exp["dx_scale"])
-            compare(L.dgamma.cpu().numpy(), exp["dgamma"], tol, f"{sp.name} e2e dgamma")
-            compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} e2e dbeta")
+            compare(L.dgamma.cpu().numpy(), exp["dgamma"], tol, f"{sp.name} e2e dgamma",
+                    exp["dgamma_scale"])
+            compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} e2e dbeta",
+                    exp["dbeta_scale"])
         # stage-separated backward from the oracle's z and variance
         z = L.load_z(exp["z"])
         L.reset_dz()
@@ -64,8 +66,9 @@ def check_layer(inp, exp, plan, *, running=False, e2e=True):
         L.backward(z=z, var=var32)
         torch.cuda.synchronize()
         compare(L.host(L.dz), exp["dx"], sp.dtype, f"{sp.name} dx", exp["dx_scale"])
-        compare(L.dgamma.cpu().numpy(), exp["dgamma"], tol, f"{sp.name} dgamma")
-        compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} dbeta")
+        compare(L.dgamma.cpu().numpy(), exp["dgamma"], tol, f"{sp.name} dgamma",
+                exp["dgamma_scale"])
+        compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} dbeta", exp["dbeta_scale"])
         # z is read-only for the backward
         np.testing.assert_array_equal(L.host(L.x), exp["z"])
         assert L.status() == 0
@@ -111,6 +114,11 @@ EDGE = [
     (3, 8200, 2, 2, wl.NHWC, wl.BF16, wl.LEAKY_RELU, 0.01),
     (32, 64, 31, 29, wl.NHWC, wl.F32, wl.ELU, 1.0),
     (32, 64, 31, 29, wl.NCHW, wl.F32, wl.LEAKY_RELU, 0.01),
+    (8, 8192, 3, 3, wl.NHWC, wl.BF16, wl.ELU, 1.0),
+    (8, 4096, 3, 3, wl.NHWC, wl.F32, wl.LEAKY_RELU, 0.01),
+    (8, 4104, 3, 3, wl.NHWC, wl.F16, wl.LEAKY_RELU, 0.01),
+    (2, 1024, 1, 1, wl.NHWC, wl.BF16, wl.IDENTITY, 0.0),
+    (64, 40, 3, 3, wl.NCHW, wl.F16, wl.ELU, 1.0),
 ]
 
 
