@@ -152,6 +152,29 @@ iabn_status iabn_get_device_status(void* workspace, void* stream);
  * process so far (all devices, all threads).  Host-only; never fails. */
 uint64_t iabn_kernel_launches(void);
 
+/* iabn_forward without a caller-supplied workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- e.g. a plugin inside a framework whose own allocator owns
+ * the GPU's memory, or a real-time loop that forbids allocation after
+ * start-up.  They still pass x_inout, gamma, beta, save_mean and save_var
+ * exactly as for iabn_forward; the scratch comes from an 8 MiB array of
+ * device memory that the library reserves on every GPU that loads it, held
+ * until the process exits.  No call allocates or frees memory.
+ *   - Descriptors whose iabn_workspace_size exceeds 8 MiB (8388608 bytes) are
+ *     rejected with IABN_ERR_WORKSPACE before anything is launched; other
+ *     argument errors are reported as by iabn_forward.
+ *   - The first call on a device (that device current) looks up the array's
+ *     device address; make that first call before any stream capture.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (other streams, other host threads) race and give wrong results.
+ *     Each call zeroes the array's control block on `stream` before its
+ *     kernels, so device-side conditions of one call (a bounded wait that ran
+ *     out) are not carried into the next and cannot be read back. */
+iabn_status iabn_forward_static_ws(const iabn_desc* d, void* x_inout,
+                                   const float* gamma, const float* beta, float eps,
+                                   int32_t act, float act_param,
+                                   float* save_mean, float* save_var, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

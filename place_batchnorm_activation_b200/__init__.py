@@ -40,7 +40,8 @@ IABN_ACT_LEAKY_RELU, IABN_ACT_ELU, IABN_ACT_IDENTITY = 0, 1, 2
 
 # Symbols include/iabn.h declares (checked by the tests).
 EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_backward",
-           "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches")
+           "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches",
+           "iabn_forward_static_ws")
 
 
 class IabnDesc(ctypes.Structure):
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
             L.iabn_get_device_status.restype = i32
             L.iabn_kernel_launches.argtypes = []
             L.iabn_kernel_launches.restype = ctypes.c_uint64
+            L.iabn_forward_static_ws.argtypes = [pd, vp, vp, vp, f32, i32, f32, vp, vp, vp]
+            L.iabn_forward_static_ws.restype = i32
             _lib = L
     return _lib
 
@@ -123,6 +126,14 @@ def iabn_get_device_status(workspace, stream) -> int:
 
 def iabn_kernel_launches() -> int:
     return int(lib().iabn_kernel_launches())
+
+
+def iabn_forward_static_ws(desc, x_inout, gamma, beta, eps, act, act_param, save_mean,
+                           save_var, stream) -> int:
+    """iabn_forward with the library's own fixed 8 MiB scratch (no workspace
+    argument) for callers that cannot allocate device memory."""
+    return int(lib().iabn_forward_static_ws(ctypes.byref(desc), x_inout, gamma, beta, eps, act,
+                                            act_param, save_mean, save_var, stream))
 
 
 # ---------------------------------------------------------- tensor helpers
