@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads and the CPU baseline")
+    ap.add_argument("--profile", type=int, default=0, metavar="WORKLOAD",
+                    help="profiling run: only `warmup` + `steps` fwd/bwd/running steps of "
+                         "workload 1, 2 or 3 (no e2e, extras or JSON line)")
     return ap.parse_args()
 
 
@@ -433,10 +436,55 @@ def run_reference(args):
 
 # ------------------------------------------------------------------- main
 
+def run_profile(args):
+    """Warm-up plus `steps` timed steps of one workload; prints per-call times."""
+    import torch
+    import workloads as wl
+    device = torch.device("cuda", 0)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device=device)
+    sp = wl.spec(args.profile)
+    layer = Layer(sp, sp.seed, device)
+    f, b, u, launches, _ = timed_layer_steps(layer, flush, args.steps, args.warmup)
+    print(f"profile {sp.name}: fwd_us={statistics.mean(f) * 1e3:.2f} "
+          f"bwd_us={statistics.mean(b) * 1e3:.2f} launches={launches}", flush=True)
+    if os.environ.get("IABN_TRACE") == "1":
+        # phase stamps of the resident kernels (see k_resident): per-CTA times
+        # relative to the earliest CTA start, median / min / max over CTAs (us)
+        names = ["start", "phaseA", "merge+prefetch", "barrier1", "finalize", "barrier2",
+                 "resident", "phaseB", "exit"]
+        for what, call in (("fwd", layer.fwd), ("bwd", layer.bwd)):
+            layer.restore()
+            flush.zero_()
+            if what == "bwd":
+                layer.fwd()
+                flush.zero_()
+                layer.ws[256:256 + 32768].zero_()
+            else:
+                layer.ws[256:256 + 32768].zero_()
+            call()
+            torch.cuda.synchronize()
+            tr = layer.ws[256:256 + 32768].view(torch.int64).view(256, 16).cpu()
+            rows = [r for r in tr.tolist() if r[0] != 0]
+            t0 = min(r[0] for r in rows)
+            parts = []
+            for k, nm in enumerate(names):
+                v = sorted((r[k] - t0) / 1e3 for r in rows)
+                parts.append(f"{nm}={v[len(v) // 2]:.1f}[{v[0]:.1f},{v[-1]:.1f}]")
+            for k, nm in ((9, "A.wait_kcyc"), (10, "A.work_kcyc"), (11, "B.wait_kcyc"),
+                          (12, "B.work_kcyc")):
+                v = sorted(r[k] / 1e3 for r in rows)
+                parts.append(f"{nm}={v[len(v) // 2]:.1f}")
+            print(f"trace {sp.name} {what} ({len(rows)} CTAs): " + " ".join(parts), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return run_profile(args)
     import torch
     import torch.distributed as dist
     import workloads as wl

@@ -33,7 +33,7 @@ int64_t partial_slots(const Geom& g) {
 static size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 static size_t workspace_bytes(const Geom& g) {
-    return round_up(sizeof(Control) + (size_t)partial_slots(g) * sizeof(double2) +
+    return round_up(sizeof(Control) + kTraceBytes + (size_t)partial_slots(g) * sizeof(double2) +
                         (size_t)g.C * sizeof(float4),
                     256);
 }
@@ -81,8 +81,9 @@ static Workspace carve(void* ws, const Geom& g) {
     Workspace w;
     char* base = static_cast<char*>(ws);
     w.ctl = reinterpret_cast<Control*>(base);
-    w.part = reinterpret_cast<double2*>(base + sizeof(Control));
-    w.coef = reinterpret_cast<float4*>(base + sizeof(Control) +
+    w.trace = reinterpret_cast<unsigned long long*>(base + sizeof(Control));
+    w.part = reinterpret_cast<double2*>(base + sizeof(Control) + kTraceBytes);
+    w.coef = reinterpret_cast<float4*>(base + sizeof(Control) + kTraceBytes +
                                        (size_t)partial_slots(g) * sizeof(double2));
     return w;
 }

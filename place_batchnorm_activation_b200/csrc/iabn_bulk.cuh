@@ -47,15 +47,66 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test for completion of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// try_wait with an explicit suspend-time hint (ns).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete, at most budget_ns.
+// mode 0: mbarrier.try_wait (the hardware may suspend the thread between
+// checks); mode 1: spin on the non-blocking test_wait; mode 2: try_wait with
+// a 32 ns suspend-time hint.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          unsigned long long budget_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+                                          unsigned long long budget_ns, int mode = 0) {
+    auto probe = [&]() -> bool {
+        if (mode == 1) return mbar_test_wait(bar, parity);
+        if (mode == 2) return mbar_try_wait_hint(bar, parity, 32u);
+        return mbar_try_wait(bar, parity);
+    };
+    if (probe()) return true;
     const unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > budget_ns) return false;
+    for (unsigned int k = 1;; ++k) {
+        if (probe()) return true;
+        // read the timer only every 64 polls
+        if ((k & 63u) == 0 && global_ns() - t0 > budget_ns) return false;
     }
-    return true;
+}
+
+// 16-byte shared-memory load / store at a 32-bit shared address.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -84,6 +135,23 @@ __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src_gmem, 
         " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst_smem)),
         "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
+}
+
+// The same without an L2 cache hint.
+__device__ __forceinline__ void bulk_load_plain(void* dst_smem, const void* src_gmem,
+                                                uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_store_plain(void* dst_gmem, const void* src_smem,
+                                                 uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst_gmem), "r"(smem_u32(src_smem)), "r"(bytes)
+                 : "memory");
 }
 
 // Shared -> global bulk copy, tracked by the issuing thread's bulk groups.

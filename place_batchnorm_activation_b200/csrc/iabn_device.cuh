@@ -35,6 +35,11 @@ static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 // Largest number of CTAs whose per-channel partials a workspace holds.
 constexpr int kMaxPartialBlocks = 256;
 
+// Optional phase trace (IABN_TRACE=1): %globaltimer stamps, kTraceSlots per
+// CTA, in the workspace right after the control block.
+constexpr int kTraceSlots = 16;
+constexpr size_t kTraceBytes = (size_t)kMaxPartialBlocks * kTraceSlots * 8;
+
 // Default time budget of one bounded wait (grid barrier, mbarrier): 1 s.
 constexpr unsigned long long kWaitBudgetNs = 1000000000ull;
 
@@ -134,14 +139,13 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v
 // Grid-wide barrier for a co-resident (cooperatively launched) grid, with a
 // time budget.  Central counter with a generation word: the last CTA to
 // arrive resets the counter and bumps the generation; the others wait for
-// the bump.  Returns false (after setting kStTimeout) if the budget ran out;
-// the caller must then skip the rest of its work.  Every thread of the CTA
-// must call it.
-__device__ __forceinline__ bool grid_barrier(Control* ctl, unsigned long long budget_ns) {
-    __shared__ int s_ok;
+// the bump.  *fail (shared memory) is the CTA's failure flag: a CTA that has
+// failed does not arrive; a wait that runs out sets *fail and kStTimeout.
+// Every thread of the CTA must call it; returns !*fail.
+__device__ __forceinline__ bool grid_barrier(Control* ctl, unsigned long long budget_ns,
+                                             int* fail) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int ok = 1;
+    if (threadIdx.x == 0 && *((volatile int*)fail) == 0) {
         const uint32_t gen = ld_acquire_gpu(&ctl->bar_gen);
         const uint32_t nblocks = gridDim.x * gridDim.y * gridDim.z;
         __threadfence();
@@ -152,21 +156,17 @@ __device__ __forceinline__ bool grid_barrier(Control* ctl, unsigned long long bu
             st_release_gpu(&ctl->bar_gen, gen + 1u);
         } else {
             const unsigned long long t0 = global_ns();
-            unsigned int backoff = 32;
             while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
                 if (global_ns() - t0 > budget_ns) {
                     atomicOr(&ctl->status, kStTimeout);
-                    ok = 0;
+                    *((volatile int*)fail) = 1;
                     break;
                 }
-                __nanosleep(backoff);
-                if (backoff < 256) backoff <<= 1;
             }
         }
-        s_ok = ok;
     }
     __syncthreads();
-    return s_ok != 0;
+    return *((volatile int*)fail) == 0;
 }
 
 // Deterministic warp reductions (fixed shuffle-down tree; lane 0 holds the

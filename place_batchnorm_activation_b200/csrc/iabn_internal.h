@@ -21,9 +21,10 @@ struct Geom {
     int esize;       // bytes per stored element
 };
 
-// Workspace carve-up: [Control | partials (double2) | coef (float4)].
+// Workspace carve-up: [Control | trace | partials (double2) | coef (float4)].
 struct Workspace {
     Control* ctl;
+    unsigned long long* trace;
     double2* part;
     float4* coef;
 };

@@ -13,9 +13,15 @@
 // Tuning knobs read from the environment (defaults in brackets):
 //   IABN_L2_HINTS [1]       L2 evict-last on tiles phase B reloads, evict-first
 //                           on the rest; 0 = no hints.
-//   IABN_TILE_KB  [16 / 8]  bytes per tensor per tile (forward / backward).
-//   IABN_RING     [5 / 4]   slots cycled by the stream (forward / backward).
+//   IABN_TILE_KB_FWD, IABN_TILE_KB_BWD [16, 8]  KiB per tensor per tile.
+//   IABN_RING_FWD, IABN_RING_BWD       [5, 5]   slots cycled by the stream.
 //   IABN_BARRIER_BUDGET_NS  [1e9] time budget of each bounded wait.
+//   IABN_WAIT_CONS, IABN_WAIT_PROD [0]  mbarrier wait mode of the consumer warps
+//                           and of the producer: 0 try_wait, 1 test_wait spin,
+//                           2 try_wait with a 32 ns suspend hint.
+//   IABN_TRACE    [0]       1: every CTA writes %globaltimer stamps at its phase
+//                           boundaries into the workspace (bytes 256 .. 256 +
+//                           32 KiB, [CTA][16] u64; see k_resident).
 #include <stdlib.h>
 
 #include <mutex>
@@ -75,17 +81,18 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     if (dl.sms <= 0 || dl.smem_optin <= 0) return false;
     const int s = g.esize;
     const int NT = dir == 0 ? 1 : 2;
-    const int target = (int)env_long("IABN_TILE_KB", dir == 0 ? 16 : 8) * 1024;
+    const int target =
+        (int)env_long(dir == 0 ? "IABN_TILE_KB_FWD" : "IABN_TILE_KB_BWD", dir == 0 ? 16 : 8) * 1024;
     if (target < 1024 || target > 65536) return false;
     P = ResPlan{};
     cpt = 1;
-    int scratch = 0;   // bytes of ring-slot scratch the per-CTA merge needs
+    int scratch = 0;   // bytes of shared memory the per-CTA merge needs
     if (g.layout == kNHWC) {
         const int64_t rby = g.C * s;
-        if (rby % 16 != 0 || rby > 16384) return false;
+        if (rby % 16 != 0 || rby > 16 * 4 * kConsumers) return false;
         P.VC = (int)(rby / 16);
-        cpt = P.VC > kResThreads ? 2 : 1;
-        P.RP = cpt == 1 ? kResThreads / P.VC : 1;
+        cpt = P.VC <= kConsumers ? 1 : (P.VC <= 2 * kConsumers ? 2 : 4);
+        P.RP = cpt == 1 ? kConsumers / P.VC : 1;
         P.unit_bytes = (int)rby;
         P.units = g.R;
         int tr = target / (int)rby;
@@ -94,7 +101,8 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         P.tile_units = tr;
         P.g = 1;
         P.L = 1;
-        if (cpt == 1 && P.RP > 1) scratch = kResThreads * (16 / s) * 8 + P.RP * 4;
+        // merge tree: ceil(RP/2) rows of VC columns of 16-byte float4 per pair
+        if (cpt == 1 && P.RP > 1) scratch = (P.RP + 1) / 2 * P.VC * (8 / s) * 16;
     } else {
         const int64_t pb = g.HW * s;
         const int gq = 16 / gcd_int(pb, 16);
@@ -115,16 +123,16 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     P.tile_bytes = P.tile_units * P.unit_bytes;
     P.half_bytes = round_up_int(P.tile_bytes, 128);
     P.slot_bytes = P.half_bytes * NT;
-    const int budget = dl.smem_optin - 1024 - kBarBytes;
+    P.scratch_bytes = round_up_int(scratch, 128);
+    const int budget = dl.smem_optin - 1024 - kBarBytes - P.scratch_bytes;
     int nslots = budget / P.slot_bytes;
     if (nslots > kMaxSlots) nslots = kMaxSlots;
-    int ring = (int)env_long("IABN_RING", dir == 0 ? 5 : 4);
-    if (ring < 3) ring = 3;
-    while (ring * P.slot_bytes < scratch) ++ring;
+    int ring = (int)env_long(dir == 0 ? "IABN_RING_FWD" : "IABN_RING_BWD", 5);
+    if (ring < 2) ring = 2;
     if (ring > nslots) return false;
     P.nslots = nslots;
     P.ring = ring;
-    P.smem_bytes = kBarBytes + nslots * P.slot_bytes;
+    P.smem_bytes = kBarBytes + P.scratch_bytes + nslots * P.slot_bytes;
     P.G = (int)(P.units < dl.sms ? P.units : dl.sms);
     if (P.G > kMaxPartialBlocks) P.G = kMaxPartialBlocks;
     P.hints = env_long("IABN_L2_HINTS", 1) != 0 ? 1 : 0;
@@ -149,8 +157,11 @@ ResArgs base_args(const Geom& g, const Workspace& w) {
     a.ctl = w.ctl;
     a.part = w.part;
     a.coef = w.coef;
+    a.trace = env_long("IABN_TRACE", 0) != 0 ? w.trace : nullptr;
     const long b = env_long("IABN_BARRIER_BUDGET_NS", (long)kWaitBudgetNs);
     a.budget_ns = b > 0 ? (unsigned long long)b : kWaitBudgetNs;
+    a.wait_cons = (int)env_long("IABN_WAIT_CONS", 0);
+    a.wait_prod = (int)env_long("IABN_WAIT_PROD", 0);
     return a;
 }
 

@@ -1,23 +1,28 @@
 // iabn_resident.cuh -- the resident plan of the InPlace-ABN layer: one
 // cooperative, persistent kernel per call (forward or backward), one CTA per
-// SM.
+// SM, warp-specialised.
 //
 // Each CTA owns a contiguous range of "units" (NHWC: rows of C channels;
 // NCHW: groups of g whole planes, g chosen so every unit starts on a 16-byte
-// boundary) and streams it through shared memory in tiles with the bulk-copy
-// engine (cp.async.bulk + mbarrier):
+// boundary) and streams it through shared-memory slots with the bulk-copy
+// engine.  One producer warp issues every bulk load and store; eight
+// consumer warps compute.  Slots are handed over with mbarriers (full: data
+// landed; empty: consumers done with a streamed tile; done: a rewritten tile
+// may be stored), so no consumer waits on a CTA-wide barrier per tile.
 //
-//   phase A  tiles 0..n-1: per-thread statistics (forward: Welford count,
-//            mean, M2; backward: sum dy and sum dy*xhat) from shared memory.
-//            The last D tiles land in dedicated slots and stay resident.
-//   merge    NHWC: the threads of a column merge in a fixed tree, one partial
-//            per (CTA, channel); NCHW: one partial per plane.
-//   barrier  grid-wide (bounded wait), then a distributed fp64 finalize (one
-//            warp per channel, fixed order), then a second grid barrier.
-//   phase B  tiles n-1..0 (reverse order): resident tiles are rewritten in
-//            place in shared memory; the others are fetched again -- the most
-//            recently read first, while they are still in L2 -- and written
-//            back with bulk stores.
+//   phase A  tiles 0..n-1: per-thread partial statistics from shared memory.
+//            Forward: pivot-shifted sums of x (pivot = the CTA's first row) or,
+//            NCHW, exact per-plane two-pass mean and M2.  Backward: sum dy and
+//            sum dy*y (the "INPLACE-ABN II" form; for leaky-ReLU dy*y = dz*z).
+//            The last D tiles land in dedicated slots and stay resident; as
+//            soon as a streamed slot frees, the producer prefetches phase B.
+//   merge    NHWC: the threads of a column add their sums in a fixed tree;
+//            one partial per (CTA, channel).  NCHW: one partial per plane.
+//   barrier  grid-wide (bounded wait), a distributed fp64 finalize (one warp
+//            per channel, fixed order), a second grid barrier.
+//   phase B  tiles n-1..0: resident tiles are rewritten in place first, then
+//            the streamed ones -- the most recently read first, while they are
+//            still in L2 -- and the producer writes each back with a bulk store.
 //
 // Method: "In-Place Activated BatchNorm for Memory-Optimized Training of
 // DNNs" (paperlayer.ai summary), section 3: "Batch Normalization Review",
@@ -31,10 +36,11 @@
 
 namespace iabn {
 
-constexpr int kResThreads = 512;
-constexpr int kResWarps = kResThreads / 32;
-constexpr int kMaxSlots = 30;
-constexpr int kBarBytes = 256;   // mbarrier area at the start of dynamic shared memory
+constexpr int kConsumers = 256;                  // consumer threads (8 warps)
+constexpr int kConsumerWarps = kConsumers / 32;
+constexpr int kResThreads = kConsumers + 32;     // + one producer warp
+constexpr int kMaxSlots = 32;
+constexpr int kBarBytes = 3 * kMaxSlots * 8;     // full[], empty[], done[] mbarriers
 
 struct ResPlan {
     int G;               // CTAs (at most one per SM)
@@ -46,6 +52,7 @@ struct ResPlan {
     int slot_bytes;      // half_bytes * tensors per tile
     int nslots;          // slots in shared memory
     int ring;            // slots cycled by the stream; the rest hold resident tiles
+    int scratch_bytes;   // shared memory for the per-CTA merge (NHWC), multiple of 128
     int smem_bytes;      // dynamic shared memory of the launch
     int VC, RP;          // NHWC: 16-byte columns per row; row phases (threads per column)
     int g, L;            // NCHW: planes per unit; lanes per plane
@@ -68,7 +75,10 @@ struct ResArgs {
     Control* ctl;
     double2* part;
     float4* coef;
+    unsigned long long* trace;   // null, or [G][kTraceSlots] phase stamps
     unsigned long long budget_ns;
+    int wait_cons;               // mbarrier wait mode of the consumers (see mbar_wait)
+    int wait_prod;               // mbarrier wait mode of the producer
 };
 
 // Sum over aligned groups of L lanes (L a power of two); every lane of the
@@ -78,19 +88,121 @@ __device__ __forceinline__ float group_sum(float v, int L) {
     return __shfl_sync(0xffffffffu, v, 0, L);
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 16 bytes <-> float2 pairs of consecutive elements.
+template <int DT> struct Pairs;
+template <> struct Pairs<kF32> {
+    static constexpr int NP = 2;
+    static __device__ __forceinline__ void unpack(const uint4& v, float2* f) {
+        f[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+        f[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+    }
+    static __device__ __forceinline__ uint4 pack(const float2* f) {
+        return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y),
+                          __float_as_uint(f[1].x), __float_as_uint(f[1].y));
+    }
+};
+template <> struct Pairs<kBF16> {
+    static constexpr int NP = 4;
+    static __device__ __forceinline__ float2 u(uint32_t w) {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    static __device__ __forceinline__ uint32_t p(float2 f) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(f.x, f.y);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    static __device__ __forceinline__ void unpack(const uint4& v, float2* f) {
+        f[0] = u(v.x); f[1] = u(v.y); f[2] = u(v.z); f[3] = u(v.w);
+    }
+    static __device__ __forceinline__ uint4 pack(const float2* f) {
+        return make_uint4(p(f[0]), p(f[1]), p(f[2]), p(f[3]));
+    }
+};
+template <> struct Pairs<kF16> {
+    static constexpr int NP = 4;
+    static __device__ __forceinline__ float2 u(uint32_t w) {
+        return __half22float2(*reinterpret_cast<__half2*>(&w));
+    }
+    static __device__ __forceinline__ uint32_t p(float2 f) {
+        __half2 h = __floats2half2_rn(f.x, f.y);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    static __device__ __forceinline__ void unpack(const uint4& v, float2* f) {
+        f[0] = u(v.x); f[1] = u(v.y); f[2] = u(v.z); f[3] = u(v.w);
+    }
+    static __device__ __forceinline__ uint4 pack(const float2* f) {
+        return make_uint4(p(f[0]), p(f[1]), p(f[2]), p(f[3]));
+    }
+};
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// Forward activation on a pair (leaky with slope <= 1 is max(y, a*y), with
+// slope > 1 it is min(y, a*y)).
+template <int ACT, int DT>
+__device__ __forceinline__ float2 act_forward2(float2 y, float p, bool slope_le1) {
+    if (ACT == kLeaky) {
+        const float2 t = __fmul2_rn(y, f2(p, p));
+        return slope_le1 ? f2(fmaxf(y.x, t.x), fmaxf(y.y, t.y))
+                         : f2(fminf(y.x, t.x), fminf(y.y, t.y));
+    }
+    if (ACT == kElu) return f2(act_forward<kElu, DT>(y.x, p), act_forward<kElu, DT>(y.y, p));
+    return y;
+}
+
 template <int DT, int ACT, int LAYOUT, int CPT, int DIR>
 __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     constexpr int NT = DIR == 0 ? 1 : 2;       // tensors per tile
-    constexpr int V = Vec<DT>::N;              // elements per 16-byte vector
-    constexpr int NV = CPT * V;                // channels per thread (NHWC)
+    constexpr int NP = Pairs<DT>::NP;          // channel pairs per 16-byte vector
+    constexpr int NQ = CPT * NP;               // channel pairs per thread (NHWC)
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned char* slots = smem + kBarBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxSlots;
+    uint64_t* done = empty + kMaxSlots;
+    __shared__ int s_fail;
 
     const ResPlan& P = a.P;
+    unsigned char* scratch = smem + kBarBytes;
+    unsigned char* slots = scratch + P.scratch_bytes;
     const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const bool producer = warp == kConsumerWarps;
     const int b = blockIdx.x;
     const int G = P.G;
+    // Phase trace: 0 start, 1 phase A done, 2 merged, 3 barrier 1, 4 finalize,
+    // 5 barrier 2, 6 resident tiles stored, 7 phase B stored, 8 stores complete
+    // (%globaltimer ns); 9/10/13 phase A and 11/12/15 phase B SM cycles of
+    // consumer warp 0: waiting for tiles / bookkeeping / the row loops.
+    auto stamp = [&](int k, bool who) {
+        if (a.trace != nullptr && who) a.trace[(size_t)b * kTraceSlots + k] = global_ns();
+    };
+    stamp(0, tid == 0);
+    // Consumer warp 0 also accounts its SM cycles: waiting for tiles vs the
+    // rest of the loop, per phase (trace slots 9..12).
+    const bool acct = a.trace != nullptr && tid == 0;
+    long long cyc_wait = 0, cyc_work = 0, cyc_comp = 0, cyc_mark = 0;
+    auto acct_start = [&]() { if (acct) cyc_mark = clock64(); };
+    auto acct_wait = [&]() {
+        if (acct) { const long long c = clock64(); cyc_wait += c - cyc_mark; cyc_mark = c; }
+    };
+    auto acct_work = [&]() {
+        if (acct) { const long long c = clock64(); cyc_work += c - cyc_mark; cyc_mark = c; }
+    };
+    auto acct_comp = [&]() {
+        if (acct) { const long long c = clock64(); cyc_comp += c - cyc_mark; cyc_mark = c; }
+    };
+    auto acct_flush = [&](int k) {
+        if (acct) {
+            a.trace[(size_t)b * kTraceSlots + k] = (unsigned long long)cyc_wait;
+            a.trace[(size_t)b * kTraceSlots + k + 1] = (unsigned long long)cyc_work;
+            a.trace[(size_t)b * kTraceSlots + k + 4] = (unsigned long long)cyc_comp;
+            cyc_wait = cyc_work = cyc_comp = 0;
+        }
+    };
+
     const int64_t u0 = (int64_t)b * P.units / G;
     const int64_t u1 = (int64_t)(b + 1) * P.units / G;
     const int n = (int)((u1 - u0 + P.tile_units - 1) / P.tile_units);
@@ -99,21 +211,15 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int nring = n - D;
 
     if (tid == 0) {
-        for (int s = 0; s < P.nslots; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < P.nslots; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+            mbar_init(&done[s], kConsumerWarps);
+        }
         mbar_init_fence();
+        s_fail = 0;
     }
     __syncthreads();
-
-    uint64_t pol_keep, pol_stream;
-    if (P.hints) {
-        pol_keep = policy_evict_last();
-        pol_stream = policy_evict_first();
-    } else {
-        pol_keep = pol_stream = policy_evict_normal();
-    }
-
-    uint32_t parity = 0;    // per-slot mbarrier phase (identical in every thread)
-    uint32_t pending = 0;   // slots with a load in flight (identical in every thread)
 
     auto t_u0 = [&](int t) -> int64_t { return u0 + (int64_t)t * P.tile_units; };
     auto t_nu = [&](int t) -> int {
@@ -122,27 +228,86 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     };
     auto slotA = [&](int t) -> int { return t < nring ? t % ring : ring + (t - nring); };
     auto slot_ptr = [&](int s) -> unsigned char* { return slots + (size_t)s * P.slot_bytes; };
-    // Thread 0 issues; every thread records the slot as pending.
-    auto issue = [&](int t, int s, uint64_t pol) {
-        if (tid == 0) {
-            const uint32_t bytes = (uint32_t)t_nu(t) * (uint32_t)P.unit_bytes;
-            const int64_t off = t_u0(t) * P.unit_bytes;
-            unsigned char* d = slot_ptr(s);
-            mbar_arrive_expect_tx(&bars[s], bytes * NT);
-            bulk_load(d, a.src0 + off, bytes, &bars[s], pol);
-            if (NT == 2) bulk_load(d + P.half_bytes, a.src1 + off, bytes, &bars[s], pol);
+    auto failed = [&]() -> bool { return *((volatile int*)&s_fail) != 0; };
+    auto set_failed = [&]() { *((volatile int*)&s_fail) = 1; };
+
+    // ================================================================ producer
+    // Lane 0 of the producer warp issues every bulk copy.
+    uint32_t fiss = 0;        // parity of the next load's full[] phase, per slot
+    uint32_t loaded = 0;      // slots that received at least one load
+    uint32_t epar = 0;        // next empty[] phase to wait for, per ring slot
+    uint32_t used = 0;        // ring slots holding a phase A tile not yet released
+    uint64_t pol_keep = 0, pol_stream = 0;
+    const bool pl = producer && lane == 0;
+    if (pl) {
+        if (P.hints) {
+            pol_keep = policy_evict_last();
+            pol_stream = policy_evict_first();
+        } else {
+            pol_keep = pol_stream = policy_evict_normal();
         }
-        pending |= 1u << s;
+    }
+    auto issue = [&](int t, int s, uint64_t pol) {
+        const uint32_t bytes = (uint32_t)t_nu(t) * (uint32_t)P.unit_bytes;
+        const int64_t off = t_u0(t) * P.unit_bytes;
+        unsigned char* d = slot_ptr(s);
+        mbar_arrive_expect_tx(&full[s], bytes * NT);
+        if (P.hints) {
+            bulk_load(d, a.src0 + off, bytes, &full[s], pol);
+            if (NT == 2) bulk_load(d + P.half_bytes, a.src1 + off, bytes, &full[s], pol);
+        } else {
+            bulk_load_plain(d, a.src0 + off, bytes, &full[s]);
+            if (NT == 2) bulk_load_plain(d + P.half_bytes, a.src1 + off, bytes, &full[s]);
+        }
+        fiss ^= 1u << s;
+        loaded |= 1u << s;
     };
-    auto wait = [&](int s) -> bool {
-        const bool ok = mbar_wait(&bars[s], (parity >> s) & 1u, a.budget_ns);
-        parity ^= 1u << s;
-        pending &= ~(1u << s);
+    // Waits until the consumers released ring slot s after its phase A tile.
+    auto wait_empty = [&](int s) -> bool {
+        if (!((used >> s) & 1u)) return true;
+        const bool ok = mbar_wait(&empty[s], (epar >> s) & 1u, a.budget_ns, a.wait_prod);
+        epar ^= 1u << s;
+        used &= ~(1u << s);
         return ok;
     };
+    if (pl) {
+        for (int t = 0; t < n && !failed(); ++t) {
+            const int s = slotA(t);
+            if (t < nring) {
+                if (!wait_empty(s)) { set_failed(); break; }
+                used |= 1u << s;
+            }
+            issue(t, s, t < nring ? pol_keep : pol_stream);
+        }
+        // Phase B prefetch into the streamed slots as they free up: the j-th
+        // streamed tile of phase B (tile nring-1-j) goes to slot j % ring.
+        const int pro = min(ring, nring);
+        for (int j = 0; j < pro && !failed(); ++j) {
+            if (!wait_empty(j)) { set_failed(); break; }
+            issue(nring - 1 - j, j, pol_stream);
+        }
+    }
 
-    // ---------------------------------------------------------- mapping
-    // NHWC: thread -> 16-byte column(s) and a row phase.
+    // ================================================================ consumers
+    uint32_t fpar = 0;   // consumers' next full[] phase parity, per slot
+    // Warp-uniform bounded wait for slot s: lane 0 polls the barrier, the warp
+    // then synchronises (ordering lane 0's acquire before the other lanes'
+    // reads of the slot).
+    auto cwait = [&](int s) -> bool {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&full[s], (fpar >> s) & 1u, a.budget_ns, a.wait_cons);
+        __syncwarp();
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        fpar ^= 1u << s;
+        if (!ok) set_failed();
+        return ok && !__any_sync(0xffffffffu, failed() ? 1 : 0);
+    };
+    auto release = [&](uint64_t* bar) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+    };
+
+    // NHWC mapping: consumer thread -> 16-byte column(s) and a row phase.
     int col[CPT];
     bool colok[CPT];
     int phase = 0;
@@ -151,262 +316,296 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         if (CPT == 1) {
             col[0] = tid % VC;
             phase = tid / VC;
-            colok[0] = phase < RP;
+            colok[0] = !producer && phase < RP;
         } else {
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
-                col[k] = tid + k * kResThreads;
-                colok[k] = col[k] < VC;
+                col[k] = tid + k * kConsumers;
+                colok[k] = !producer && col[k] < VC;
             }
         }
+    } else {
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+            col[k] = 0;
+            colok[k] = false;
+        }
     }
-    // NCHW: groups of L lanes per plane.
+    const bool active = LAYOUT == kNHWC && colok[0];
+    // byte offset of this thread's first 16-byte vector in a tile, and the
+    // stride between its rows
+    uint32_t voff[CPT];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) voff[k] = (uint32_t)(phase * RBY + col[k] * 16);
+    const uint32_t vstep = (uint32_t)(RP * RBY);
+    const uint32_t slots_sa = smem_u32(slots);
+    // rows of a tile with `rows` rows that this thread handles
+    auto my_rows = [&](int rows) -> int { return rows > phase ? (rows - 1 - phase) / RP + 1 : 0; };
+    // NCHW mapping: groups of L lanes per plane.
     const int L = P.L;
-    const int GP = kResThreads / L;
+    const int GP = kConsumers / L;
     const int grp = tid / L, glane = tid % L;
     const int HW = (int)a.HW;
     const int pbytes = HW * (int)sizeof(typename Storage<DT>::T);
     const float inv_hw = 1.f / (float)HW;
+    const float p = a.p, inv_p = a.inv_p;
+    const bool le1 = p <= 1.f;
 
-    // per-thread accumulators (NHWC): forward (cnt, mean, m2); backward (s1, s2)
-    float cnt = 0.f;
-    float acc0[NV], acc1[NV];
-    float kx[NV], ky[NV];   // backward: 1/gamma and -beta/gamma per channel
+    // NHWC accumulators: forward (sum d, sum d^2 with d = x - pivot); backward
+    // (sum dy, sum dy*y).
+    float2 acc0[NQ], acc1[NQ], piv[NQ];
 #pragma unroll
-    for (int j = 0; j < NV; ++j) { acc0[j] = 0.f; acc1[j] = 0.f; kx[j] = 0.f; ky[j] = 0.f; }
-    if (LAYOUT == kNHWC && DIR == 1) {
-#pragma unroll
-        for (int k = 0; k < CPT; ++k)
-            if (colok[k])
-#pragma unroll
-                for (int j = 0; j < V; ++j) {
-                    const int ch = col[k] * V + j;
-                    const float ig = 1.f / a.gamma[ch];
-                    kx[k * V + j] = ig;
-                    ky[k * V + j] = -a.beta[ch] * ig;
-                }
+    for (int q = 0; q < NQ; ++q) {
+        acc0[q] = f2(0.f, 0.f);
+        acc1[q] = f2(0.f, 0.f);
+        piv[q] = f2(0.f, 0.f);
     }
 
-    bool fail = false;
-
-    // ---------------------------------------------------------- phase A
-    {
-        const int pro = min(ring - 1, n);
-        for (int t = 0; t < pro; ++t) issue(t, slotA(t), t < nring ? pol_keep : pol_stream);
+    if (!producer) {
+        acct_start();
         for (int t = 0; t < n; ++t) {
-            const int tn = t + ring - 1;
-            if (tn < n) issue(tn, slotA(tn), tn < nring ? pol_keep : pol_stream);
             const int s = slotA(t);
-            const bool ok = wait(s);
-            if (ok) {
-                const unsigned char* base = slot_ptr(s);
-                if (LAYOUT == kNHWC) {
-                    const int rows = t_nu(t);
-                    if (CPT == 2 || colok[0]) {
-                        for (int r = phase; r < rows; r += RP) {
+            if (!cwait(s)) break;
+            acct_wait();
+            const unsigned char* base = slot_ptr(s);
+            if (LAYOUT == kNHWC) {
+                const int rows = t_nu(t);
+                if (active) {
+                    if (DIR == 0 && t == 0) {
+                        // pivot: the CTA's first row
+#pragma unroll
+                        for (int k = 0; k < CPT; ++k)
+                            if (colok[k]) {
+                                float2 f[NP];
+                                Pairs<DT>::unpack(
+                                    *reinterpret_cast<const uint4*>(base + col[k] * 16), f);
+#pragma unroll
+                                for (int q = 0; q < NP; ++q)
+                                    piv[k * NP + q] = f2(-f[q].x, -f[q].y);
+                            }
+                    }
+                    const int m = my_rows(rows);
+                    const uint32_t sb = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
+                    acct_work();
+#pragma unroll 2
+                    for (int i = 0; i < m; ++i) {
+#pragma unroll
+                        for (int k = 0; k < CPT; ++k) {
+                            if (CPT > 1 && !colok[k]) continue;
+                            const uint32_t o = sb + voff[k] + (uint32_t)i * vstep;
                             if (DIR == 0) {
-                                cnt += 1.f;
-                                const float inv = __fdividef(1.f, cnt);
+                                float2 f[NP];
+                                Pairs<DT>::unpack(lds128(o), f);
 #pragma unroll
-                                for (int k = 0; k < CPT; ++k) {
-                                    if (!colok[k]) continue;
-                                    const uint4 v = *reinterpret_cast<const uint4*>(
-                                        base + (size_t)r * RBY + col[k] * 16);
-                                    float f[V];
-                                    Vec<DT>::unpack(v, f);
-#pragma unroll
-                                    for (int j = 0; j < V; ++j) {
-                                        float& mu = acc0[k * V + j];
-                                        const float d = f[j] - mu;
-                                        mu = fmaf(d, inv, mu);
-                                        acc1[k * V + j] = fmaf(d, f[j] - mu, acc1[k * V + j]);
-                                    }
+                                for (int q = 0; q < NP; ++q) {
+                                    const int j = k * NP + q;
+                                    const float2 d = __fadd2_rn(f[q], piv[j]);
+                                    acc0[j] = __fadd2_rn(acc0[j], d);
+                                    acc1[j] = __ffma2_rn(d, d, acc1[j]);
                                 }
                             } else {
+                                float2 fz[NP], fd[NP];
+                                Pairs<DT>::unpack(lds128(o), fz);
+                                Pairs<DT>::unpack(lds128(o + (uint32_t)P.half_bytes), fd);
 #pragma unroll
-                                for (int k = 0; k < CPT; ++k) {
-                                    if (!colok[k]) continue;
-                                    const size_t o = (size_t)r * RBY + col[k] * 16;
-                                    const uint4 vz = *reinterpret_cast<const uint4*>(base + o);
-                                    const uint4 vd =
-                                        *reinterpret_cast<const uint4*>(base + P.half_bytes + o);
-                                    float fz[V], fd[V];
-                                    Vec<DT>::unpack(vz, fz);
-                                    Vec<DT>::unpack(vd, fd);
-#pragma unroll
-                                    for (int j = 0; j < V; ++j) {
-                                        float y, dy;
-                                        act_backward<ACT, DT>(fz[j], fd[j], a.p, a.inv_p, y, dy);
-                                        const int q = k * V + j;
-                                        acc0[q] += dy;
-                                        acc1[q] = fmaf(dy, fmaf(y, kx[q], ky[q]), acc1[q]);
+                                for (int q = 0; q < NP; ++q) {
+                                    const int j = k * NP + q;
+                                    if (ACT == kLeaky) {
+                                        // dy*y = dz*z on both branches
+                                        acc1[j] = __ffma2_rn(fd[q], fz[q], acc1[j]);
+                                        const float2 ad = __fmul2_rn(fd[q], f2(p, p));
+                                        const float2 dy = f2(fz[q].x > 0.f ? fd[q].x : ad.x,
+                                                             fz[q].y > 0.f ? fd[q].y : ad.y);
+                                        acc0[j] = __fadd2_rn(acc0[j], dy);
+                                    } else if (ACT == kIdent) {
+                                        acc1[j] = __ffma2_rn(fd[q], fz[q], acc1[j]);
+                                        acc0[j] = __fadd2_rn(acc0[j], fd[q]);
+                                    } else {
+                                        float y0, y1, d0, d1;
+                                        act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0, d0);
+                                        act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1, d1);
+                                        acc0[j] = __fadd2_rn(acc0[j], f2(d0, d1));
+                                        acc1[j] = __ffma2_rn(f2(d0, d1), f2(y0, y1), acc1[j]);
                                     }
                                 }
                             }
                         }
                     }
-                } else {
-                    // NCHW: one partial per plane
-                    const int np = t_nu(t) * P.g;
-                    const int64_t plane0 = t_u0(t) * P.g;
-                    for (int bp = 0; bp < np; bp += GP) {
-                        const int pp = bp + grp;
-                        const bool valid = pp < np;
-                        const unsigned char* pz = base + (size_t)pp * pbytes;
-                        if (DIR == 0) {
-                            float sum = 0.f;
-                            if (valid)
-                                for (int i = glane; i < HW; i += L) sum += Elem<DT>::ld(pz, i);
-                            const float mean = group_sum(sum, L) * inv_hw;
-                            float sq = 0.f;
-                            if (valid)
-                                for (int i = glane; i < HW; i += L) {
-                                    const float d = Elem<DT>::ld(pz, i) - mean;
-                                    sq = fmaf(d, d, sq);
-                                }
-                            sq = group_sum(sq, L);
-                            if (valid && glane == 0) a.part[plane0 + pp] = make_double2(mean, sq);
-                        } else {
-                            float s1 = 0.f, s2 = 0.f;
-                            if (valid) {
-                                const int c = (int)((uint64_t)(plane0 + pp) % (uint64_t)a.C);
-                                const float ig = 1.f / __ldg(a.gamma + c);
-                                const float nb = -__ldg(a.beta + c) * ig;
-                                const unsigned char* pd = pz + P.half_bytes;
-                                for (int i = glane; i < HW; i += L) {
-                                    float y, dy;
-                                    act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i),
-                                                          a.p, a.inv_p, y, dy);
-                                    s1 += dy;
-                                    s2 = fmaf(dy, fmaf(y, ig, nb), s2);
-                                }
+                    acct_comp();
+                }
+            } else {
+                // NCHW: one partial per plane
+                const int np = t_nu(t) * P.g;
+                const int64_t plane0 = t_u0(t) * P.g;
+                for (int bp = 0; bp < np; bp += GP) {
+                    const int pp = bp + grp;
+                    const bool valid = pp < np;
+                    const unsigned char* pz = base + (size_t)pp * pbytes;
+                    if (DIR == 0) {
+                        float sum = 0.f;
+                        if (valid)
+                            for (int i = glane; i < HW; i += L) sum += Elem<DT>::ld(pz, i);
+                        const float mean = group_sum(sum, L) * inv_hw;
+                        float sq = 0.f;
+                        if (valid)
+                            for (int i = glane; i < HW; i += L) {
+                                const float d = Elem<DT>::ld(pz, i) - mean;
+                                sq = fmaf(d, d, sq);
                             }
-                            s1 = group_sum(s1, L);
-                            s2 = group_sum(s2, L);
-                            if (valid && glane == 0) a.part[plane0 + pp] = make_double2(s1, s2);
+                        sq = group_sum(sq, L);
+                        if (valid && glane == 0) a.part[plane0 + pp] = make_double2(mean, sq);
+                    } else {
+                        float s1 = 0.f, sy = 0.f;
+                        if (valid) {
+                            const unsigned char* pd = pz + P.half_bytes;
+                            for (int i = glane; i < HW; i += L) {
+                                float y, dy;
+                                act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
+                                                      inv_p, y, dy);
+                                s1 += dy;
+                                sy = fmaf(dy, y, sy);
+                            }
                         }
+                        s1 = group_sum(s1, L);
+                        sy = group_sum(sy, L);
+                        if (valid && glane == 0) a.part[plane0 + pp] = make_double2(s1, sy);
                     }
                 }
             }
-            if (__syncthreads_or(!ok)) {
-                fail = true;
-                break;
-            }
+            if (t < nring) release(&empty[s]);
+            acct_work();
         }
+        acct_flush(9);
     }
+    __syncthreads();
+    stamp(1, tid == 0);
 
     // ------------------------------------------- per-CTA merge (NHWC)
-    if (!fail && LAYOUT == kNHWC) {
+    if (!failed() && LAYOUT == kNHWC) {
         if (CPT == 1 && RP > 1) {
-            // Scratch in the ring slots (no load is in flight there now).
-            float2* scr = reinterpret_cast<float2*>(slots);          // [RP][VC][V]
-            float* scnt = reinterpret_cast<float*>(slots + (size_t)kResThreads * V * 8);
-            if (colok[0]) {
-#pragma unroll
-                for (int j = 0; j < V; ++j)
-                    scr[((size_t)phase * VC + col[0]) * V + j] = make_float2(acc0[j], acc1[j]);
-                if (col[0] == 0) scnt[phase] = cnt;
-            }
+            // Fixed tree over row phases: in round st the phases p with
+            // p % 2st == st write their sums, those with p % 2st == 0 add them.
+            float4* scr = reinterpret_cast<float4*>(scratch);   // [ceil(RP/2)][VC][NP]
             for (int st = 1; st < RP; st <<= 1) {
+                const bool writer = colok[0] && (phase % (2 * st)) == st;
+                const bool reader = colok[0] && (phase % (2 * st)) == 0 && phase + st < RP;
+                const size_t row = (size_t)(phase / (2 * st)) * VC + col[0];
+                if (writer) {
+#pragma unroll
+                    for (int q = 0; q < NP; ++q)
+                        scr[row * NP + q] = make_float4(acc0[q].x, acc0[q].y, acc1[q].x, acc1[q].y);
+                }
                 __syncthreads();
-                const bool act = colok[0] && (phase % (2 * st)) == 0 && phase + st < RP;
-                if (act) {
-                    const int o = phase + st;
-                    if (DIR == 0) {
-                        const float na = cnt, nb = scnt[o], nt = na + nb;
-                        if (nb > 0.f) {
-                            const float f = na > 0.f ? nb / nt : 1.f;
+                if (reader) {
 #pragma unroll
-                            for (int j = 0; j < V; ++j) {
-                                const float2 q = scr[((size_t)o * VC + col[0]) * V + j];
-                                const float d = q.x - acc0[j];
-                                acc0[j] = fmaf(d, f, acc0[j]);
-                                acc1[j] = acc1[j] + q.y + d * d * na * f;
-                            }
-                            cnt = nt;
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < V; ++j) {
-                            const float2 q = scr[((size_t)o * VC + col[0]) * V + j];
-                            acc0[j] += q.x;
-                            acc1[j] += q.y;
-                        }
+                    for (int q = 0; q < NP; ++q) {
+                        const float4 v = scr[row * NP + q];
+                        acc0[q] = __fadd2_rn(acc0[q], f2(v.x, v.y));
+                        acc1[q] = __fadd2_rn(acc1[q], f2(v.z, v.w));
                     }
                 }
                 __syncthreads();
-                if (act) {
-#pragma unroll
-                    for (int j = 0; j < V; ++j)
-                        scr[((size_t)phase * VC + col[0]) * V + j] = make_float2(acc0[j], acc1[j]);
-                    if (col[0] == 0) scnt[phase] = cnt;
-                }
             }
-            __syncthreads();
         }
-        if (phase == 0) {
+        if (active && phase == 0) {
+            const double nb = (double)(u1 - u0);
 #pragma unroll
             for (int k = 0; k < CPT; ++k)
                 if (colok[k])
 #pragma unroll
-                    for (int j = 0; j < V; ++j)
-                        a.part[(int64_t)b * a.C + col[k] * V + j] =
-                            make_double2(acc0[k * V + j], acc1[k * V + j]);
+                    for (int q = 0; q < NP; ++q) {
+                        const int64_t ch = (int64_t)(col[k] * NP + q) * 2;
+                        const int i = k * NP + q;
+                        double2* dstp = a.part + (int64_t)b * a.C + ch;
+                        if (DIR == 0) {
+                            // (mean, M2) of the CTA from its pivot-shifted sums
+                            const double s1x = acc0[i].x, s1y = acc0[i].y;
+                            dstp[0] = make_double2(-(double)piv[i].x + s1x / nb,
+                                                   (double)acc1[i].x - s1x * s1x / nb);
+                            dstp[1] = make_double2(-(double)piv[i].y + s1y / nb,
+                                                   (double)acc1[i].y - s1y * s1y / nb);
+                        } else {
+                            dstp[0] = make_double2(acc0[i].x, acc1[i].x);
+                            dstp[1] = make_double2(acc0[i].y, acc1[i].y);
+                        }
+                    }
         }
-        __syncthreads();   // scratch reads done before the ring slots are reloaded
     }
+    stamp(2, tid == 0);
 
-    // ------------------------------------- prefetch phase B, then barriers
-    // Phase B order: resident tiles n-1..nring, then ring tiles nring-1..0;
-    // the j-th ring tile of phase B (tile nring-1-j) uses ring slot j % ring.
-    const int depthB = max(1, ring - 2);
-    if (!fail) {
-        const int pro = min(depthB, nring);
-        for (int j = 0; j < pro; ++j) issue(nring - 1 - j, j % ring, pol_stream);
-    }
-    if (!fail && !grid_barrier(a.ctl, a.budget_ns)) fail = true;
-
-    // finalize: one warp per channel over the whole grid, fp64, fixed order
-    if (!fail) {
-        const int wid = tid >> 5, lane = tid & 31;
-        const int64_t nw = (int64_t)G * kResWarps;
+    // ------------------------------------------------- barriers and finalize
+    grid_barrier(a.ctl, a.budget_ns, &s_fail);
+    stamp(3, tid == 0);
+    if (!failed() && !producer) {
+        // one consumer warp per channel over the whole grid, fp64, fixed order
+        const int64_t nw = (int64_t)G * kConsumerWarps;
         const int64_t K = LAYOUT == kNHWC ? (int64_t)G : a.N;
-        for (int64_t c = (int64_t)b * kResWarps + wid; c < a.C; c += nw) {
+        constexpr int KC = 5;   // partials cached per lane when K <= 160
+        const bool cached = K <= 32 * KC;
+        auto count_at = [&](int64_t k) -> double {
+            return LAYOUT == kNHWC ? (double)((k + 1) * P.units / G - k * P.units / G)
+                                   : (double)a.HW;
+        };
+        for (int64_t c = (int64_t)b * kConsumerWarps + warp; c < a.C; c += nw) {
+            double2 pk[KC];
+            double ck[KC];
+#pragma unroll
+            for (int i = 0; i < KC; ++i) {
+                const int64_t k = lane + 32 * i;
+                const bool in = cached && k < K;
+                pk[i] = in ? a.part[k * a.C + c] : make_double2(0.0, 0.0);
+                ck[i] = in ? count_at(k) : 0.0;
+            }
             if (DIR == 0) {
                 double s = 0.0;
-                for (int64_t k = lane; k < K; k += 32) {
-                    const double cntk = LAYOUT == kNHWC
-                                            ? (double)((k + 1) * P.units / G - k * P.units / G)
-                                            : (double)a.HW;
-                    s += cntk * a.part[k * a.C + c].x;
+                if (cached) {
+#pragma unroll
+                    for (int i = 0; i < KC; ++i) s += ck[i] * pk[i].x;
+                } else {
+                    for (int64_t k = lane; k < K; k += 32) s += count_at(k) * a.part[k * a.C + c].x;
                 }
                 const double mean = warp_sum(s) / a.M;
                 double q = 0.0;
-                for (int64_t k = lane; k < K; k += 32) {
-                    const double cntk = LAYOUT == kNHWC
-                                            ? (double)((k + 1) * P.units / G - k * P.units / G)
-                                            : (double)a.HW;
-                    const double2 pk = a.part[k * a.C + c];
-                    const double d = pk.x - mean;
-                    q += pk.y + cntk * d * d;
+                if (cached) {
+#pragma unroll
+                    for (int i = 0; i < KC; ++i) {
+                        const double d = pk[i].x - mean;
+                        q += pk[i].y + ck[i] * d * d;
+                    }
+                } else {
+                    for (int64_t k = lane; k < K; k += 32) {
+                        const double2 v = a.part[k * a.C + c];
+                        const double d = v.x - mean;
+                        q += v.y + count_at(k) * d * d;
+                    }
                 }
                 const double var = warp_sum(q) / a.M;
                 if (lane == 0) {
                     a.out0[c] = (float)mean;
                     a.out1[c] = (float)var;
                     const double rstd = 1.0 / sqrt(var + (double)a.eps);
-                    a.coef[c] = make_float4((float)mean, (float)((double)a.gamma[c] * rstd),
-                                            a.beta[c], 0.f);
+                    const double sc = (double)a.gamma[c] * rstd;
+                    // (mean, scale, beta, beta - mean*scale)
+                    a.coef[c] = make_float4((float)mean, (float)sc, a.beta[c],
+                                            (float)((double)a.beta[c] - mean * sc));
                 }
             } else {
-                double s1 = 0.0, s2 = 0.0;
-                for (int64_t k = lane; k < K; k += 32) {
-                    const double2 pk = a.part[k * a.C + c];
-                    s1 += pk.x;
-                    s2 += pk.y;
+                double s1 = 0.0, sy = 0.0;
+                if (cached) {
+#pragma unroll
+                    for (int i = 0; i < KC; ++i) {
+                        s1 += pk[i].x;
+                        sy += pk[i].y;
+                    }
+                } else {
+                    for (int64_t k = lane; k < K; k += 32) {
+                        const double2 v = a.part[k * a.C + c];
+                        s1 += v.x;
+                        sy += v.y;
+                    }
                 }
                 s1 = warp_sum(s1);
-                s2 = warp_sum(s2);
+                sy = warp_sum(sy);
                 if (lane == 0) {
                     const double gm = a.gamma[c], bt = a.beta[c];
                     const double rstd = 1.0 / sqrt((double)a.var_in[c] + (double)a.eps);
@@ -417,9 +616,12 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         a.out1[c] = qnan;
                         a.coef[c] = make_float4(qnan, qnan, qnan, 0.f);
                     } else {
-                        a.out0[c] = (float)s2;
+                        // dbeta = sum dy; dgamma = sum dy*xhat = (sum dy*y - beta sum dy)/gamma
+                        const double dg = (sy - bt * s1) / gm;
+                        a.out0[c] = (float)dg;
                         a.out1[c] = (float)s1;
-                        const double A = gm * rstd, B = -rstd * s2 / a.M;
+                        // dx = A dy + B y + Cc
+                        const double A = gm * rstd, B = -rstd * dg / a.M;
                         const double Cc = -gm * rstd * s1 / a.M - B * bt;
                         a.coef[c] = make_float4((float)A, (float)B, (float)Cc, 0.f);
                     }
@@ -427,60 +629,145 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             }
         }
     }
-    if (!fail && !grid_barrier(a.ctl, a.budget_ns)) fail = true;
+    stamp(4, tid == 0);
+    grid_barrier(a.ctl, a.budget_ns, &s_fail);
+    stamp(5, tid == 0);
 
-    // ---------------------------------------------------------- phase B
-    if (!fail) {
-        float c0[NV], c1[NV], c2[NV];
-        if (LAYOUT == kNHWC) {
-#pragma unroll
-            for (int k = 0; k < CPT; ++k)
-#pragma unroll
-                for (int j = 0; j < V; ++j) {
-                    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (colok[k]) q = a.coef[col[k] * V + j];
-                    c0[k * V + j] = q.x;
-                    c1[k * V + j] = q.y;
-                    c2[k * V + j] = q.z;
+    // ================================================================ phase B
+    // Producer: write tile t back from slot s.
+    auto store_tile = [&](int t, int s) {
+        unsigned char* dst = a.dst + t_u0(t) * P.unit_bytes;
+        const unsigned char* src = slot_ptr(s) + (DIR == 0 ? 0 : P.half_bytes);
+        const uint32_t bytes = (uint32_t)t_nu(t) * (uint32_t)P.unit_bytes;
+        if (P.hints)
+            bulk_store(dst, src, bytes, pol_stream);
+        else
+            bulk_store_plain(dst, src, bytes);
+    };
+    if (producer) {
+        if (pl && !failed()) {
+            uint32_t dpar = 0;
+            bool ok = true;
+            // resident tiles, in the consumers' order
+            for (int t = n - 1; t >= nring && ok; --t) {
+                const int s = ring + (t - nring);
+                ok = mbar_wait(&done[s], (dpar >> s) & 1u, a.budget_ns, a.wait_prod);
+                dpar ^= 1u << s;
+                if (!ok) break;
+                store_tile(t, s);
+                bulk_commit();
+            }
+            stamp(6, true);
+            for (int j = 0; j < nring && ok; ++j) {
+                const int s = j % ring;
+                ok = mbar_wait(&done[s], (dpar >> s) & 1u, a.budget_ns, a.wait_prod);
+                dpar ^= 1u << s;
+                if (!ok) break;
+                const int t = nring - 1 - j;
+                store_tile(t, s);
+                bulk_commit();
+                const int jn = j + ring;
+                if (jn < nring) {
+                    bulk_wait_read<0>();   // the store above has finished reading the slot
+                    issue(nring - 1 - jn, s, pol_stream);
                 }
+            }
+            if (!ok) set_failed();
+            stamp(7, true);
         }
+    } else if (!failed()) {
+        // coefficients of this thread's channels (NHWC)
+        // c3/c4 are kept per channel only when a thread owns one column;
+        // otherwise the backward forms them on the fly (register budget).
+        constexpr int NQ34 = CPT == 1 ? NQ : 1;
+        float2 c0[NQ], c1[NQ], c2[NQ], c3[NQ34], c4[NQ34];
+#pragma unroll
+        for (int k = 0; k < CPT; ++k)
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const int i = k * NP + q;
+                float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+                if (colok[k]) {
+                    v0 = a.coef[(col[k] * NP + q) * 2];
+                    v1 = a.coef[(col[k] * NP + q) * 2 + 1];
+                }
+                if (DIR == 0) {
+                    c0[i] = f2(-v0.x, -v1.x);    // -mean
+                    c1[i] = f2(v0.y, v1.y);      // scale
+                    c2[i] = f2(v0.w, v1.w);      // beta - mean*scale (16-bit storage)
+                    if (DT == kF32) c2[i] = f2(v0.z, v1.z);   // beta (fp32 storage)
+                } else {
+                    c0[i] = f2(v0.x, v1.x);                   // A
+                    c1[i] = f2(v0.y, v1.y);                   // B
+                    c2[i] = f2(v0.z, v1.z);                   // Cc
+                    if (CPT == 1) {
+                        c3[i] = f2(v0.x * p, v1.x * p);           // A*a (leaky, z <= 0)
+                        c4[i] = f2(v0.y * inv_p, v1.y * inv_p);   // B/a (leaky, z <= 0)
+                    }
+                }
+            }
         // Rewrites the tile in slot s in place (forward: x -> z; backward: dz -> dx).
         auto apply_tile = [&](int t, int s) {
             unsigned char* base = slot_ptr(s);
             if (LAYOUT == kNHWC) {
                 const int rows = t_nu(t);
-                if (CPT == 2 || colok[0]) {
-                    for (int r = phase; r < rows; r += RP) {
+                if (!active) return;
+                const int m = my_rows(rows);
+                const uint32_t sb = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
+#pragma unroll 2
+                for (int i = 0; i < m; ++i) {
 #pragma unroll
-                        for (int k = 0; k < CPT; ++k) {
-                            if (!colok[k]) continue;
-                            const size_t o = (size_t)r * RBY + col[k] * 16;
-                            if (DIR == 0) {
-                                uint4* pv = reinterpret_cast<uint4*>(base + o);
-                                float f[V];
-                                Vec<DT>::unpack(*pv, f);
+                    for (int k = 0; k < CPT; ++k) {
+                        if (CPT > 1 && !colok[k]) continue;
+                        const uint32_t o = sb + voff[k] + (uint32_t)i * vstep;
+                        if (DIR == 0) {
+                            float2 f[NP];
+                            Pairs<DT>::unpack(lds128(o), f);
 #pragma unroll
-                                for (int j = 0; j < V; ++j) {
-                                    const int q = k * V + j;
-                                    f[j] = act_forward<ACT, DT>(fmaf(f[j] - c0[q], c1[q], c2[q]),
-                                                                a.p);
-                                }
-                                *pv = Vec<DT>::pack(f);
-                            } else {
-                                const uint4 vz = *reinterpret_cast<const uint4*>(base + o);
-                                uint4* pd = reinterpret_cast<uint4*>(base + P.half_bytes + o);
-                                float fz[V], fd[V];
-                                Vec<DT>::unpack(vz, fz);
-                                Vec<DT>::unpack(*pd, fd);
-#pragma unroll
-                                for (int j = 0; j < V; ++j) {
-                                    const int q = k * V + j;
-                                    float y, dy;
-                                    act_backward<ACT, DT>(fz[j], fd[j], a.p, a.inv_p, y, dy);
-                                    fd[j] = fmaf(c0[q], dy, fmaf(c1[q], y, c2[q]));
-                                }
-                                *pd = Vec<DT>::pack(fd);
+                            for (int q = 0; q < NP; ++q) {
+                                const int j = k * NP + q;
+                                // 16-bit storage: y = x*scale + (beta - mean*scale); its
+                                // rounding error is far below one storage ulp.  fp32:
+                                // y = (x - mean)*scale + beta.
+                                const float2 y = DT == kF32
+                                                     ? __ffma2_rn(__fadd2_rn(f[q], c0[j]), c1[j],
+                                                                  c2[j])
+                                                     : __ffma2_rn(f[q], c1[j], c2[j]);
+                                f[q] = act_forward2<ACT, DT>(y, p, le1);
                             }
+                            sts128(o, Pairs<DT>::pack(f));
+                        } else {
+                            const uint32_t od = o + (uint32_t)P.half_bytes;
+                            float2 fz[NP], fd[NP];
+                            Pairs<DT>::unpack(lds128(o), fz);
+                            Pairs<DT>::unpack(lds128(od), fd);
+#pragma unroll
+                            for (int q = 0; q < NP; ++q) {
+                                const int j = k * NP + q;
+                                if (ACT == kLeaky) {
+                                    // dx = A dy + B y + Cc with (dy, y) = (dz, z) for z > 0
+                                    // and (a dz, z/a) otherwise
+                                    const bool px = fz[q].x > 0.f, py = fz[q].y > 0.f;
+                                    const float2 a3 = CPT == 1 ? c3[j < NQ34 ? j : 0]
+                                                               : __fmul2_rn(c0[j], f2(p, p));
+                                    const float2 a4 = CPT == 1
+                                                          ? c4[j < NQ34 ? j : 0]
+                                                          : __fmul2_rn(c1[j], f2(inv_p, inv_p));
+                                    const float2 Ak = f2(px ? c0[j].x : a3.x, py ? c0[j].y : a3.y);
+                                    const float2 Bk = f2(px ? c1[j].x : a4.x, py ? c1[j].y : a4.y);
+                                    fd[q] = __ffma2_rn(Ak, fd[q], __ffma2_rn(Bk, fz[q], c2[j]));
+                                } else if (ACT == kIdent) {
+                                    fd[q] = __ffma2_rn(c0[j], fd[q],
+                                                       __ffma2_rn(c1[j], fz[q], c2[j]));
+                                } else {
+                                    float y0, y1, d0, d1;
+                                    act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0, d0);
+                                    act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1, d1);
+                                    fd[q] = __ffma2_rn(c0[j], f2(d0, d1),
+                                                       __ffma2_rn(c1[j], f2(y0, y1), c2[j]));
+                                }
+                            }
+                            sts128(od, Pairs<DT>::pack(fd));
                         }
                     }
                 }
@@ -495,67 +782,56 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     if (DIR == 0) {
                         for (int i = glane; i < HW; i += L)
                             Elem<DT>::st(pz, i, act_forward<ACT, DT>(
-                                                    fmaf(Elem<DT>::ld(pz, i) - q.x, q.y, q.z), a.p));
+                                                    fmaf(Elem<DT>::ld(pz, i) - q.x, q.y, q.z), p));
                     } else {
                         unsigned char* pd = pz + P.half_bytes;
                         for (int i = glane; i < HW; i += L) {
                             float y, dy;
-                            act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), a.p,
-                                                  a.inv_p, y, dy);
+                            act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
+                                                  inv_p, y, dy);
                             Elem<DT>::st(pd, i, fmaf(q.x, dy, fmaf(q.y, y, q.z)));
                         }
                     }
                 }
             }
         };
-        // Thread 0 stores the rewritten tile (after every thread's writes are
-        // ordered before the bulk copy's reads).
-        auto store_tile = [&](int t, int s) {
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (tid == 0) {
-                const uint32_t bytes = (uint32_t)t_nu(t) * (uint32_t)P.unit_bytes;
-                const int64_t off = t_u0(t) * P.unit_bytes;
-                bulk_store(a.dst + off, slot_ptr(s) + (DIR == 0 ? 0 : P.half_bytes), bytes,
-                           pol_stream);
-                bulk_commit();
-            }
-        };
+        acct_start();
         for (int t = n - 1; t >= nring; --t) {
             const int s = ring + (t - nring);
             apply_tile(t, s);
-            store_tile(t, s);
+            fence_proxy_async_smem();
+            release(&done[s]);
         }
+        acct_work();
         for (int j = 0; j < nring; ++j) {
-            const int jn = j + depthB;
-            if (jn < nring) {
-                // the slot of ring tile jn last held ring tile jn - ring, stored
-                // at least two iterations ago
-                if (tid == 0) bulk_wait_read<1>();
-                issue(nring - 1 - jn, jn % ring, pol_stream);
-            }
             const int s = j % ring;
-            const bool ok = wait(s);
-            if (ok) apply_tile(nring - 1 - j, s);
-            if (__syncthreads_or(!ok)) {
-                fail = true;
-                break;
-            }
-            store_tile(nring - 1 - j, s);
+            if (!cwait(s)) break;
+            acct_wait();
+            apply_tile(nring - 1 - j, s);
+            acct_comp();
+            fence_proxy_async_smem();
+            release(&done[s]);
+            acct_work();
         }
+        acct_flush(11);
     }
 
     // ----------------------------------------------------------- exit
-    if (fail && tid == 0) {
-        atomicOr(&a.ctl->status, kStTimeout);
-        for (int s = 0; s < P.nslots; ++s)
-            if (pending & (1u << s)) mbar_wait(&bars[s], (parity >> s) & 1u, a.budget_ns);
+    if (pl) {
+        if (failed()) {
+            atomicOr(&a.ctl->status, kStTimeout);
+            // Wait (bounded) for the last load into every slot before the CTA
+            // exits; completed ones return at once.
+            for (int s = 0; s < P.nslots; ++s)
+                if ((loaded >> s) & 1u)
+                    mbar_wait(&full[s], ((fiss >> s) & 1u) ^ 1u, a.budget_ns / 4);
+        }
+        bulk_wait_all();
+        stamp(8, true);
     }
-    if (tid == 0) bulk_wait_all();
 }
 
 }  // namespace iabn
-
 #include <atomic>
 
 namespace iabn {
@@ -606,7 +882,8 @@ cudaError_t launch_resident_dir(const ResArgs& a, int layout, int cpt, int act, 
                                 cudaStream_t s) {
     if (layout == kNCHW) return launch_resident_act<DT, kNCHW, 1, DIR>(a, act, smem_optin, s);
     if (cpt == 1) return launch_resident_act<DT, kNHWC, 1, DIR>(a, act, smem_optin, s);
-    return launch_resident_act<DT, kNHWC, 2, DIR>(a, act, smem_optin, s);
+    if (cpt == 2) return launch_resident_act<DT, kNHWC, 2, DIR>(a, act, smem_optin, s);
+    return launch_resident_act<DT, kNHWC, 4, DIR>(a, act, smem_optin, s);
 }
 
 // Defined in iabn_resident_{f32,bf16,f16}.cu.
