@@ -207,6 +207,27 @@ class Layer:
                                        count=self.sp.per_channel, momentum=self.sp.momentum)
 
 
+class L2Flush:
+    """Evicts the L2 before a timed call: writes a buffer of twice the L2 size,
+    then reads another one as large, so the L2 holds only clean lines and the
+    timed kernel is not charged for writing back the flush's own dirty data.
+    ``write_only=True`` skips the read (the timed kernel then pays for that
+    write-back)."""
+
+    def __init__(self, device, write_only=False):
+        import torch
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        n = 2 * max(l2, 64 << 20)
+        self.w = torch.empty(n, dtype=torch.uint8, device=device)
+        self.r = torch.ones(n // 4, dtype=torch.int32, device=device)
+        self.write_only = write_only
+
+    def zero_(self):
+        self.w.zero_()
+        if not self.write_only:
+            self.r.sum()
+
+
 def timed_layer_steps(layer, flush, steps, warmup, dist_barrier=None, sampler=None):
     """Warm-up, then `steps` timed steps; returns per-step event times (ms) of
     fwd, bwd and the running-stat update, and the launch count in between."""
@@ -434,6 +455,26 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------- multi-rank
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (plain value when world == 1)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processed its own replica of the work;
+    the job took as long as the slowest rank."""
+    return world * bytes_per_rank / (max_ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------- main
 
 def run_profile(args):
@@ -441,8 +482,7 @@ def run_profile(args):
     import torch
     import workloads as wl
     device = torch.device("cuda", 0)
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device=device)
+    flush = L2Flush(device, write_only=os.environ.get("IABN_BENCH_WRITE_FLUSH") == "1")
     sp = wl.spec(args.profile)
     layer = Layer(sp, sp.seed, device)
     f, b, u, launches, _ = timed_layer_steps(layer, flush, args.steps, args.warmup)
@@ -502,8 +542,7 @@ def main():
         barrier = dist.barrier
 
     hbm_peak, peak_kind = measured_hbm_gbs()
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     sp = wl.spec(1)
     layer = Layer(sp, sp.seed + 1000 * rank, device)
 
@@ -512,23 +551,20 @@ def main():
                                                 barrier, sampler)
     t_step = [x + y + z for x, y, z in zip(f, b, u)]
     mean_ms = statistics.mean(t_step)
-    t_max = mean_ms
-    if world > 1:
-        tt = torch.tensor([mean_ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-    value = world * layer.bytes / (t_max * 1e-3) / 1e9
+    # the same steps with a write-only flush (the kernels then also pay for
+    # writing back the flush's dirty lines)
+    fw, bw, uw, _, _ = timed_layer_steps(layer, L2Flush(device, write_only=True),
+                                         max(5, args.steps // 5), 2, barrier)
+    wf_ms = reduce_max(statistics.mean([x + y + z for x, y, z in zip(fw, bw, uw)]), world,
+                       device)
+    t_max = reduce_max(mean_ms, world, device)
+    value = whole_job_gbs(layer.bytes, world, t_max)
     fwd_us, bwd_us = statistics.mean(f) * 1e3, statistics.mean(b) * 1e3
 
     # e2e through host buffers
     e_ms, h2d, d2h = e2e_steps(layer, max(3, args.steps // 10), 2)
-    e_mean = statistics.mean(e_ms)
-    e_max = e_mean
-    if world > 1:
-        tt = torch.tensor([e_mean], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_max = float(tt.item())
-    e2e_value = world * layer.bytes / (e_max * 1e-3) / 1e9
+    e_max = reduce_max(statistics.mean(e_ms), world, device)
+    e2e_value = whole_job_gbs(layer.bytes, world, e_max)
 
     extra = {}
     if not args.no_extra and world == 1:
@@ -547,11 +583,15 @@ def main():
                                    "leaky_relu 0.01, eps 1e-5, fwd+bwd+running stats",
                        "storage_dtype": "bf16", "elements": sp.numel,
                        "compulsory_bytes_per_step": layer.bytes,
-                       "l2": "flushed (2x L2 write) before every fwd and every bwd call",
+                       "l2": "flushed before every fwd and every bwd call: write 2x L2, then "
+                             "read another 2x L2 so only clean lines remain (outside the "
+                             "timed events); value_write_only_flush: same steps after a "
+                             "write-only flush",
                        "inputs": "restored from pristine device copies before each step",
                        "parallelism": f"replicas x{world} (no cross-GPU statistics)",
                        "plan": os.environ.get("IABN_FORCE_PLAN", "auto")},
             "elements_per_s": world * sp.numel / (t_max * 1e-3),
+            "value_write_only_flush": round(whole_job_gbs(layer.bytes, world, wf_ms), 1),
             "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
             "running_update_us": round(statistics.mean(u) * 1e3, 2),
             "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),

@@ -13,8 +13,8 @@
 // Tuning knobs read from the environment (defaults in brackets):
 //   IABN_L2_HINTS [1]       L2 evict-last on tiles phase B reloads, evict-first
 //                           on the rest; 0 = no hints.
-//   IABN_TILE_KB_FWD, IABN_TILE_KB_BWD [16, 8]  KiB per tensor per tile.
-//   IABN_RING_FWD, IABN_RING_BWD       [5, 5]   slots cycled by the stream.
+//   IABN_TILE_KB_FWD, IABN_TILE_KB_BWD [48, 24] KiB per tensor per tile.
+//   IABN_RING_FWD, IABN_RING_BWD       [4, 4]   slots cycled by the stream.
 //   IABN_BARRIER_BUDGET_NS  [1e9] time budget of each bounded wait.
 //   IABN_WAIT_CONS, IABN_WAIT_PROD [0]  mbarrier wait mode of the consumer warps
 //                           and of the producer: 0 try_wait, 1 test_wait spin,
@@ -82,7 +82,7 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     const int s = g.esize;
     const int NT = dir == 0 ? 1 : 2;
     const int target =
-        (int)env_long(dir == 0 ? "IABN_TILE_KB_FWD" : "IABN_TILE_KB_BWD", dir == 0 ? 16 : 8) * 1024;
+        (int)env_long(dir == 0 ? "IABN_TILE_KB_FWD" : "IABN_TILE_KB_BWD", dir == 0 ? 48 : 24) * 1024;
     if (target < 1024 || target > 65536) return false;
     P = ResPlan{};
     cpt = 1;
@@ -127,7 +127,7 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     const int budget = dl.smem_optin - 1024 - kBarBytes - P.scratch_bytes;
     int nslots = budget / P.slot_bytes;
     if (nslots > kMaxSlots) nslots = kMaxSlots;
-    int ring = (int)env_long(dir == 0 ? "IABN_RING_FWD" : "IABN_RING_BWD", 5);
+    int ring = (int)env_long(dir == 0 ? "IABN_RING_FWD" : "IABN_RING_BWD", 4);
     if (ring < 2) ring = 2;
     if (ring > nslots) return false;
     P.nslots = nslots;

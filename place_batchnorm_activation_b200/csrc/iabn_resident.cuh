@@ -658,18 +658,21 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 bulk_commit();
             }
             stamp(6, true);
+            // Streamed tiles: store tile j as soon as the consumers are done
+            // with it; its slot is refilled (with streamed tile j + ring) one
+            // step later, once the store has finished reading it, so a store
+            // and the next reload never wait for each other.
             for (int j = 0; j < nring && ok; ++j) {
                 const int s = j % ring;
                 ok = mbar_wait(&done[s], (dpar >> s) & 1u, a.budget_ns, a.wait_prod);
                 dpar ^= 1u << s;
                 if (!ok) break;
-                const int t = nring - 1 - j;
-                store_tile(t, s);
+                store_tile(nring - 1 - j, s);
                 bulk_commit();
-                const int jn = j + ring;
-                if (jn < nring) {
-                    bulk_wait_read<0>();   // the store above has finished reading the slot
-                    issue(nring - 1 - jn, s, pol_stream);
+                const int jp = j - 1, jn = jp + ring;   // refill the previous slot
+                if (jp >= 0 && jn < nring) {
+                    bulk_wait_read<1>();   // all stores but the one just issued have read
+                    issue(nring - 1 - jn, jp % ring, pol_stream);
                 }
             }
             if (!ok) set_failed();
