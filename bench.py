@@ -511,8 +511,8 @@ def run_profile(args):
             for k, nm in enumerate(names):
                 v = sorted((r[k] - t0) / 1e3 for r in rows)
                 parts.append(f"{nm}={v[len(v) // 2]:.1f}[{v[0]:.1f},{v[-1]:.1f}]")
-            for k, nm in ((9, "A.wait_kcyc"), (10, "A.work_kcyc"), (11, "B.wait_kcyc"),
-                          (12, "B.work_kcyc")):
+            for k, nm in ((9, "A.wait_kcyc"), (10, "A.work_kcyc"), (13, "A.comp_kcyc"),
+                          (11, "B.wait_kcyc"), (12, "B.work_kcyc"), (15, "B.comp_kcyc")):
                 v = sorted(r[k] / 1e3 for r in rows)
                 parts.append(f"{nm}={v[len(v) // 2]:.1f}")
             print(f"trace {sp.name} {what} ({len(rows)} CTAs): " + " ".join(parts), flush=True)

@@ -94,6 +94,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     }
 }
 
+// 16-byte global store.
+__device__ __forceinline__ void stg128(void* p, const uint4& v) {
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 // 16-byte shared-memory load / store at a 32-bit shared address.
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
@@ -103,10 +110,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
+// (No "memory" clobber: ordering against the mbarrier arrive and the async
+// proxy fence that follow comes from those volatile asm statements, and a
+// clobber here would serialise every row of the tile loops.)
 __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
-                 : "memory");
+                 "r"(v.z), "r"(v.w));
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {

@@ -158,6 +158,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     constexpr int NT = DIR == 0 ? 1 : 2;       // tensors per tile
     constexpr int NP = Pairs<DT>::NP;          // channel pairs per 16-byte vector
     constexpr int NQ = CPT * NP;               // channel pairs per thread (NHWC)
+    // rows per batch in the tile loops
+    constexpr int RB = 4 / CPT > 0 ? 4 / CPT : 1;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxSlots;
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int b = blockIdx.x;
     const int G = P.G;
     // Phase trace: 0 start, 1 phase A done, 2 merged, 3 barrier 1, 4 finalize,
-    // 5 barrier 2, 6 resident tiles stored, 7 phase B stored, 8 stores complete
+    // 5 barrier 2, 6 unused, 7 last refill issued, 8 producer exit
     // (%globaltimer ns); 9/10/13 phase A and 11/12/15 phase B SM cycles of
     // consumer warp 0: waiting for tiles / bookkeeping / the row loops.
     auto stamp = [&](int k, bool who) {
@@ -387,49 +389,62 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     const int m = my_rows(rows);
                     const uint32_t sb = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
                     acct_work();
-#pragma unroll 2
-                    for (int i = 0; i < m; ++i) {
+                    // rows in batches of RB: all loads of a batch first, then the math
+                    for (int i0 = 0; i0 < m; i0 += RB) {
+                        uint4 vz[RB][CPT], vd[RB][CPT];
 #pragma unroll
-                        for (int k = 0; k < CPT; ++k) {
-                            if (CPT > 1 && !colok[k]) continue;
-                            const uint32_t o = sb + voff[k] + (uint32_t)i * vstep;
-                            if (DIR == 0) {
-                                float2 f[NP];
-                                Pairs<DT>::unpack(lds128(o), f);
+                        for (int u = 0; u < RB; ++u)
 #pragma unroll
-                                for (int q = 0; q < NP; ++q) {
-                                    const int j = k * NP + q;
-                                    const float2 d = __fadd2_rn(f[q], piv[j]);
-                                    acc0[j] = __fadd2_rn(acc0[j], d);
-                                    acc1[j] = __ffma2_rn(d, d, acc1[j]);
-                                }
-                            } else {
-                                float2 fz[NP], fd[NP];
-                                Pairs<DT>::unpack(lds128(o), fz);
-                                Pairs<DT>::unpack(lds128(o + (uint32_t)P.half_bytes), fd);
+                            for (int k = 0; k < CPT; ++k) {
+                                if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
+                                const uint32_t o = sb + voff[k] + (uint32_t)(i0 + u) * vstep;
+                                vz[u][k] = lds128(o);
+                                if (DIR == 1) vd[u][k] = lds128(o + (uint32_t)P.half_bytes);
+                            }
 #pragma unroll
-                                for (int q = 0; q < NP; ++q) {
-                                    const int j = k * NP + q;
-                                    if (ACT == kLeaky) {
-                                        // dy*y = dz*z on both branches
-                                        acc1[j] = __ffma2_rn(fd[q], fz[q], acc1[j]);
-                                        const float2 ad = __fmul2_rn(fd[q], f2(p, p));
-                                        const float2 dy = f2(fz[q].x > 0.f ? fd[q].x : ad.x,
-                                                             fz[q].y > 0.f ? fd[q].y : ad.y);
-                                        acc0[j] = __fadd2_rn(acc0[j], dy);
-                                    } else if (ACT == kIdent) {
-                                        acc1[j] = __ffma2_rn(fd[q], fz[q], acc1[j]);
-                                        acc0[j] = __fadd2_rn(acc0[j], fd[q]);
-                                    } else {
-                                        float y0, y1, d0, d1;
-                                        act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0, d0);
-                                        act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1, d1);
-                                        acc0[j] = __fadd2_rn(acc0[j], f2(d0, d1));
-                                        acc1[j] = __ffma2_rn(f2(d0, d1), f2(y0, y1), acc1[j]);
+                        for (int u = 0; u < RB; ++u)
+#pragma unroll
+                            for (int k = 0; k < CPT; ++k) {
+                                if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
+                                if (DIR == 0) {
+                                    float2 f[NP];
+                                    Pairs<DT>::unpack(vz[u][k], f);
+#pragma unroll
+                                    for (int q = 0; q < NP; ++q) {
+                                        const int j = k * NP + q;
+                                        const float2 d = __fadd2_rn(f[q], piv[j]);
+                                        acc0[j] = __fadd2_rn(acc0[j], d);
+                                        acc1[j] = __ffma2_rn(d, d, acc1[j]);
+                                    }
+                                } else {
+                                    float2 fz[NP], fd[NP];
+                                    Pairs<DT>::unpack(vz[u][k], fz);
+                                    Pairs<DT>::unpack(vd[u][k], fd);
+#pragma unroll
+                                    for (int q = 0; q < NP; ++q) {
+                                        const int j = k * NP + q;
+                                        if (ACT == kLeaky) {
+                                            // dy*y = dz*z on both branches
+                                            acc1[j] = __ffma2_rn(fd[q], fz[q], acc1[j]);
+                                            const float2 ad = __fmul2_rn(fd[q], f2(p, p));
+                                            const float2 dy = f2(fz[q].x > 0.f ? fd[q].x : ad.x,
+                                                                 fz[q].y > 0.f ? fd[q].y : ad.y);
+                                            acc0[j] = __fadd2_rn(acc0[j], dy);
+                                        } else if (ACT == kIdent) {
+                                            acc1[j] = __ffma2_rn(fd[q], fz[q], acc1[j]);
+                                            acc0[j] = __fadd2_rn(acc0[j], fd[q]);
+                                        } else {
+                                            float y0, y1, d0, d1;
+                                            act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0,
+                                                                  d0);
+                                            act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1,
+                                                                  d1);
+                                            acc0[j] = __fadd2_rn(acc0[j], f2(d0, d1));
+                                            acc1[j] = __ffma2_rn(f2(d0, d1), f2(y0, y1), acc1[j]);
+                                        }
                                     }
                                 }
                             }
-                        }
                     }
                     acct_comp();
                 }
@@ -509,6 +524,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
         if (active && phase == 0) {
             const double nb = (double)(u1 - u0);
+            const double inv_nb = 1.0 / nb;
 #pragma unroll
             for (int k = 0; k < CPT; ++k)
                 if (colok[k])
@@ -520,10 +536,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         if (DIR == 0) {
                             // (mean, M2) of the CTA from its pivot-shifted sums
                             const double s1x = acc0[i].x, s1y = acc0[i].y;
-                            dstp[0] = make_double2(-(double)piv[i].x + s1x / nb,
-                                                   (double)acc1[i].x - s1x * s1x / nb);
-                            dstp[1] = make_double2(-(double)piv[i].y + s1y / nb,
-                                                   (double)acc1[i].y - s1y * s1y / nb);
+                            dstp[0] = make_double2(fma(s1x, inv_nb, -(double)piv[i].x),
+                                                   fma(-s1x * s1x, inv_nb, (double)acc1[i].x));
+                            dstp[1] = make_double2(fma(s1y, inv_nb, -(double)piv[i].y),
+                                                   fma(-s1y * s1y, inv_nb, (double)acc1[i].y));
                         } else {
                             dstp[0] = make_double2(acc0[i].x, acc1[i].x);
                             dstp[1] = make_double2(acc0[i].y, acc1[i].y);
@@ -634,46 +650,19 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     stamp(5, tid == 0);
 
     // ================================================================ phase B
-    // Producer: write tile t back from slot s.
-    auto store_tile = [&](int t, int s) {
-        unsigned char* dst = a.dst + t_u0(t) * P.unit_bytes;
-        const unsigned char* src = slot_ptr(s) + (DIR == 0 ? 0 : P.half_bytes);
-        const uint32_t bytes = (uint32_t)t_nu(t) * (uint32_t)P.unit_bytes;
-        if (P.hints)
-            bulk_store(dst, src, bytes, pol_stream);
-        else
-            bulk_store_plain(dst, src, bytes);
-    };
     if (producer) {
         if (pl && !failed()) {
+            // The consumers write their results to global memory themselves;
+            // the producer refills each streamed slot with streamed tile
+            // j + ring once they are done with tile j.
             uint32_t dpar = 0;
             bool ok = true;
-            // resident tiles, in the consumers' order
-            for (int t = n - 1; t >= nring && ok; --t) {
-                const int s = ring + (t - nring);
-                ok = mbar_wait(&done[s], (dpar >> s) & 1u, a.budget_ns, a.wait_prod);
-                dpar ^= 1u << s;
-                if (!ok) break;
-                store_tile(t, s);
-                bulk_commit();
-            }
-            stamp(6, true);
-            // Streamed tiles: store tile j as soon as the consumers are done
-            // with it; its slot is refilled (with streamed tile j + ring) one
-            // step later, once the store has finished reading it, so a store
-            // and the next reload never wait for each other.
-            for (int j = 0; j < nring && ok; ++j) {
+            for (int j = 0; j + ring < nring && ok; ++j) {
                 const int s = j % ring;
                 ok = mbar_wait(&done[s], (dpar >> s) & 1u, a.budget_ns, a.wait_prod);
                 dpar ^= 1u << s;
                 if (!ok) break;
-                store_tile(nring - 1 - j, s);
-                bulk_commit();
-                const int jp = j - 1, jn = jp + ring;   // refill the previous slot
-                if (jp >= 0 && jn < nring) {
-                    bulk_wait_read<1>();   // all stores but the one just issued have read
-                    issue(nring - 1 - jn, jp % ring, pol_stream);
-                }
+                issue(nring - 1 - (j + ring), s, pol_stream);
             }
             if (!ok) set_failed();
             stamp(7, true);
@@ -717,62 +706,86 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 if (!active) return;
                 const int m = my_rows(rows);
                 const uint32_t sb = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
-#pragma unroll 2
-                for (int i = 0; i < m; ++i) {
+                const uint32_t hb = DIR == 0 ? 0u : (uint32_t)P.half_bytes;
+                unsigned char* gtile = a.dst + t_u0(t) * P.unit_bytes;
+                // rows in batches of RB: loads, then math, then stores
+                for (int i0 = 0; i0 < m; i0 += RB) {
+                    uint4 vz[RB][CPT], vd[RB][CPT];
 #pragma unroll
-                    for (int k = 0; k < CPT; ++k) {
-                        if (CPT > 1 && !colok[k]) continue;
-                        const uint32_t o = sb + voff[k] + (uint32_t)i * vstep;
-                        if (DIR == 0) {
-                            float2 f[NP];
-                            Pairs<DT>::unpack(lds128(o), f);
+                    for (int u = 0; u < RB; ++u)
 #pragma unroll
-                            for (int q = 0; q < NP; ++q) {
-                                const int j = k * NP + q;
-                                // 16-bit storage: y = x*scale + (beta - mean*scale); its
-                                // rounding error is far below one storage ulp.  fp32:
-                                // y = (x - mean)*scale + beta.
-                                const float2 y = DT == kF32
-                                                     ? __ffma2_rn(__fadd2_rn(f[q], c0[j]), c1[j],
-                                                                  c2[j])
-                                                     : __ffma2_rn(f[q], c1[j], c2[j]);
-                                f[q] = act_forward2<ACT, DT>(y, p, le1);
-                            }
-                            sts128(o, Pairs<DT>::pack(f));
-                        } else {
-                            const uint32_t od = o + (uint32_t)P.half_bytes;
-                            float2 fz[NP], fd[NP];
-                            Pairs<DT>::unpack(lds128(o), fz);
-                            Pairs<DT>::unpack(lds128(od), fd);
-#pragma unroll
-                            for (int q = 0; q < NP; ++q) {
-                                const int j = k * NP + q;
-                                if (ACT == kLeaky) {
-                                    // dx = A dy + B y + Cc with (dy, y) = (dz, z) for z > 0
-                                    // and (a dz, z/a) otherwise
-                                    const bool px = fz[q].x > 0.f, py = fz[q].y > 0.f;
-                                    const float2 a3 = CPT == 1 ? c3[j < NQ34 ? j : 0]
-                                                               : __fmul2_rn(c0[j], f2(p, p));
-                                    const float2 a4 = CPT == 1
-                                                          ? c4[j < NQ34 ? j : 0]
-                                                          : __fmul2_rn(c1[j], f2(inv_p, inv_p));
-                                    const float2 Ak = f2(px ? c0[j].x : a3.x, py ? c0[j].y : a3.y);
-                                    const float2 Bk = f2(px ? c1[j].x : a4.x, py ? c1[j].y : a4.y);
-                                    fd[q] = __ffma2_rn(Ak, fd[q], __ffma2_rn(Bk, fz[q], c2[j]));
-                                } else if (ACT == kIdent) {
-                                    fd[q] = __ffma2_rn(c0[j], fd[q],
-                                                       __ffma2_rn(c1[j], fz[q], c2[j]));
-                                } else {
-                                    float y0, y1, d0, d1;
-                                    act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0, d0);
-                                    act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1, d1);
-                                    fd[q] = __ffma2_rn(c0[j], f2(d0, d1),
-                                                       __ffma2_rn(c1[j], f2(y0, y1), c2[j]));
-                                }
-                            }
-                            sts128(od, Pairs<DT>::pack(fd));
+                        for (int k = 0; k < CPT; ++k) {
+                            if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
+                            const uint32_t o = sb + voff[k] + (uint32_t)(i0 + u) * vstep;
+                            vz[u][k] = lds128(o);
+                            if (DIR == 1) vd[u][k] = lds128(o + hb);
                         }
-                    }
+#pragma unroll
+                    for (int u = 0; u < RB; ++u)
+#pragma unroll
+                        for (int k = 0; k < CPT; ++k) {
+                            if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
+                            if (DIR == 0) {
+                                float2 f[NP];
+                                Pairs<DT>::unpack(vz[u][k], f);
+#pragma unroll
+                                for (int q = 0; q < NP; ++q) {
+                                    const int j = k * NP + q;
+                                    // 16-bit storage: y = x*scale + (beta - mean*scale); its
+                                    // rounding error is far below one storage ulp.  fp32:
+                                    // y = (x - mean)*scale + beta.
+                                    const float2 y =
+                                        DT == kF32 ? __ffma2_rn(__fadd2_rn(f[q], c0[j]), c1[j], c2[j])
+                                                   : __ffma2_rn(f[q], c1[j], c2[j]);
+                                    f[q] = act_forward2<ACT, DT>(y, p, le1);
+                                }
+                                vz[u][k] = Pairs<DT>::pack(f);
+                            } else {
+                                float2 fz[NP], fd[NP];
+                                Pairs<DT>::unpack(vz[u][k], fz);
+                                Pairs<DT>::unpack(vd[u][k], fd);
+#pragma unroll
+                                for (int q = 0; q < NP; ++q) {
+                                    const int j = k * NP + q;
+                                    if (ACT == kLeaky) {
+                                        // dx = A dy + B y + Cc with (dy, y) = (dz, z) for z > 0
+                                        // and (a dz, z/a) otherwise
+                                        const bool px = fz[q].x > 0.f, py = fz[q].y > 0.f;
+                                        const float2 a3 = CPT == 1
+                                                              ? c3[j < NQ34 ? j : 0]
+                                                              : __fmul2_rn(c0[j], f2(p, p));
+                                        const float2 a4 =
+                                            CPT == 1 ? c4[j < NQ34 ? j : 0]
+                                                     : __fmul2_rn(c1[j], f2(inv_p, inv_p));
+                                        const float2 Ak = f2(px ? c0[j].x : a3.x,
+                                                             py ? c0[j].y : a3.y);
+                                        const float2 Bk = f2(px ? c1[j].x : a4.x,
+                                                             py ? c1[j].y : a4.y);
+                                        fd[q] = __ffma2_rn(Ak, fd[q],
+                                                           __ffma2_rn(Bk, fz[q], c2[j]));
+                                    } else if (ACT == kIdent) {
+                                        fd[q] = __ffma2_rn(c0[j], fd[q],
+                                                           __ffma2_rn(c1[j], fz[q], c2[j]));
+                                    } else {
+                                        float y0, y1, d0, d1;
+                                        act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0, d0);
+                                        act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1, d1);
+                                        fd[q] = __ffma2_rn(c0[j], f2(d0, d1),
+                                                           __ffma2_rn(c1[j], f2(y0, y1), c2[j]));
+                                    }
+                                }
+                                vd[u][k] = Pairs<DT>::pack(fd);
+                            }
+                        }
+                    // results go straight to their place in global memory
+#pragma unroll
+                    for (int u = 0; u < RB; ++u)
+#pragma unroll
+                        for (int k = 0; k < CPT; ++k) {
+                            if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
+                            unsigned char* g = gtile + voff[k] + (size_t)(i0 + u) * vstep;
+                            stg128(g, DIR == 0 ? vz[u][k] : vd[u][k]);
+                        }
                 }
             } else {
                 const int np = t_nu(t) * P.g;
@@ -781,18 +794,19 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 for (int pp = grp; pp < np; pp += GP) {
                     const uint32_t c = (cbase + (uint32_t)pp) % (uint32_t)a.C;
                     const float4 q = __ldg(a.coef + c);
-                    unsigned char* pz = base + (size_t)pp * pbytes;
+                    const unsigned char* pz = base + (size_t)pp * pbytes;
+                    unsigned char* gz = a.dst + (t_u0(t) * P.g + pp) * (int64_t)pbytes;
                     if (DIR == 0) {
                         for (int i = glane; i < HW; i += L)
-                            Elem<DT>::st(pz, i, act_forward<ACT, DT>(
+                            Elem<DT>::st(gz, i, act_forward<ACT, DT>(
                                                     fmaf(Elem<DT>::ld(pz, i) - q.x, q.y, q.z), p));
                     } else {
-                        unsigned char* pd = pz + P.half_bytes;
+                        const unsigned char* pd = pz + P.half_bytes;
                         for (int i = glane; i < HW; i += L) {
                             float y, dy;
                             act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
                                                   inv_p, y, dy);
-                            Elem<DT>::st(pd, i, fmaf(q.x, dy, fmaf(q.y, y, q.z)));
+                            Elem<DT>::st(gz, i, fmaf(q.x, dy, fmaf(q.y, y, q.z)));
                         }
                     }
                 }
@@ -802,7 +816,6 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         for (int t = n - 1; t >= nring; --t) {
             const int s = ring + (t - nring);
             apply_tile(t, s);
-            fence_proxy_async_smem();
             release(&done[s]);
         }
         acct_work();
@@ -812,7 +825,6 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             acct_wait();
             apply_tile(nring - 1 - j, s);
             acct_comp();
-            fence_proxy_async_smem();
             release(&done[s]);
             acct_work();
         }
@@ -829,7 +841,6 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 if ((loaded >> s) & 1u)
                     mbar_wait(&full[s], ((fiss >> s) & 1u) ^ 1u, a.budget_ns / 4);
         }
-        bulk_wait_all();
         stamp(8, true);
     }
 }
