@@ -491,8 +491,8 @@ def run_profile(args):
     if os.environ.get("IABN_TRACE") == "1":
         # phase stamps of the resident kernels (see k_resident): per-CTA times
         # relative to the earliest CTA start, median / min / max over CTAs (us)
-        names = ["start", "phaseA", "merge+prefetch", "barrier1", "finalize", "barrier2",
-                 "resident", "phaseB", "exit"]
+        names = ["start", "phaseA", "merged", "barrier1", "finalize", "barrier2",
+                 "merge_rounds", "last_refill", "exit"]
         for what, call in (("fwd", layer.fwd), ("bwd", layer.bwd)):
             layer.restore()
             flush.zero_()

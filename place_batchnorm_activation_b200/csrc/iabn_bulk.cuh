@@ -175,6 +175,18 @@ __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+// Asynchronous 4-byte global -> shared copy (no register staging, so the
+// issuing thread does not stall on the load); cp_async_wait_all() makes the
+// issuing thread's copies visible to it.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Waits until at most N committed store groups still read shared memory.
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {

@@ -26,8 +26,8 @@ constexpr uint32_t kStSingular = 1u << 1;
 // First 256 bytes of every workspace.
 struct Control {
     uint32_t status;     // sticky kSt* bits
-    uint32_t bar_count;  // grid-barrier arrivals in the current round (0 between rounds)
-    uint32_t bar_gen;    // grid-barrier generation, bumped once per completed round
+    uint32_t bar_count;  // grid-barrier arrivals; a multiple of kBarStride between launches
+    uint32_t bar_gen;    // unused
     uint32_t pad[61];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
@@ -137,26 +137,32 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v
 }
 
 // Grid-wide barrier for a co-resident (cooperatively launched) grid, with a
-// time budget.  Central counter with a generation word: the last CTA to
-// arrive resets the counter and bumps the generation; the others wait for
-// the bump.  *fail (shared memory) is the CTA's failure flag: a CTA that has
-// failed does not arrive; a wait that runs out sets *fail and kStTimeout.
-// Every thread of the CTA must call it; returns !*fail.
-__device__ __forceinline__ bool grid_barrier(Control* ctl, unsigned long long budget_ns,
-                                             int* fail) {
+// time budget.  The arrival counter only grows: each CTA adds 1 and waits
+// until the counter reaches `target`, so the last arrival releases every
+// poller directly.  Targets of one launch are base + G, base + 2G, ...; base
+// is the counter at launch rounded down to a multiple of kBarStride (a CTA
+// that starts late may already see up to G-1 early arrivals, and G <=
+// kBarStride), and the launch pads the counter to base + 2*kBarStride before
+// it ends (bar_pad), so the next launch again starts on a multiple.  The
+// __syncthreads() before the arrival orders the CTA's writes before thread
+// 0's release (a cumulative release after a CTA barrier).  *fail (shared
+// memory) is the CTA's failure flag: a CTA that has failed does not arrive; a
+// wait that runs out sets *fail and kStTimeout (the control block must then
+// be cleared before the next launch).  Every thread of the CTA must call it.
+constexpr uint32_t kBarStride = 256;
+
+__device__ __forceinline__ uint32_t bar_base(const Control* ctl) {
+    return ld_acquire_gpu(&ctl->bar_count) & ~(kBarStride - 1u);
+}
+
+__device__ __forceinline__ bool grid_barrier(Control* ctl, uint32_t target,
+                                             unsigned long long budget_ns, int* fail) {
     __syncthreads();
     if (threadIdx.x == 0 && *((volatile int*)fail) == 0) {
-        const uint32_t gen = ld_acquire_gpu(&ctl->bar_gen);
-        const uint32_t nblocks = gridDim.x * gridDim.y * gridDim.z;
-        __threadfence();
         const uint32_t arrived = atom_add_acq_rel_gpu(&ctl->bar_count, 1u) + 1u;
-        if (arrived == nblocks) {
-            ctl->bar_count = 0u;
-            __threadfence();
-            st_release_gpu(&ctl->bar_gen, gen + 1u);
-        } else {
+        if (arrived != target) {
             const unsigned long long t0 = global_ns();
-            while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
+            while ((int32_t)(ld_acquire_gpu(&ctl->bar_count) - target) < 0) {
                 if (global_ns() - t0 > budget_ns) {
                     atomicOr(&ctl->status, kStTimeout);
                     *((volatile int*)fail) = 1;
@@ -167,6 +173,12 @@ __device__ __forceinline__ bool grid_barrier(Control* ctl, unsigned long long bu
     }
     __syncthreads();
     return *((volatile int*)fail) == 0;
+}
+
+// Called by one thread of one CTA after the launch's last barrier (nbar
+// barriers of G arrivals each): brings the counter to base + 2*kBarStride.
+__device__ __forceinline__ void bar_pad(Control* ctl, uint32_t G, uint32_t nbar) {
+    atomicAdd(&ctl->bar_count, 2u * kBarStride - nbar * G);
 }
 
 // Deterministic warp reductions (fixed shuffle-down tree; lane 0 holds the

@@ -101,8 +101,8 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         P.tile_units = tr;
         P.g = 1;
         P.L = 1;
-        // merge tree: ceil(RP/2) rows of VC columns of 16-byte float4 per pair
-        if (cpt == 1 && P.RP > 1) scratch = (P.RP + 1) / 2 * P.VC * (8 / s) * 16;
+        // merge: RP-1 row phases x VC columns x one 16-byte float4 per pair
+        if (cpt == 1 && P.RP > 1) scratch = (P.RP - 1) * P.VC * (8 / s) * 16;
     } else {
         const int64_t pb = g.HW * s;
         const int gq = 16 / gcd_int(pb, 16);

@@ -5,24 +5,27 @@
 // Each CTA owns a contiguous range of "units" (NHWC: rows of C channels;
 // NCHW: groups of g whole planes, g chosen so every unit starts on a 16-byte
 // boundary) and streams it through shared-memory slots with the bulk-copy
-// engine.  One producer warp issues every bulk load and store; eight
-// consumer warps compute.  Slots are handed over with mbarriers (full: data
-// landed; empty: consumers done with a streamed tile; done: a rewritten tile
-// may be stored), so no consumer waits on a CTA-wide barrier per tile.
+// engine.  One producer warp issues every bulk load; eight consumer warps
+// compute and store.  Slots are handed over with mbarriers (full: data
+// landed; empty: consumers done with a phase A tile; done: consumers done
+// with a phase B tile, so the slot may be refilled), so no consumer waits on
+// a CTA-wide barrier per tile.
 //
 //   phase A  tiles 0..n-1: per-thread partial statistics from shared memory.
-//            Forward: pivot-shifted sums of x (pivot = the CTA's first row) or,
-//            NCHW, exact per-plane two-pass mean and M2.  Backward: sum dy and
-//            sum dy*y (the "INPLACE-ABN II" form; for leaky-ReLU dy*y = dz*z).
+//            Forward: pivot-shifted sums of x (pivot = the tensor's first row,
+//            the same in every CTA) or, NCHW, exact per-plane two-pass mean and
+//            M2.  Backward: sum dy and sum dy*y (the "INPLACE-ABN II" form; for
+//            leaky-ReLU dy*y = dz*z).
 //            The last D tiles land in dedicated slots and stay resident; as
 //            soon as a streamed slot frees, the producer prefetches phase B.
-//   merge    NHWC: the threads of a column add their sums in a fixed tree;
-//            one partial per (CTA, channel).  NCHW: one partial per plane.
+//   merge    NHWC: the threads of a column add their sums in row-phase
+//            order; one partial per (CTA, channel).  NCHW: one partial per plane.
 //   barrier  grid-wide (bounded wait), a distributed fp64 finalize (one warp
 //            per channel, fixed order), a second grid barrier.
-//   phase B  tiles n-1..0: resident tiles are rewritten in place first, then
-//            the streamed ones -- the most recently read first, while they are
-//            still in L2 -- and the producer writes each back with a bulk store.
+//   phase B  tiles n-1..0: resident tiles first, then the streamed ones -- the
+//            most recently read first, while they are still in L2.  The
+//            consumers write their results straight to global memory with
+//            128-bit stores; the producer refills each freed streamed slot.
 //
 // Method: "In-Place Activated BatchNorm for Memory-Optimized Training of
 // DNNs" (paperlayer.ai summary), section 3: "Batch Normalization Review",
@@ -165,6 +168,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     uint64_t* empty = full + kMaxSlots;
     uint64_t* done = empty + kMaxSlots;
     __shared__ int s_fail;
+    // gamma, beta (and, backward, the saved variance) of the first channel
+    // each consumer warp finalizes, fetched while phase A streams
+    __shared__ float s_par[kConsumerWarps][3];
 
     const ResPlan& P = a.P;
     unsigned char* scratch = smem + kBarBytes;
@@ -175,7 +181,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int b = blockIdx.x;
     const int G = P.G;
     // Phase trace: 0 start, 1 phase A done, 2 merged, 3 barrier 1, 4 finalize,
-    // 5 barrier 2, 6 unused, 7 last refill issued, 8 producer exit
+    // 5 barrier 2, 6 in-CTA merge rounds done, 7 last refill issued, 8 consumer
+    // warp 0 done
     // (%globaltimer ns); 9/10/13 phase A and 11/12/15 phase B SM cycles of
     // consumer warp 0: waiting for tiles / bookkeeping / the row loops.
     auto stamp = [&](int k, bool who) {
@@ -220,6 +227,19 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
         mbar_init_fence();
         s_fail = 0;
+    }
+    // grid-barrier counter base of this launch (thread 0 only; see grid_barrier)
+    const uint32_t bbase = tid == 0 ? bar_base(a.ctl) : 0u;
+    if (!producer && lane == 0) {
+        const int64_t c = (int64_t)b * kConsumerWarps + warp;
+        if (c < a.C) {
+            cp_async4(&s_par[warp][0], a.gamma + c);
+            cp_async4(&s_par[warp][1], a.beta + c);
+            if (DIR == 1) cp_async4(&s_par[warp][2], a.var_in + c);
+            // forward NHWC: the aligned word holding the pivot x[0, c]
+            if (DIR == 0 && LAYOUT == kNHWC)
+                cp_async4(&s_par[warp][2], a.src0 + ((c * (int64_t)sizeof(typename Storage<DT>::T)) & ~int64_t(3)));
+        }
     }
     __syncthreads();
 
@@ -362,6 +382,18 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         acc1[q] = f2(0.f, 0.f);
         piv[q] = f2(0.f, 0.f);
     }
+    if (DIR == 0 && LAYOUT == kNHWC && active) {
+        // pivot (negated): the tensor's first row, the same for every CTA, so
+        // the CTA partials are plain sums around it (no per-CTA counts)
+#pragma unroll
+        for (int k = 0; k < CPT; ++k)
+            if (colok[k]) {
+                float2 f[NP];
+                Pairs<DT>::unpack(__ldg(reinterpret_cast<const uint4*>(a.src0) + col[k]), f);
+#pragma unroll
+                for (int q = 0; q < NP; ++q) piv[k * NP + q] = f2(-f[q].x, -f[q].y);
+            }
+    }
 
     if (!producer) {
         acct_start();
@@ -373,19 +405,6 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             if (LAYOUT == kNHWC) {
                 const int rows = t_nu(t);
                 if (active) {
-                    if (DIR == 0 && t == 0) {
-                        // pivot: the CTA's first row
-#pragma unroll
-                        for (int k = 0; k < CPT; ++k)
-                            if (colok[k]) {
-                                float2 f[NP];
-                                Pairs<DT>::unpack(
-                                    *reinterpret_cast<const uint4*>(base + col[k] * 16), f);
-#pragma unroll
-                                for (int q = 0; q < NP; ++q)
-                                    piv[k * NP + q] = f2(-f[q].x, -f[q].y);
-                            }
-                    }
                     const int m = my_rows(rows);
                     const uint32_t sb = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
                     acct_work();
@@ -498,33 +517,33 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     // ------------------------------------------- per-CTA merge (NHWC)
     if (!failed() && LAYOUT == kNHWC) {
         if (CPT == 1 && RP > 1) {
-            // Fixed tree over row phases: in round st the phases p with
-            // p % 2st == st write their sums, those with p % 2st == 0 add them.
-            float4* scr = reinterpret_cast<float4*>(scratch);   // [ceil(RP/2)][VC][NP]
-            for (int st = 1; st < RP; st <<= 1) {
-                const bool writer = colok[0] && (phase % (2 * st)) == st;
-                const bool reader = colok[0] && (phase % (2 * st)) == 0 && phase + st < RP;
-                const size_t row = (size_t)(phase / (2 * st)) * VC + col[0];
-                if (writer) {
+            // Row phases 1..RP-1 publish their sums ([phase-1][pair][column]
+            // float4s, so a warp's stores and loads are contiguous); phase 0
+            // adds them in phase order.
+            float4* scr = reinterpret_cast<float4*>(scratch);
+            if (colok[0] && phase > 0) {
 #pragma unroll
-                    for (int q = 0; q < NP; ++q)
-                        scr[row * NP + q] = make_float4(acc0[q].x, acc0[q].y, acc1[q].x, acc1[q].y);
-                }
-                __syncthreads();
-                if (reader) {
+                for (int q = 0; q < NP; ++q)
+                    scr[((phase - 1) * NP + q) * VC + col[0]] =
+                        make_float4(acc0[q].x, acc0[q].y, acc1[q].x, acc1[q].y);
+            }
+            __syncthreads();
+            if (colok[0] && phase == 0) {
+                for (int ph = 1; ph < RP; ++ph) {
+                    float4 v[NP];
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) v[q] = scr[((ph - 1) * NP + q) * VC + col[0]];
 #pragma unroll
                     for (int q = 0; q < NP; ++q) {
-                        const float4 v = scr[row * NP + q];
-                        acc0[q] = __fadd2_rn(acc0[q], f2(v.x, v.y));
-                        acc1[q] = __fadd2_rn(acc1[q], f2(v.z, v.w));
+                        acc0[q] = __fadd2_rn(acc0[q], f2(v[q].x, v[q].y));
+                        acc1[q] = __fadd2_rn(acc1[q], f2(v[q].z, v[q].w));
                     }
                 }
-                __syncthreads();
             }
         }
+        stamp(6, tid == 0);
         if (active && phase == 0) {
-            const double nb = (double)(u1 - u0);
-            const double inv_nb = 1.0 / nb;
+            // forward: (sum d, sum d^2) around the pivot; backward: (sum dy, sum dy*y)
 #pragma unroll
             for (int k = 0; k < CPT; ++k)
                 if (colok[k])
@@ -533,36 +552,33 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         const int64_t ch = (int64_t)(col[k] * NP + q) * 2;
                         const int i = k * NP + q;
                         double2* dstp = a.part + (int64_t)b * a.C + ch;
-                        if (DIR == 0) {
-                            // (mean, M2) of the CTA from its pivot-shifted sums
-                            const double s1x = acc0[i].x, s1y = acc0[i].y;
-                            dstp[0] = make_double2(fma(s1x, inv_nb, -(double)piv[i].x),
-                                                   fma(-s1x * s1x, inv_nb, (double)acc1[i].x));
-                            dstp[1] = make_double2(fma(s1y, inv_nb, -(double)piv[i].y),
-                                                   fma(-s1y * s1y, inv_nb, (double)acc1[i].y));
-                        } else {
-                            dstp[0] = make_double2(acc0[i].x, acc1[i].x);
-                            dstp[1] = make_double2(acc0[i].y, acc1[i].y);
-                        }
+                        dstp[0] = make_double2(acc0[i].x, acc1[i].x);
+                        dstp[1] = make_double2(acc0[i].y, acc1[i].y);
                     }
         }
     }
     stamp(2, tid == 0);
 
     // ------------------------------------------------- barriers and finalize
-    grid_barrier(a.ctl, a.budget_ns, &s_fail);
+    grid_barrier(a.ctl, bbase + (uint32_t)G, a.budget_ns, &s_fail);
     stamp(3, tid == 0);
+    if (!producer && lane == 0) cp_async_wait_all();   // s_par (issued at launch)
     if (!failed() && !producer) {
         // one consumer warp per channel over the whole grid, fp64, fixed order
         const int64_t nw = (int64_t)G * kConsumerWarps;
         const int64_t K = LAYOUT == kNHWC ? (int64_t)G : a.N;
         constexpr int KC = 5;   // partials cached per lane when K <= 160
         const bool cached = K <= 32 * KC;
-        auto count_at = [&](int64_t k) -> double {
-            return LAYOUT == kNHWC ? (double)((k + 1) * P.units / G - k * P.units / G)
-                                   : (double)a.HW;
+        const double hw = (double)a.HW;   // elements behind each NCHW partial
+        // the pivot x[0, c] from the aligned 32-bit word that holds it
+        auto pivot_of = [&](uint32_t w, int64_t c) -> float {
+            if (DT == kF32) return __uint_as_float(w);
+            const uint32_t h = (c & 1) ? (w >> 16) : (w & 0xffffu);
+            if (DT == kBF16) return __uint_as_float(h << 16);
+            return __half2float(__ushort_as_half((unsigned short)h));
         };
-        for (int64_t c = (int64_t)b * kConsumerWarps + warp; c < a.C; c += nw) {
+        bool first = true;
+        for (int64_t c = (int64_t)b * kConsumerWarps + warp; c < a.C; c += nw, first = false) {
             double2 pk[KC];
             double ck[KC];
 #pragma unroll
@@ -570,40 +586,71 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 const int64_t k = lane + 32 * i;
                 const bool in = cached && k < K;
                 pk[i] = in ? a.part[k * a.C + c] : make_double2(0.0, 0.0);
-                ck[i] = in ? count_at(k) : 0.0;
+                ck[i] = in ? hw : 0.0;
+            }
+            // per-channel parameters (lane 0 uses them)
+            float gmf = 0.f, btf = 0.f, vif = 0.f;
+            if (lane == 0) {
+                if (first) {
+                    gmf = s_par[warp][0];
+                    btf = s_par[warp][1];
+                    vif = s_par[warp][2];
+                } else {
+                    gmf = a.gamma[c];
+                    btf = a.beta[c];
+                    if (DIR == 1) vif = a.var_in[c];
+                    if (DIR == 0 && LAYOUT == kNHWC)
+                        vif = __uint_as_float(*reinterpret_cast<const uint32_t*>(
+                            a.src0 + ((c * (int64_t)sizeof(typename Storage<DT>::T)) & ~int64_t(3))));
+                }
             }
             if (DIR == 0) {
-                double s = 0.0;
-                if (cached) {
-#pragma unroll
-                    for (int i = 0; i < KC; ++i) s += ck[i] * pk[i].x;
-                } else {
-                    for (int64_t k = lane; k < K; k += 32) s += count_at(k) * a.part[k * a.C + c].x;
-                }
-                const double mean = warp_sum(s) / a.M;
-                double q = 0.0;
+                // NHWC partials are sums around the pivot p (mean = p + s1/M,
+                // M2 = s2 - s1^2/M).  NCHW partials are per-plane (mean, M2): one
+                // pass around r, the first plane's mean:
+                //   s1 = sum n (mean_k - r),  s2 = sum M2_k + n (mean_k - r)^2.
+                double r = 0.0;
+                if (LAYOUT == kNCHW)
+                    r = __shfl_sync(0xffffffffu, cached ? pk[0].x : a.part[c].x, 0);
+                double s1 = 0.0, s2 = 0.0;
                 if (cached) {
 #pragma unroll
                     for (int i = 0; i < KC; ++i) {
-                        const double d = pk[i].x - mean;
-                        q += pk[i].y + ck[i] * d * d;
+                        if (LAYOUT == kNHWC) {
+                            s1 += pk[i].x;
+                            s2 += pk[i].y;
+                        } else {
+                            const double w = ck[i] * (pk[i].x - r);
+                            s1 += w;
+                            s2 += pk[i].y + w * (pk[i].x - r);
+                        }
                     }
                 } else {
                     for (int64_t k = lane; k < K; k += 32) {
                         const double2 v = a.part[k * a.C + c];
-                        const double d = v.x - mean;
-                        q += v.y + count_at(k) * d * d;
+                        if (LAYOUT == kNHWC) {
+                            s1 += v.x;
+                            s2 += v.y;
+                        } else {
+                            const double w = hw * (v.x - r);
+                            s1 += w;
+                            s2 += v.y + w * (v.x - r);
+                        }
                     }
                 }
-                const double var = warp_sum(q) / a.M;
+                s1 = warp_sum(s1);
+                s2 = warp_sum(s2);
+                if (LAYOUT == kNHWC && lane == 0) r = (double)pivot_of(__float_as_uint(vif), c);
                 if (lane == 0) {
+                    const double mean = r + s1 / a.M;
+                    const double var = fmax((s2 - s1 * (s1 / a.M)) / a.M, 0.0);
                     a.out0[c] = (float)mean;
                     a.out1[c] = (float)var;
                     const double rstd = 1.0 / sqrt(var + (double)a.eps);
-                    const double sc = (double)a.gamma[c] * rstd;
+                    const double sc = (double)gmf * rstd;
                     // (mean, scale, beta, beta - mean*scale)
-                    a.coef[c] = make_float4((float)mean, (float)sc, a.beta[c],
-                                            (float)((double)a.beta[c] - mean * sc));
+                    a.coef[c] = make_float4((float)mean, (float)sc, btf,
+                                            (float)((double)btf - mean * sc));
                 }
             } else {
                 double s1 = 0.0, sy = 0.0;
@@ -623,8 +670,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 s1 = warp_sum(s1);
                 sy = warp_sum(sy);
                 if (lane == 0) {
-                    const double gm = a.gamma[c], bt = a.beta[c];
-                    const double rstd = 1.0 / sqrt((double)a.var_in[c] + (double)a.eps);
+                    const double gm = gmf, bt = btf;
+                    const double rstd = 1.0 / sqrt((double)vif + (double)a.eps);
                     if (!(fabs(gm) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN
                         atomicOr(&a.ctl->status, kStSingular);
                         const float qnan = __int_as_float(0x7fc00000);
@@ -646,7 +693,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
     }
     stamp(4, tid == 0);
-    grid_barrier(a.ctl, a.budget_ns, &s_fail);
+    if (grid_barrier(a.ctl, bbase + 2u * (uint32_t)G, a.budget_ns, &s_fail) && b == 0 && tid == 0)
+        bar_pad(a.ctl, (uint32_t)G, 2u);
     stamp(5, tid == 0);
 
     // ================================================================ phase B
@@ -841,8 +889,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 if ((loaded >> s) & 1u)
                     mbar_wait(&full[s], ((fiss >> s) & 1u) ^ 1u, a.budget_ns / 4);
         }
-        stamp(8, true);
     }
+    stamp(8, tid == 0);
 }
 
 }  // namespace iabn
