@@ -182,13 +182,18 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int G = P.G;
     // Phase trace: 0 start, 1 phase A done, 2 merged, 3 barrier 1, 4 finalize,
     // 5 barrier 2, 6 in-CTA merge rounds done, 7 last refill issued, 8 consumer
-    // warp 0 done
+    // warp 0 done, 14 the SM's id
     // (%globaltimer ns); 9/10/13 phase A and 11/12/15 phase B SM cycles of
     // consumer warp 0: waiting for tiles / bookkeeping / the row loops.
     auto stamp = [&](int k, bool who) {
         if (a.trace != nullptr && who) a.trace[(size_t)b * kTraceSlots + k] = global_ns();
     };
     stamp(0, tid == 0);
+    if (a.trace != nullptr && tid == 0) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        a.trace[(size_t)b * kTraceSlots + 14] = smid;
+    }
     // Consumer warp 0 also accounts its SM cycles: waiting for tiles vs the
     // rest of the loop, per phase (trace slots 9..12).
     const bool acct = a.trace != nullptr && tid == 0;
