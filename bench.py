@@ -34,6 +34,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elements/s"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# resident kernels on the ResNet-trunk layer, from one ncu capture of
+# `python bench.py --profile 1 --steps 1 --warmup 1` (see
+# profiles/k_resident_resnet_trunk.md).  Reported only while the CUDA sources
+# hash to the value they were captured on; otherwise "traffic" is null.
+NCU_TRAFFIC = {
+    "sources_sha256": "026899106d55b525e976ad606a3a21bac260fb23f6f5bf63947b8535cdef7539",
+    "backward": 320371712 + 35237632,
+    "forward": 117835776 + 21308928,
+}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
@@ -44,6 +54,26 @@ def measured_hbm_gbs():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_sha256() -> str:
+    """sha256 over the CUDA sources of the library (file names and bytes)."""
+    import hashlib
+    d = os.path.join(ROOT, "place_batchnorm_activation_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            with open(os.path.join(d, name), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(direction: str):
+    """Captured DRAM bytes per launch, or None if the kernels changed since."""
+    if kernel_sources_sha256() != NCU_TRAFFIC["sources_sha256"]:
+        return None
+    return NCU_TRAFFIC[direction]
 
 
 def parse_args():
@@ -598,12 +628,14 @@ def main():
             "frac_of_measured_hbm": round(value / world / hbm_peak, 4),
             "roofline": {"bound": "hbm", "kernel": "backward (iabn_backward)",
                          "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                         "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                         "frac": round(achieved / hbm_peak, 4),
+                         "traffic": ncu_traffic("backward"),
                          "peak_source": f"{peak_kind} hbm_gbs",
                          "algorithmic_bytes_per_launch": bwd_bytes},
             "roofline_fwd": {"bound": "hbm", "achieved": round(fwd_achieved, 1),
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(fwd_achieved / hbm_peak, 4),
+                             "traffic": ncu_traffic("forward"),
                              "algorithmic_bytes_per_launch": 2 * sp.numel * sp.itemsize},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e_max, 3)},

@@ -74,3 +74,12 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_ncu_traffic_only_for_captured_sources(monkeypatch):
+    import bench
+    traffic = dict(bench.NCU_TRAFFIC)
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", dict(traffic, sources_sha256=bench.kernel_sources_sha256()))
+    assert bench.ncu_traffic("backward") == traffic["backward"]
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", dict(traffic, sources_sha256="0" * 64))
+    assert bench.ncu_traffic("backward") is None
