@@ -103,6 +103,10 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         P.L = 1;
         // merge: RP-1 row phases x VC columns x one 16-byte float4 per pair
         if (cpt == 1 && P.RP > 1) scratch = (P.RP - 1) * P.VC * (8 / s) * 16;
+        // TMEM stash: 1 KB (64 vectors) per consumer thread; TMEM accesses are
+        // warp-wide, so every warp must hold a single row phase
+        if ((cpt > 1 || P.VC % 32 == 0) && env_long("IABN_TMEM_STASH", 1) != 0)
+            P.stash = 64 / (cpt * NT);
     } else {
         const int64_t pb = g.HW * s;
         const int gq = 16 / gcd_int(pb, 16);
@@ -130,6 +134,8 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     int ring = (int)env_long(dir == 0 ? "IABN_RING_FWD" : "IABN_RING_BWD", 4);
     if (ring < 2) ring = 2;
     if (ring > nslots) return false;
+    if (P.stash > 0) nslots = ring;   // the stash replaces resident tiles
+    P.stash_first = (int)env_long("IABN_STASH_FIRST", 1);
     P.nslots = nslots;
     P.ring = ring;
     P.smem_bytes = kBarBytes + P.scratch_bytes + nslots * P.slot_bytes;

@@ -33,8 +33,11 @@
 // bounded and a timeout sets kStTimeout in the workspace status word.
 #pragma once
 
+#include <climits>
+
 #include "iabn_bulk.cuh"
 #include "iabn_device.cuh"
+#include "iabn_tmem.cuh"
 #include "iabn_internal.h"
 
 namespace iabn {
@@ -60,6 +63,9 @@ struct ResPlan {
     int VC, RP;          // NHWC: 16-byte columns per row; row phases (threads per column)
     int g, L;            // NCHW: planes per unit; lanes per plane
     int hints;           // 1: L2 eviction-priority hints on the bulk copies
+    int stash_first;     // 1: the stash holds each thread's first rows, 0: its last
+    int stash;           // NHWC: rows per consumer thread kept in TMEM from phase A
+                         // to phase B (0: off); all slots then form the ring
 };
 
 struct ResArgs {
@@ -223,6 +229,27 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int ring = P.ring;
     const int D = min(P.nslots - ring, n);
     const int nring = n - D;
+    // TMEM stash (NHWC): every consumer thread keeps Jc of its rows in TMEM --
+    // its first Jc (the CTA's first S = RP*Jc rows, the ones most likely gone
+    // from L2 by phase B) or its last Jc (the CTA's last S rows).  Phase B
+    // streams only the tiles [tlo, thi) that hold other rows, the j-th one
+    // being tile thi-1-j.
+    const bool stash = LAYOUT == kNHWC && P.stash > 0;
+    const bool sfirst = stash && P.stash_first != 0;
+    const int64_t nrows = u1 - u0;
+    const int Jc = stash ? (int)min((int64_t)P.stash, nrows / P.RP) : 0;
+    const int64_t S = (int64_t)P.RP * Jc;
+    int tlo = 0, thi = nring;
+    if (stash) {
+        if (sfirst) {
+            tlo = S >= nrows ? n : (int)(S / P.tile_units);
+            thi = n;
+        } else {
+            thi = (int)((nrows - S + P.tile_units - 1) / P.tile_units);
+        }
+    }
+    const int nB = thi - tlo;
+    __shared__ uint32_t s_tmem;
 
     if (tid == 0) {
         for (int s = 0; s < P.nslots; ++s) {
@@ -246,7 +273,14 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 cp_async4(&s_par[warp][2], a.src0 + ((c * (int64_t)sizeof(typename Storage<DT>::T)) & ~int64_t(3)));
         }
     }
+    if (stash && warp == 0) {
+        __syncwarp();
+        tmem_alloc_all(&s_tmem);
+        tmem_fence_before_sync();
+    }
     __syncthreads();
+    if (stash) tmem_fence_after_sync();
+    const uint32_t tmem_base = stash ? s_tmem : 0u;
 
     auto t_u0 = [&](int t) -> int64_t { return u0 + (int64_t)t * P.tile_units; };
     auto t_nu = [&](int t) -> int {
@@ -304,14 +338,15 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 if (!wait_empty(s)) { set_failed(); break; }
                 used |= 1u << s;
             }
-            issue(t, s, t < nring ? pol_keep : pol_stream);
+            // tiles read again in phase B stay in L2; stashed or resident ones need not
+            issue(t, s, (stash ? t >= tlo && t < thi : t < nring) ? pol_keep : pol_stream);
         }
         // Phase B prefetch into the streamed slots as they free up: the j-th
-        // streamed tile of phase B (tile nring-1-j) goes to slot j % ring.
-        const int pro = min(ring, nring);
+        // streamed tile of phase B (tile thi-1-j) goes to slot j % ring.
+        const int pro = min(ring, nB);
         for (int j = 0; j < pro && !failed(); ++j) {
             if (!wait_empty(j)) { set_failed(); break; }
-            issue(nring - 1 - j, j, pol_stream);
+            issue(thi - 1 - j, j, pol_stream);
         }
     }
 
@@ -368,6 +403,21 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const uint32_t slots_sa = smem_u32(slots);
     // rows of a tile with `rows` rows that this thread handles
     auto my_rows = [&](int rows) -> int { return rows > phase ? (rows - 1 - phase) / RP + 1 : 0; };
+    // Stash: js is the ordinal of this thread's first stashed row (its rows
+    // are phase + RP*j of the CTA's range); stashed row js+i lives at TMEM
+    // columns (i*VPR + v)*4 .. +3 (v: vector of the row) of the thread's lane
+    // in the warp's quadrant, the two warps of a quadrant 256 columns apart.
+    constexpr int VPR = CPT * NT;
+    int js = 0;
+    if (stash && !sfirst) {
+        const int64_t sb0 = nrows - S;
+        int64_t r = ((int64_t)phase - sb0) % RP;
+        if (r < 0) r += RP;
+        js = (int)((sb0 + r - phase) / RP);
+    }
+    const uint32_t tm_thread =
+        tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(256 * ((warp >> 2) & 1));
+    const int tile_ord = P.tile_units / RP;   // row ordinals per tile and thread (NHWC)
     // NCHW mapping: groups of L lanes per plane.
     const int L = P.L;
     const int GP = kConsumers / L;
@@ -425,6 +475,41 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                                 vz[u][k] = lds128(o);
                                 if (DIR == 1) vd[u][k] = lds128(o + (uint32_t)P.half_bytes);
                             }
+                        if (stash) {
+                            // rows from ordinal js on also go to TMEM (warp-uniform:
+                            // a warp's lanes share the row phase): a whole batch as
+                            // one 16/32-column store, else vector by vector
+                            const int ib = t * tile_ord + i0 - js;
+                            const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+                            if (ib >= 0 && ib + RB <= Jc && i0 + RB <= m) {
+                                uint4 w[RB * VPR];
+#pragma unroll
+                                for (int u = 0; u < RB; ++u)
+#pragma unroll
+                                    for (int k = 0; k < CPT; ++k) {
+                                        const bool ok = CPT == 1 || colok[k];
+                                        w[(u * CPT + k) * NT] = ok ? vz[u][k] : z4;
+                                        if (DIR == 1) w[(u * CPT + k) * NT + 1] = ok ? vd[u][k] : z4;
+                                    }
+                                const uint32_t ta = tm_thread + (uint32_t)(ib * VPR * 4);
+                                if (NT == 1) tmem_st16(ta, w);
+                                else tmem_st32(ta, w);
+                            } else {
+#pragma unroll
+                                for (int u = 0; u < RB; ++u) {
+                                    const int i = ib + u;
+                                    if (i0 + u < m && i >= 0 && i < Jc) {
+#pragma unroll
+                                        for (int k = 0; k < CPT; ++k) {
+                                            const uint32_t ta = tm_thread + (uint32_t)((i * VPR + k * NT) * 4);
+                                            const bool ok = CPT == 1 || colok[k];
+                                            tmem_st4(ta, ok ? vz[u][k] : z4);
+                                            if (DIR == 1) tmem_st4(ta + 4, ok ? vd[u][k] : z4);
+                                        }
+                                    }
+                                }
+                            }
+                        }
 #pragma unroll
                         for (int u = 0; u < RB; ++u)
 #pragma unroll
@@ -515,6 +600,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             acct_work();
         }
         acct_flush(9);
+        if (stash) tmem_wait_st();   // this thread's stores land before its phase B loads
     }
     __syncthreads();
     stamp(1, tid == 0);
@@ -710,12 +796,12 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             // j + ring once they are done with tile j.
             uint32_t dpar = 0;
             bool ok = true;
-            for (int j = 0; j + ring < nring && ok; ++j) {
+            for (int j = 0; j + ring < nB && ok; ++j) {
                 const int s = j % ring;
                 ok = mbar_wait(&done[s], (dpar >> s) & 1u, a.budget_ns, a.wait_prod);
                 dpar ^= 1u << s;
                 if (!ok) break;
-                issue(nring - 1 - (j + ring), s, pol_stream);
+                issue(thi - 1 - (j + ring), s, pol_stream);
             }
             if (!ok) set_failed();
             stamp(7, true);
@@ -752,17 +838,70 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 }
             }
         // Rewrites the tile in slot s in place (forward: x -> z; backward: dz -> dx).
-        auto apply_tile = [&](int t, int s) {
+        // Rewrites one row's CPT vectors: forward x -> z in vz, backward
+        // dz -> dx in vd (z in vz).
+        auto rewrite = [&](uint4* vz, uint4* vd) {
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                if (CPT > 1 && !colok[k]) continue;
+                if (DIR == 0) {
+                    float2 f[NP];
+                    Pairs<DT>::unpack(vz[k], f);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const int j = k * NP + q;
+                        // 16-bit storage: y = x*scale + (beta - mean*scale); its
+                        // rounding error is far below one storage ulp.  fp32:
+                        // y = (x - mean)*scale + beta.
+                        const float2 y = DT == kF32 ? __ffma2_rn(__fadd2_rn(f[q], c0[j]), c1[j], c2[j])
+                                                    : __ffma2_rn(f[q], c1[j], c2[j]);
+                        f[q] = act_forward2<ACT, DT>(y, p, le1);
+                    }
+                    vz[k] = Pairs<DT>::pack(f);
+                } else {
+                    float2 fz[NP], fd[NP];
+                    Pairs<DT>::unpack(vz[k], fz);
+                    Pairs<DT>::unpack(vd[k], fd);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const int j = k * NP + q;
+                        if (ACT == kLeaky) {
+                            // dx = A dy + B y + Cc with (dy, y) = (dz, z) for z > 0
+                            // and (a dz, z/a) otherwise
+                            const bool px = fz[q].x > 0.f, py = fz[q].y > 0.f;
+                            const float2 a3 = CPT == 1 ? c3[j < NQ34 ? j : 0]
+                                                       : __fmul2_rn(c0[j], f2(p, p));
+                            const float2 a4 = CPT == 1 ? c4[j < NQ34 ? j : 0]
+                                                       : __fmul2_rn(c1[j], f2(inv_p, inv_p));
+                            const float2 Ak = f2(px ? c0[j].x : a3.x, py ? c0[j].y : a3.y);
+                            const float2 Bk = f2(px ? c1[j].x : a4.x, py ? c1[j].y : a4.y);
+                            fd[q] = __ffma2_rn(Ak, fd[q], __ffma2_rn(Bk, fz[q], c2[j]));
+                        } else if (ACT == kIdent) {
+                            fd[q] = __ffma2_rn(c0[j], fd[q], __ffma2_rn(c1[j], fz[q], c2[j]));
+                        } else {
+                            float y0, y1, d0, d1;
+                            act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0, d0);
+                            act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1, d1);
+                            fd[q] = __ffma2_rn(c0[j], f2(d0, d1), __ffma2_rn(c1[j], f2(y0, y1), c2[j]));
+                        }
+                    }
+                    vd[k] = Pairs<DT>::pack(fd);
+                }
+            }
+        };
+        // Rewrites the tile in slot s -- this thread's rows q in [qlo, qhi) of
+        // it -- and writes the results to global memory.
+        auto apply_tile = [&](int t, int s, int qlo, int qhi) {
             unsigned char* base = slot_ptr(s);
             if (LAYOUT == kNHWC) {
                 const int rows = t_nu(t);
                 if (!active) return;
-                const int m = my_rows(rows);
+                const int m = min(my_rows(rows), qhi);
                 const uint32_t sb = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
                 const uint32_t hb = DIR == 0 ? 0u : (uint32_t)P.half_bytes;
                 unsigned char* gtile = a.dst + t_u0(t) * P.unit_bytes;
                 // rows in batches of RB: loads, then math, then stores
-                for (int i0 = 0; i0 < m; i0 += RB) {
+                for (int i0 = max(qlo, 0); i0 < m; i0 += RB) {
                     uint4 vz[RB][CPT], vd[RB][CPT];
 #pragma unroll
                     for (int u = 0; u < RB; ++u)
@@ -775,61 +914,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         }
 #pragma unroll
                     for (int u = 0; u < RB; ++u)
-#pragma unroll
-                        for (int k = 0; k < CPT; ++k) {
-                            if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
-                            if (DIR == 0) {
-                                float2 f[NP];
-                                Pairs<DT>::unpack(vz[u][k], f);
-#pragma unroll
-                                for (int q = 0; q < NP; ++q) {
-                                    const int j = k * NP + q;
-                                    // 16-bit storage: y = x*scale + (beta - mean*scale); its
-                                    // rounding error is far below one storage ulp.  fp32:
-                                    // y = (x - mean)*scale + beta.
-                                    const float2 y =
-                                        DT == kF32 ? __ffma2_rn(__fadd2_rn(f[q], c0[j]), c1[j], c2[j])
-                                                   : __ffma2_rn(f[q], c1[j], c2[j]);
-                                    f[q] = act_forward2<ACT, DT>(y, p, le1);
-                                }
-                                vz[u][k] = Pairs<DT>::pack(f);
-                            } else {
-                                float2 fz[NP], fd[NP];
-                                Pairs<DT>::unpack(vz[u][k], fz);
-                                Pairs<DT>::unpack(vd[u][k], fd);
-#pragma unroll
-                                for (int q = 0; q < NP; ++q) {
-                                    const int j = k * NP + q;
-                                    if (ACT == kLeaky) {
-                                        // dx = A dy + B y + Cc with (dy, y) = (dz, z) for z > 0
-                                        // and (a dz, z/a) otherwise
-                                        const bool px = fz[q].x > 0.f, py = fz[q].y > 0.f;
-                                        const float2 a3 = CPT == 1
-                                                              ? c3[j < NQ34 ? j : 0]
-                                                              : __fmul2_rn(c0[j], f2(p, p));
-                                        const float2 a4 =
-                                            CPT == 1 ? c4[j < NQ34 ? j : 0]
-                                                     : __fmul2_rn(c1[j], f2(inv_p, inv_p));
-                                        const float2 Ak = f2(px ? c0[j].x : a3.x,
-                                                             py ? c0[j].y : a3.y);
-                                        const float2 Bk = f2(px ? c1[j].x : a4.x,
-                                                             py ? c1[j].y : a4.y);
-                                        fd[q] = __ffma2_rn(Ak, fd[q],
-                                                           __ffma2_rn(Bk, fz[q], c2[j]));
-                                    } else if (ACT == kIdent) {
-                                        fd[q] = __ffma2_rn(c0[j], fd[q],
-                                                           __ffma2_rn(c1[j], fz[q], c2[j]));
-                                    } else {
-                                        float y0, y1, d0, d1;
-                                        act_backward<ACT, DT>(fz[q].x, fd[q].x, p, inv_p, y0, d0);
-                                        act_backward<ACT, DT>(fz[q].y, fd[q].y, p, inv_p, y1, d1);
-                                        fd[q] = __ffma2_rn(c0[j], f2(d0, d1),
-                                                           __ffma2_rn(c1[j], f2(y0, y1), c2[j]));
-                                    }
-                                }
-                                vd[u][k] = Pairs<DT>::pack(fd);
-                            }
-                        }
+                        if (i0 + u < m) rewrite(vz[u], vd[u]);
                     // results go straight to their place in global memory
 #pragma unroll
                     for (int u = 0; u < RB; ++u)
@@ -866,17 +951,47 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             }
         };
         acct_start();
+        if (stash && active) {
+            // the stashed rows first: no wait for any tile
+            unsigned char* grow = a.dst + u0 * P.unit_bytes;
+            for (int i0 = 0; i0 < Jc; i0 += RB) {
+                uint4 buf[RB * VPR];   // RB*CPT = 4 vectors per tensor
+                if (NT == 1) tmem_ld16(tm_thread + (uint32_t)(i0 * VPR * 4), buf);
+                else tmem_ld32(tm_thread + (uint32_t)(i0 * VPR * 4), buf);
+#pragma unroll
+                for (int u = 0; u < RB; ++u) {
+                    if (i0 + u >= Jc) continue;
+                    uint4 vz[CPT], vd[CPT];
+#pragma unroll
+                    for (int k = 0; k < CPT; ++k) {
+                        vz[k] = buf[(u * CPT + k) * NT];
+                        vd[k] = buf[(u * CPT + k) * NT + (NT - 1)];
+                    }
+                    rewrite(vz, vd);
+                    const size_t j = (size_t)(js + i0 + u);
+#pragma unroll
+                    for (int k = 0; k < CPT; ++k) {
+                        if (CPT > 1 && !colok[k]) continue;
+                        stg128(grow + voff[k] + j * vstep, DIR == 0 ? vz[k] : vd[k]);
+                    }
+                }
+            }
+        }
         for (int t = n - 1; t >= nring; --t) {
             const int s = ring + (t - nring);
-            apply_tile(t, s);
+            apply_tile(t, s, 0, INT_MAX);
             release(&done[s]);
         }
         acct_work();
-        for (int j = 0; j < nring; ++j) {
+        for (int j = 0; j < nB; ++j) {
             const int s = j % ring;
             if (!cwait(s)) break;
             acct_wait();
-            apply_tile(nring - 1 - j, s);
+            const int t = thi - 1 - j;
+            // skip the stashed rows: ordinals [js, js + Jc)
+            const int qlo = stash && sfirst ? Jc - t * tile_ord : 0;
+            const int qhi = stash && !sfirst ? js - t * tile_ord : INT_MAX;
+            apply_tile(t, s, qlo, qhi);
             acct_comp();
             release(&done[s]);
             acct_work();
@@ -896,6 +1011,16 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
     }
     stamp(8, tid == 0);
+    if (stash) {
+        // every TMEM load of the CTA has completed (each waits in place)
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
+        if (warp == 0) {
+            __syncwarp();
+            tmem_free_all(tmem_base);
+        }
+    }
 }
 
 }  // namespace iabn

@@ -174,3 +174,42 @@ def test_singular_gamma(plan):
         assert np.isfinite(np.delete(dx, 2, axis=1)).all()
         dg = L.dgamma.cpu().numpy()
         assert np.isnan(dg[2]) and np.isfinite(np.delete(dg, 2)).all()
+
+
+STASH_CASES = [
+    # NHWC shapes whose resident plan keeps rows in Tensor Memory
+    (8, 256, 14, 14, wl.BF16, wl.LEAKY_RELU, 0.01),   # 8 row phases, full stash
+    (4, 512, 9, 9, wl.BF16, wl.ELU, 1.0),             # 4 row phases
+    (3, 128, 10, 10, wl.F32, wl.LEAKY_RELU, 0.2),     # fp32, 8 row phases
+    (6, 768, 7, 7, wl.BF16, wl.IDENTITY, 0.0),        # 2 row phases, two idle warps
+    (2, 4096, 5, 5, wl.BF16, wl.LEAKY_RELU, 0.01),    # 2 columns per thread
+    (8, 4104, 3, 3, wl.F16, wl.ELU, 1.0),             # 4 columns per thread, ragged
+    (64, 256, 8, 8, wl.BF16, wl.LEAKY_RELU, 0.01),    # ~28 rows per CTA: partial stash
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", STASH_CASES, ids=lambda c: "x".join(map(str, c[:4])))
+def test_tmem_stash_bitwise(case, monkeypatch):
+    """Rows kept in Tensor Memory give the same bits as rows streamed back
+    through L2 (the stash only changes where phase B reads them from), and
+    both match the oracle."""
+    n, c, h, w, dtype, act, p = case
+    sp = wl.LayerSpec("stash", n, c, h, w, wl.NHWC, dtype, act, p, seed=4242 + c + n)
+    inp = wl.draw(sp)
+    outs = {}
+    for on in ("1", "0"):
+        monkeypatch.setenv("IABN_TMEM_STASH", on)
+        with forced_plan("resident"):
+            L = GpuLayer(inp)
+            L.forward()
+            L.backward()
+            torch.cuda.synchronize()
+            assert L.status() == 0
+            outs[on] = [wl.torch_to_storage(L.x, sp.dtype), wl.torch_to_storage(L.dz, sp.dtype),
+                        L.mean.cpu().numpy(), L.var.cpu().numpy(), L.dgamma.cpu().numpy(),
+                        L.dbeta.cpu().numpy()]
+    for a, b in zip(outs["1"], outs["0"]):
+        np.testing.assert_array_equal(a, b)
+    monkeypatch.setenv("IABN_TMEM_STASH", "1")
+    check_layer(inp, oracle_expect(inp), "resident", running=False)
