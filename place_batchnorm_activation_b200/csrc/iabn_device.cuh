@@ -77,8 +77,10 @@ template <int ACT, int DT>
 __device__ __forceinline__ float act_forward(float y, float p) {
     if (ACT == kLeaky) return y > 0.f ? y : p * y;
     if (ACT == kElu) {
-        if (y > 0.f) return y;
-        return DT == kF32 ? p * expm1f(y) : p * (__expf(y) - 1.f);
+        if (DT == kF32) return y > 0.f ? y : p * expm1f(y);
+        // 16-bit storage: both branches, then a select (no divergence)
+        const float e = p * (__expf(fminf(y, 0.f)) - 1.f);
+        return y > 0.f ? y : e;
     }
     return y;
 }
@@ -92,18 +94,22 @@ __device__ __forceinline__ void act_backward(float z, float dz, float p, float i
         y = pos ? z : z * inv_p;
         dy = pos ? dz : dz * p;
     } else if (ACT == kElu) {
-        if (z > 0.f) {
-            y = z;
-            dy = dz;
-        } else {
-            const float t = z * inv_p;
-            const float u = 1.f + t;
-            if (u <= kEluFloorU) {
-                y = kEluFloorY;
+        if (DT == kF32) {
+            if (z > 0.f) {
+                y = z;
+                dy = dz;
             } else {
-                y = DT == kF32 ? log1pf(t) : __logf(u);
+                const float t = z * inv_p;
+                y = 1.f + t <= kEluFloorU ? kEluFloorY : log1pf(t);
+                dy = dz * fmaxf(z + p, 0.f);   // phi'(y) = alpha*e^y = z + alpha
             }
-            dy = dz * fmaxf(z + p, 0.f);   // phi'(y) = alpha*e^y = z + alpha
+        } else {
+            // 16-bit storage: both branches, then selects (no divergence)
+            const float u = 1.f + z * inv_p;
+            const float yn = u <= kEluFloorU ? kEluFloorY : __logf(fmaxf(u, kEluFloorU));
+            const bool pos = z > 0.f;
+            y = pos ? z : yn;
+            dy = pos ? dz : dz * fmaxf(z + p, 0.f);
         }
     } else {
         y = z;

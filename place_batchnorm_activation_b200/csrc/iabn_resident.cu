@@ -26,6 +26,8 @@
 
 #include <mutex>
 
+#include <algorithm>
+
 #include "iabn_resident.cuh"
 
 namespace iabn {
@@ -118,8 +120,11 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         int tu = target / P.unit_bytes;
         P.tile_units = tu < 1 ? 1 : tu;
         P.g = gq;
+        // lanes per plane: one for small planes (no shuffles; the CTA's 256
+        // threads take 256 planes at once), else enough for ~8 elements each
         int L = 1;
-        while (L < 32 && L * 8 < g.HW) L *= 2;
+        if (g.HW > 64)
+            while (L < 32 && L * 8 < g.HW) L *= 2;
         P.L = L;
         P.VC = 1;
         P.RP = 1;
@@ -127,12 +132,25 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     P.tile_bytes = P.tile_units * P.unit_bytes;
     P.half_bytes = round_up_int(P.tile_bytes, 128);
     P.slot_bytes = P.half_bytes * NT;
+    int ring = (int)env_long(dir == 0 ? "IABN_RING_FWD" : "IABN_RING_BWD", 4);
+    if (ring < 2) ring = 2;
+    if (g.layout == kNCHW) {
+        // phase B coefficients of the CTA's channel window, if they fit next to
+        // the ring: min(C, planes of the largest CTA range) float4s
+        const int64_t G0 = g.N * g.C / P.g < dl.sms ? g.N * g.C / P.g : dl.sms;
+        const int64_t planes = (P.units + G0 - 1) / G0 * P.g;
+        const int64_t w = planes < g.C ? planes : g.C;
+        const int64_t bytes = round_up_int((int)std::min<int64_t>(w * 16, 1 << 20), 128);
+        if (env_long("IABN_NCHW_SMEM_COEF", 1) != 0 &&
+            1024 + kBarBytes + bytes + (int64_t)ring * P.slot_bytes <= dl.smem_optin) {
+            P.ncoef = (int)w;
+            scratch = (int)bytes;
+        }
+    }
     P.scratch_bytes = round_up_int(scratch, 128);
     const int budget = dl.smem_optin - 1024 - kBarBytes - P.scratch_bytes;
     int nslots = budget / P.slot_bytes;
     if (nslots > kMaxSlots) nslots = kMaxSlots;
-    int ring = (int)env_long(dir == 0 ? "IABN_RING_FWD" : "IABN_RING_BWD", 4);
-    if (ring < 2) ring = 2;
     if (ring > nslots) return false;
     if (P.stash > 0) nslots = ring;   // the stash replaces resident tiles
     P.stash_first = (int)env_long("IABN_STASH_FIRST", 1);

@@ -58,12 +58,15 @@ struct ResPlan {
     int slot_bytes;      // half_bytes * tensors per tile
     int nslots;          // slots in shared memory
     int ring;            // slots cycled by the stream; the rest hold resident tiles
-    int scratch_bytes;   // shared memory for the per-CTA merge (NHWC), multiple of 128
+    int scratch_bytes;   // shared memory for the per-CTA merge (NHWC) or the phase B
+                         // coefficients (NCHW), multiple of 128
     int smem_bytes;      // dynamic shared memory of the launch
     int VC, RP;          // NHWC: 16-byte columns per row; row phases (threads per column)
     int g, L;            // NCHW: planes per unit; lanes per plane
     int hints;           // 1: L2 eviction-priority hints on the bulk copies
     int stash_first;     // 1: the stash holds each thread's first rows, 0: its last
+    int ncoef;           // NCHW: channels of the CTA's coefficient window kept in shared
+                         // memory (scratch) for phase B; 0: read from global memory
     int stash;           // NHWC: rows per consumer thread kept in TMEM from phase A
                          // to phase B (0: off); all slots then form the ring
 };
@@ -148,6 +151,26 @@ template <> struct Pairs<kF16> {
 };
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// 16 bytes <-> the 16/s consecutive elements they hold, as floats.
+template <int DT>
+__device__ __forceinline__ void unpack_all(const uint4& v, float* x) {
+    float2 f[Pairs<DT>::NP];
+    Pairs<DT>::unpack(v, f);
+#pragma unroll
+    for (int q = 0; q < Pairs<DT>::NP; ++q) {
+        x[2 * q] = f[q].x;
+        x[2 * q + 1] = f[q].y;
+    }
+}
+
+template <int DT>
+__device__ __forceinline__ uint4 pack_all(const float* x) {
+    float2 f[Pairs<DT>::NP];
+#pragma unroll
+    for (int q = 0; q < Pairs<DT>::NP; ++q) f[q] = make_float2(x[2 * q], x[2 * q + 1]);
+    return Pairs<DT>::pack(f);
+}
 
 // Forward activation on a pair (leaky with slope <= 1 is max(y, a*y), with
 // slope > 1 it is min(y, a*y)).
@@ -425,6 +448,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int HW = (int)a.HW;
     const int pbytes = HW * (int)sizeof(typename Storage<DT>::T);
     const float inv_hw = 1.f / (float)HW;
+    const double inv_hw_d = 1.0 / (double)HW;
     const float p = a.p, inv_p = a.inv_p;
     const bool le1 = p <= 1.f;
 
@@ -565,33 +589,95 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     const int pp = bp + grp;
                     const bool valid = pp < np;
                     const unsigned char* pz = base + (size_t)pp * pbytes;
-                    if (DIR == 0) {
-                        float sum = 0.f;
-                        if (valid)
-                            for (int i = glane; i < HW; i += L) sum += Elem<DT>::ld(pz, i);
-                        const float mean = group_sum(sum, L) * inv_hw;
-                        float sq = 0.f;
-                        if (valid)
-                            for (int i = glane; i < HW; i += L) {
-                                const float d = Elem<DT>::ld(pz, i) - mean;
-                                sq = fmaf(d, d, sq);
-                            }
-                        sq = group_sum(sq, L);
-                        if (valid && glane == 0) a.part[plane0 + pp] = make_double2(mean, sq);
-                    } else {
-                        float s1 = 0.f, sy = 0.f;
+                    // two independent accumulator chains per lane (elements
+                    // i and i+L of each step), added at the end
+                    if (DIR == 0 && DT == kF32) {
+                        // fp32 storage: exact two passes, mean then M2
+                        float sa = 0.f, sb = 0.f;
                         if (valid) {
-                            const unsigned char* pd = pz + P.half_bytes;
-                            for (int i = glane; i < HW; i += L) {
-                                float y, dy;
-                                act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
-                                                      inv_p, y, dy);
-                                s1 += dy;
-                                sy = fmaf(dy, y, sy);
+                            int i = glane;
+#pragma unroll 4
+                            for (; i + L < HW; i += 2 * L) {
+                                sa += Elem<DT>::ld(pz, i);
+                                sb += Elem<DT>::ld(pz, i + L);
+                            }
+                            if (i < HW) sa += Elem<DT>::ld(pz, i);
+                        }
+                        const float mean = group_sum(sa + sb, L) * inv_hw;
+                        float qa = 0.f, qb = 0.f;
+                        if (valid) {
+                            int i = glane;
+#pragma unroll 4
+                            for (; i + L < HW; i += 2 * L) {
+                                const float da = Elem<DT>::ld(pz, i) - mean;
+                                const float db = Elem<DT>::ld(pz, i + L) - mean;
+                                qa = fmaf(da, da, qa);
+                                qb = fmaf(db, db, qb);
+                            }
+                            if (i < HW) {
+                                const float da = Elem<DT>::ld(pz, i) - mean;
+                                qa = fmaf(da, da, qa);
                             }
                         }
-                        s1 = group_sum(s1, L);
-                        sy = group_sum(sy, L);
+                        const float sq = group_sum(qa + qb, L);
+                        if (valid && glane == 0) a.part[plane0 + pp] = make_double2(mean, sq);
+                    } else if (DIR == 0) {
+                        // 16-bit storage: one pass around the plane's first element
+                        // k: mean = k + S1/HW, M2 = S2 - S1^2/HW
+                        float s1a = 0.f, s2a = 0.f, s1b = 0.f, s2b = 0.f, piv = 0.f;
+                        if (valid) {
+                            piv = Elem<DT>::ld(pz, 0);
+                            int i = glane;
+#pragma unroll 4
+                            for (; i + L < HW; i += 2 * L) {
+                                const float da = Elem<DT>::ld(pz, i) - piv;
+                                const float db = Elem<DT>::ld(pz, i + L) - piv;
+                                s1a += da;
+                                s2a = fmaf(da, da, s2a);
+                                s1b += db;
+                                s2b = fmaf(db, db, s2b);
+                            }
+                            if (i < HW) {
+                                const float da = Elem<DT>::ld(pz, i) - piv;
+                                s1a += da;
+                                s2a = fmaf(da, da, s2a);
+                            }
+                        }
+                        const float s1 = group_sum(s1a + s1b, L);
+                        const float s2 = group_sum(s2a + s2b, L);
+                        if (valid && glane == 0) {
+                            const double d1 = s1;
+                            a.part[plane0 + pp] =
+                                make_double2((double)piv + d1 * (double)inv_hw_d,
+                                             (double)s2 - d1 * d1 * (double)inv_hw_d);
+                        }
+                    } else {
+                        float s1a = 0.f, sya = 0.f, s1b = 0.f, syb = 0.f;
+                        if (valid) {
+                            const unsigned char* pd = pz + P.half_bytes;
+                            int i = glane;
+#pragma unroll 4
+                            for (; i + L < HW; i += 2 * L) {
+                                float ya, dya, yb, dyb;
+                                act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
+                                                      inv_p, ya, dya);
+                                act_backward<ACT, DT>(Elem<DT>::ld(pz, i + L),
+                                                      Elem<DT>::ld(pd, i + L), p, inv_p, yb, dyb);
+                                s1a += dya;
+                                sya = fmaf(dya, ya, sya);
+                                s1b += dyb;
+                                syb = fmaf(dyb, yb, syb);
+                            }
+                            if (i < HW) {
+                                float ya, dya;
+                                act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
+                                                      inv_p, ya, dya);
+                                s1a += dya;
+                                sya = fmaf(dya, ya, sya);
+                            }
+                        }
+                        const float s1 = group_sum(s1a + s1b, L);
+                        const float sy = group_sum(sya + syb, L);
                         if (valid && glane == 0) a.part[plane0 + pp] = make_double2(s1, sy);
                     }
                 }
@@ -786,6 +872,18 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     stamp(4, tid == 0);
     if (grid_barrier(a.ctl, bbase + 2u * (uint32_t)G, a.budget_ns, &s_fail) && b == 0 && tid == 0)
         bar_pad(a.ctl, (uint32_t)G, 2u);
+    // NCHW: the coefficients of the CTA's channel window, (u0*g + i) mod C for
+    // i < ncoef, into shared memory (every thread reaches the barrier)
+    const int64_t ch0 = LAYOUT == kNCHW ? (u0 * P.g) % a.C : 0;
+    float4* scoef = reinterpret_cast<float4*>(scratch);
+    if (LAYOUT == kNCHW && P.ncoef > 0) {
+        if (!producer && !failed())
+            for (int i = tid; i < P.ncoef; i += kConsumers) {
+                const int64_t c = ch0 + i;
+                scoef[i] = a.coef[c >= a.C ? c - a.C : c];
+            }
+        __syncthreads();
+    }
     stamp(5, tid == 0);
 
     // ================================================================ phase B
@@ -926,27 +1024,69 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         }
                 }
             } else {
-                const int np = t_nu(t) * P.g;
-                const int64_t plane0 = t_u0(t) * P.g;
-                const uint32_t cbase = (uint32_t)((uint64_t)plane0 % (uint64_t)a.C);
-                for (int pp = grp; pp < np; pp += GP) {
-                    const uint32_t c = (cbase + (uint32_t)pp) % (uint32_t)a.C;
-                    const float4 q = __ldg(a.coef + c);
-                    const unsigned char* pz = base + (size_t)pp * pbytes;
-                    unsigned char* gz = a.dst + (t_u0(t) * P.g + pp) * (int64_t)pbytes;
-                    if (DIR == 0) {
-                        for (int i = glane; i < HW; i += L)
-                            Elem<DT>::st(gz, i, act_forward<ACT, DT>(
-                                                    fmaf(Elem<DT>::ld(pz, i) - q.x, q.y, q.z), p));
-                    } else {
-                        const unsigned char* pd = pz + P.half_bytes;
-                        for (int i = glane; i < HW; i += L) {
+                // NCHW: 16-byte vectors of the tile.  An element's plane (and so
+                // its channel) follows from its index in the tile; the
+                // coefficients switch at plane boundaries.  128-bit global stores.
+                constexpr int EPV = 16 / (int)sizeof(typename Storage<DT>::T);
+                const int nvec = t_nu(t) * (P.unit_bytes / 16);
+                const uint32_t C32 = (uint32_t)a.C, hw = (uint32_t)HW;
+                // window index of the tile's first plane (channel = ch0 + index mod C)
+                const uint32_t ibase = (uint32_t)(((t_u0(t) - u0) * P.g) % a.C);
+                const uint32_t sbv = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
+                auto coef_at = [&](uint32_t i) -> float4 {
+                    if (P.ncoef > 0) return scoef[i];
+                    const int64_t c = ch0 + i;
+                    return a.coef[c >= a.C ? c - a.C : c];
+                };
+                unsigned char* gt = a.dst + t_u0(t) * P.unit_bytes;
+                for (int v = tid; v < nvec; v += kConsumers) {
+                    const uint32_t e0 = (uint32_t)v * EPV;
+                    // e0 / HW: e0 < 2^24, so the float quotient is off by at most one
+                    uint32_t pl = (uint32_t)((float)e0 * inv_hw);
+                    if (pl * hw > e0) --pl;
+                    if ((pl + 1u) * hw <= e0) ++pl;
+                    uint32_t rem = (pl + 1u) * hw - e0;   // elements of plane pl from e0 on
+                    uint32_t c = (ibase + pl) % C32;
+                    const uint4 vz = lds128(sbv + (uint32_t)v * 16u);
+                    uint4 vd = vz;
+                    if (DIR == 1) vd = lds128(sbv + (uint32_t)P.half_bytes + (uint32_t)v * 16u);
+                    float xz[EPV], xd[EPV];
+                    unpack_all<DT>(vz, xz);
+                    if (DIR == 1) unpack_all<DT>(vd, xd);
+                    auto rewrite_elem = [&](int k, const float4& q) {
+                        if (DIR == 0) {
+                            xz[k] = act_forward<ACT, DT>(fmaf(xz[k] - q.x, q.y, q.z), p);
+                        } else {
                             float y, dy;
-                            act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
-                                                  inv_p, y, dy);
-                            Elem<DT>::st(gz, i, fmaf(q.x, dy, fmaf(q.y, y, q.z)));
+                            act_backward<ACT, DT>(xz[k], xd[k], p, inv_p, y, dy);
+                            xz[k] = fmaf(q.x, dy, fmaf(q.y, y, q.z));
+                        }
+                    };
+                    if (hw >= (uint32_t)EPV) {
+                        // planes at least a vector long: two coefficient sets at
+                        // most, chosen per element without branches
+                        const float4 q0 = coef_at(c), q1 = coef_at(c + 1u == C32 ? 0u : c + 1u);
+#pragma unroll
+                        for (int k = 0; k < EPV; ++k) {
+                            const bool first = (uint32_t)k < rem;
+                            const float4 q = make_float4(first ? q0.x : q1.x, first ? q0.y : q1.y,
+                                                         first ? q0.z : q1.z, 0.f);
+                            rewrite_elem(k, q);
+                        }
+                    } else {
+                        float4 q = coef_at(c);
+#pragma unroll
+                        for (int k = 0; k < EPV; ++k) {
+                            if (rem == 0u) {
+                                c = c + 1u == C32 ? 0u : c + 1u;
+                                q = coef_at(c);
+                                rem = hw;
+                            }
+                            --rem;
+                            rewrite_elem(k, q);
                         }
                     }
+                    stg128(gt + (size_t)v * 16, pack_all<DT>(xz));
                 }
             }
         };
