@@ -536,6 +536,10 @@ def run_profile(args):
             torch.cuda.synchronize()
             tr = layer.ws[256:256 + 32768].view(torch.int64).view(256, 16).cpu()
             rows = [r for r in tr.tolist() if r[0] != 0]
+            if not rows:
+                print(f"trace {sp.name} {what}: no resident-kernel stamps (two-phase plan)",
+                      flush=True)
+                continue
             t0 = min(r[0] for r in rows)
             parts = []
             for k, nm in enumerate(names):

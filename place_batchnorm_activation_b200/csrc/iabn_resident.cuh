@@ -589,34 +589,45 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     const int pp = bp + grp;
                     const bool valid = pp < np;
                     const unsigned char* pz = base + (size_t)pp * pbytes;
-                    // two independent accumulator chains per lane (elements
-                    // i and i+L of each step), added at the end
+                    // Elements i = glane + L*j of the plane, in chunks of PC: the
+                    // chunk's loads first, then its math into two accumulator
+                    // chains (even / odd k), then the remainder into chain 0.
+                    constexpr int PC = 8;
+                    auto lim = [&]() { return HW - (PC - 1) * L; };   // chunk start bound
                     if (DIR == 0 && DT == kF32) {
                         // fp32 storage: exact two passes, mean then M2
                         float sa = 0.f, sb = 0.f;
                         if (valid) {
                             int i = glane;
-#pragma unroll 4
-                            for (; i + L < HW; i += 2 * L) {
-                                sa += Elem<DT>::ld(pz, i);
-                                sb += Elem<DT>::ld(pz, i + L);
+                            for (; i < lim(); i += PC * L) {
+                                float x[PC];
+#pragma unroll
+                                for (int k = 0; k < PC; ++k) x[k] = Elem<DT>::ld(pz, i + k * L);
+#pragma unroll
+                                for (int k = 0; k < PC; k += 2) {
+                                    sa += x[k];
+                                    sb += x[k + 1];
+                                }
                             }
-                            if (i < HW) sa += Elem<DT>::ld(pz, i);
+                            for (; i < HW; i += L) sa += Elem<DT>::ld(pz, i);
                         }
                         const float mean = group_sum(sa + sb, L) * inv_hw;
                         float qa = 0.f, qb = 0.f;
                         if (valid) {
                             int i = glane;
-#pragma unroll 4
-                            for (; i + L < HW; i += 2 * L) {
-                                const float da = Elem<DT>::ld(pz, i) - mean;
-                                const float db = Elem<DT>::ld(pz, i + L) - mean;
-                                qa = fmaf(da, da, qa);
-                                qb = fmaf(db, db, qb);
+                            for (; i < lim(); i += PC * L) {
+                                float x[PC];
+#pragma unroll
+                                for (int k = 0; k < PC; ++k) x[k] = Elem<DT>::ld(pz, i + k * L) - mean;
+#pragma unroll
+                                for (int k = 0; k < PC; k += 2) {
+                                    qa = fmaf(x[k], x[k], qa);
+                                    qb = fmaf(x[k + 1], x[k + 1], qb);
+                                }
                             }
-                            if (i < HW) {
-                                const float da = Elem<DT>::ld(pz, i) - mean;
-                                qa = fmaf(da, da, qa);
+                            for (; i < HW; i += L) {
+                                const float d = Elem<DT>::ld(pz, i) - mean;
+                                qa = fmaf(d, d, qa);
                             }
                         }
                         const float sq = group_sum(qa + qb, L);
@@ -628,19 +639,22 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         if (valid) {
                             piv = Elem<DT>::ld(pz, 0);
                             int i = glane;
-#pragma unroll 4
-                            for (; i + L < HW; i += 2 * L) {
-                                const float da = Elem<DT>::ld(pz, i) - piv;
-                                const float db = Elem<DT>::ld(pz, i + L) - piv;
-                                s1a += da;
-                                s2a = fmaf(da, da, s2a);
-                                s1b += db;
-                                s2b = fmaf(db, db, s2b);
+                            for (; i < lim(); i += PC * L) {
+                                float x[PC];
+#pragma unroll
+                                for (int k = 0; k < PC; ++k) x[k] = Elem<DT>::ld(pz, i + k * L) - piv;
+#pragma unroll
+                                for (int k = 0; k < PC; k += 2) {
+                                    s1a += x[k];
+                                    s2a = fmaf(x[k], x[k], s2a);
+                                    s1b += x[k + 1];
+                                    s2b = fmaf(x[k + 1], x[k + 1], s2b);
+                                }
                             }
-                            if (i < HW) {
-                                const float da = Elem<DT>::ld(pz, i) - piv;
-                                s1a += da;
-                                s2a = fmaf(da, da, s2a);
+                            for (; i < HW; i += L) {
+                                const float d = Elem<DT>::ld(pz, i) - piv;
+                                s1a += d;
+                                s2a = fmaf(d, d, s2a);
                             }
                         }
                         const float s1 = group_sum(s1a + s1b, L);
@@ -656,19 +670,25 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         if (valid) {
                             const unsigned char* pd = pz + P.half_bytes;
                             int i = glane;
-#pragma unroll 4
-                            for (; i + L < HW; i += 2 * L) {
-                                float ya, dya, yb, dyb;
-                                act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
-                                                      inv_p, ya, dya);
-                                act_backward<ACT, DT>(Elem<DT>::ld(pz, i + L),
-                                                      Elem<DT>::ld(pd, i + L), p, inv_p, yb, dyb);
-                                s1a += dya;
-                                sya = fmaf(dya, ya, sya);
-                                s1b += dyb;
-                                syb = fmaf(dyb, yb, syb);
+                            for (; i < lim(); i += PC * L) {
+                                float zv[PC], dv[PC];
+#pragma unroll
+                                for (int k = 0; k < PC; ++k) {
+                                    zv[k] = Elem<DT>::ld(pz, i + k * L);
+                                    dv[k] = Elem<DT>::ld(pd, i + k * L);
+                                }
+#pragma unroll
+                                for (int k = 0; k < PC; k += 2) {
+                                    float ya, dya, yb, dyb;
+                                    act_backward<ACT, DT>(zv[k], dv[k], p, inv_p, ya, dya);
+                                    act_backward<ACT, DT>(zv[k + 1], dv[k + 1], p, inv_p, yb, dyb);
+                                    s1a += dya;
+                                    sya = fmaf(dya, ya, sya);
+                                    s1b += dyb;
+                                    syb = fmaf(dyb, yb, syb);
+                                }
                             }
-                            if (i < HW) {
+                            for (; i < HW; i += L) {
                                 float ya, dya;
                                 act_backward<ACT, DT>(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), p,
                                                       inv_p, ya, dya);
