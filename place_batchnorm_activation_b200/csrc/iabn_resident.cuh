@@ -1059,23 +1059,38 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     return a.coef[c >= a.C ? c - a.C : c];
                 };
                 unsigned char* gt = a.dst + t_u0(t) * P.unit_bytes;
-                for (int v = tid; v < nvec; v += kConsumers) {
-                    const uint32_t e0 = (uint32_t)v * EPV;
+                // This thread's vectors v = tid + kConsumers*j start ES elements
+                // apart: its plane offset `off` and window index `c` advance by
+                // fixed steps (dq planes + dr elements), no division per vector.
+                constexpr uint32_t ES = (uint32_t)kConsumers * EPV;
+                const uint32_t dq = ES / hw, dr = ES - dq * hw, dqc = dq % C32;
+                uint32_t c, off;
+                {
+                    const uint32_t e0 = (uint32_t)tid * EPV;
                     // e0 / HW: e0 < 2^24, so the float quotient is off by at most one
                     uint32_t pl = (uint32_t)((float)e0 * inv_hw);
                     if (pl * hw > e0) --pl;
                     if ((pl + 1u) * hw <= e0) ++pl;
-                    uint32_t rem = (pl + 1u) * hw - e0;   // elements of plane pl from e0 on
-                    uint32_t c = (ibase + pl) % C32;
+                    off = e0 - pl * hw;
+                    c = (ibase + pl) % C32;
+                }
+                for (int v = tid; v < nvec; v += kConsumers) {
+                    uint32_t rem = hw - off;   // elements of plane c from this vector on
+                    uint32_t cc = c;
                     const uint4 vz = lds128(sbv + (uint32_t)v * 16u);
                     uint4 vd = vz;
                     if (DIR == 1) vd = lds128(sbv + (uint32_t)P.half_bytes + (uint32_t)v * 16u);
                     float xz[EPV], xd[EPV];
                     unpack_all<DT>(vz, xz);
                     if (DIR == 1) unpack_all<DT>(vd, xd);
+                    // one element with coefficients q: forward (16-bit) y = x*scale +
+                    // (beta - mean*scale), (fp32) y = (x - mean)*scale + beta;
+                    // backward dx = A dy + B y + Cc
                     auto rewrite_elem = [&](int k, const float4& q) {
                         if (DIR == 0) {
-                            xz[k] = act_forward<ACT, DT>(fmaf(xz[k] - q.x, q.y, q.z), p);
+                            const float y = DT == kF32 ? fmaf(xz[k] - q.x, q.y, q.z)
+                                                       : fmaf(xz[k], q.y, q.w);
+                            xz[k] = act_forward<ACT, DT>(y, p);
                         } else {
                             float y, dy;
                             act_backward<ACT, DT>(xz[k], xd[k], p, inv_p, y, dy);
@@ -1085,27 +1100,34 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     if (hw >= (uint32_t)EPV) {
                         // planes at least a vector long: two coefficient sets at
                         // most, chosen per element without branches
-                        const float4 q0 = coef_at(c), q1 = coef_at(c + 1u == C32 ? 0u : c + 1u);
+                        const float4 q0 = coef_at(cc), q1 = coef_at(cc + 1u == C32 ? 0u : cc + 1u);
 #pragma unroll
                         for (int k = 0; k < EPV; ++k) {
                             const bool first = (uint32_t)k < rem;
                             const float4 q = make_float4(first ? q0.x : q1.x, first ? q0.y : q1.y,
-                                                         first ? q0.z : q1.z, 0.f);
+                                                         first ? q0.z : q1.z, first ? q0.w : q1.w);
                             rewrite_elem(k, q);
                         }
                     } else {
-                        float4 q = coef_at(c);
+                        float4 q = coef_at(cc);
 #pragma unroll
                         for (int k = 0; k < EPV; ++k) {
                             if (rem == 0u) {
-                                c = c + 1u == C32 ? 0u : c + 1u;
-                                q = coef_at(c);
+                                cc = cc + 1u == C32 ? 0u : cc + 1u;
+                                q = coef_at(cc);
                                 rem = hw;
                             }
                             --rem;
                             rewrite_elem(k, q);
                         }
                     }
+                    off += dr;
+                    c += dqc;
+                    if (off >= hw) {
+                        off -= hw;
+                        ++c;
+                    }
+                    if (c >= C32) c -= C32;
                     stg128(gt + (size_t)v * 16, pack_all<DT>(xz));
                 }
             }
