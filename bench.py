@@ -40,9 +40,9 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # profiles/k_resident_resnet_trunk.md).  Reported only while the CUDA sources
 # hash to the value they were captured on; otherwise "traffic" is null.
 NCU_TRAFFIC = {
-    "sources_sha256": "026899106d55b525e976ad606a3a21bac260fb23f6f5bf63947b8535cdef7539",
-    "backward": 320371712 + 35237632,
-    "forward": 117835776 + 21308928,
+    "sources_sha256": "df7df459f1cf0d338877164655fa41f65e52b9a16bfa19b8bafaf6a5d4da4831",
+    "backward": 296427520 + 34526976,
+    "forward": 113115648 + 22217728,
 }
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
