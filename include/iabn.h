@@ -145,7 +145,9 @@ iabn_status iabn_update_running_stats(int64_t c, int64_t count,
  * clears it (resetting the workspace's control block for reuse).  Returns
  * IABN_OK, IABN_ERR_TIMEOUT, IABN_ERR_SINGULAR_GAMMA (the most severe
  * condition seen since the last read), or IABN_ERR_CUDA if the stream or a
- * copy failed. */
+ * copy failed.  After IABN_ERR_TIMEOUT the outputs of the call(s) that timed
+ * out are undefined; the workspace itself stays usable (later calls are
+ * correct whether or not the status has been read in between). */
 iabn_status iabn_get_device_status(void* workspace, void* stream);
 
 /* Diagnostics: the number of kernels this library has launched in this

@@ -27,7 +27,7 @@ constexpr uint32_t kStSingular = 1u << 1;
 struct Control {
     uint32_t status;     // sticky kSt* bits
     uint32_t bar_count;  // grid-barrier arrivals; a multiple of kBarStride between launches
-    uint32_t bar_gen;    // unused
+    uint32_t never_set;  // a word no code writes (failure-injection wait target)
     uint32_t pad[61];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
@@ -152,9 +152,10 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v
 // it ends (bar_pad), so the next launch again starts on a multiple.  The
 // __syncthreads() before the arrival orders the CTA's writes before thread
 // 0's release (a cumulative release after a CTA barrier).  *fail (shared
-// memory) is the CTA's failure flag: a CTA that has failed does not arrive; a
-// wait that runs out sets *fail and kStTimeout (the control block must then
-// be cleared before the next launch).  Every thread of the CTA must call it.
+// memory) is the CTA's failure flag: a CTA that has failed still arrives (so
+// the counter stays balanced for the next launch) but does not wait; a wait
+// that runs out sets *fail and kStTimeout.  Every thread of the CTA must call
+// it, and every CTA calls every barrier of the launch.
 constexpr uint32_t kBarStride = 256;
 
 __device__ __forceinline__ uint32_t bar_base(const Control* ctl) {
@@ -164,9 +165,9 @@ __device__ __forceinline__ uint32_t bar_base(const Control* ctl) {
 __device__ __forceinline__ bool grid_barrier(Control* ctl, uint32_t target,
                                              unsigned long long budget_ns, int* fail) {
     __syncthreads();
-    if (threadIdx.x == 0 && *((volatile int*)fail) == 0) {
+    if (threadIdx.x == 0) {
         const uint32_t arrived = atom_add_acq_rel_gpu(&ctl->bar_count, 1u) + 1u;
-        if (arrived != target) {
+        if (*((volatile int*)fail) == 0 && arrived != target) {
             const unsigned long long t0 = global_ns();
             while ((int32_t)(ld_acquire_gpu(&ctl->bar_count) - target) < 0) {
                 if (global_ns() - t0 > budget_ns) {
@@ -182,7 +183,8 @@ __device__ __forceinline__ bool grid_barrier(Control* ctl, uint32_t target,
 }
 
 // Called by one thread of one CTA after the launch's last barrier (nbar
-// barriers of G arrivals each): brings the counter to base + 2*kBarStride.
+// barriers of G arrivals each, every CTA arriving at each, failed or not):
+// brings the counter to base + 2*kBarStride once all arrivals are in.
 __device__ __forceinline__ void bar_pad(Control* ctl, uint32_t G, uint32_t nbar) {
     atomicAdd(&ctl->bar_count, 2u * kBarStride - nbar * G);
 }

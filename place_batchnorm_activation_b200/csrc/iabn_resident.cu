@@ -186,6 +186,7 @@ ResArgs base_args(const Geom& g, const Workspace& w) {
     a.budget_ns = b > 0 ? (unsigned long long)b : kWaitBudgetNs;
     a.wait_cons = (int)env_long("IABN_WAIT_CONS", 0);
     a.wait_prod = (int)env_long("IABN_WAIT_PROD", 0);
+    a.stall_cta = (int)env_long("IABN_TEST_STALL_CTA", -1);
     return a;
 }
 

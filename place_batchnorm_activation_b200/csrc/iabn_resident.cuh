@@ -91,6 +91,9 @@ struct ResArgs {
     unsigned long long budget_ns;
     int wait_cons;               // mbarrier wait mode of the consumers (see mbar_wait)
     int wait_prod;               // mbarrier wait mode of the producer
+    int stall_cta;               // failure injection (tests): this CTA waits, for twice
+                                 // the budget, on a word nothing sets before barrier 1;
+                                 // -1: none
 };
 
 // Sum over aligned groups of L lanes (L a power of two); every lane of the
@@ -757,6 +760,14 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     stamp(2, tid == 0);
 
     // ------------------------------------------------- barriers and finalize
+    if (b == a.stall_cta && tid == 0) {
+        // injected failure: a wait on a flag nothing sets runs out (bounded)
+        const unsigned long long t0 = global_ns();
+        while (ld_acquire_gpu(&a.ctl->never_set) == 0u && global_ns() - t0 < 2 * a.budget_ns) {
+        }
+        atomicOr(&a.ctl->status, kStTimeout);
+        set_failed();
+    }
     grid_barrier(a.ctl, bbase + (uint32_t)G, a.budget_ns, &s_fail);
     stamp(3, tid == 0);
     if (!producer && lane == 0) cp_async_wait_all();   // s_par (issued at launch)
@@ -890,8 +901,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
     }
     stamp(4, tid == 0);
-    if (grid_barrier(a.ctl, bbase + 2u * (uint32_t)G, a.budget_ns, &s_fail) && b == 0 && tid == 0)
-        bar_pad(a.ctl, (uint32_t)G, 2u);
+    grid_barrier(a.ctl, bbase + 2u * (uint32_t)G, a.budget_ns, &s_fail);
+    if (b == 0 && tid == 0) bar_pad(a.ctl, (uint32_t)G, 2u);
     // NCHW: the coefficients of the CTA's channel window, (u0*g + i) mod C for
     // i < ncoef, into shared memory (every thread reaches the barrier)
     const int64_t ch0 = LAYOUT == kNCHW ? (u0 * P.g) % a.C : 0;
@@ -1185,11 +1196,12 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     if (pl) {
         if (failed()) {
             atomicOr(&a.ctl->status, kStTimeout);
-            // Wait (bounded) for the last load into every slot before the CTA
-            // exits; completed ones return at once.
+            // Wait for the last load into every slot before the CTA exits;
+            // completed ones return at once.  The budget is the fixed default,
+            // whatever the configured one: loads of valid memory always land.
             for (int s = 0; s < P.nslots; ++s)
                 if ((loaded >> s) & 1u)
-                    mbar_wait(&full[s], ((fiss >> s) & 1u) ^ 1u, a.budget_ns / 4);
+                    mbar_wait(&full[s], ((fiss >> s) & 1u) ^ 1u, kWaitBudgetNs);
         }
     }
     stamp(8, tid == 0);
