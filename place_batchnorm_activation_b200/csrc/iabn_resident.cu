@@ -107,8 +107,14 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         if (cpt == 1 && P.RP > 1) scratch = (P.RP - 1) * P.VC * (8 / s) * 16;
         // TMEM stash: 1 KB (64 vectors) per consumer thread; TMEM accesses are
         // warp-wide, so every warp must hold a single row phase
-        if ((cpt > 1 || P.VC % 32 == 0) && env_long("IABN_TMEM_STASH", 1) != 0)
-            P.stash = 64 / (cpt * NT);
+        if (env_long("IABN_TMEM_STASH", 1) != 0) {
+            if (cpt == 1 && P.RP * P.VC == kConsumers && env_long("IABN_STASH_CP", 1) != 0) {
+                P.stash = 64 / NT;   // copy engine: 8 columns per row group and tensor
+                P.stash_cp = 1;
+            } else if (cpt > 1 || P.VC % 32 == 0) {
+                P.stash = 64 / (cpt * NT);
+            }
+        }
     } else {
         const int64_t pb = g.HW * s;
         const int gq = 16 / gcd_int(pb, 16);
@@ -153,7 +159,7 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     if (nslots > kMaxSlots) nslots = kMaxSlots;
     if (ring > nslots) return false;
     if (P.stash > 0) nslots = ring;   // the stash replaces resident tiles
-    P.stash_first = (int)env_long("IABN_STASH_FIRST", 1);
+    P.stash_first = P.stash_cp ? 1 : (int)env_long("IABN_STASH_FIRST", 1);
     P.nslots = nslots;
     P.ring = ring;
     P.smem_bytes = kBarBytes + P.scratch_bytes + nslots * P.slot_bytes;

@@ -6,7 +6,8 @@
 // NCHW: groups of g whole planes, g chosen so every unit starts on a 16-byte
 // boundary) and streams it through shared-memory slots with the bulk-copy
 // engine.  One producer warp issues every bulk load; eight consumer warps
-// compute and store.  Slots are handed over with mbarriers (full: data
+// compute and store; one copier warp moves stashed rows from the landed
+// slots into Tensor Memory (see the TMEM stash below).  Slots are handed over with mbarriers (full: data
 // landed; empty: consumers done with a phase A tile; done: consumers done
 // with a phase B tile, so the slot may be refilled), so no consumer waits on
 // a CTA-wide barrier per tile.
@@ -44,9 +45,9 @@ namespace iabn {
 
 constexpr int kConsumers = 256;                  // consumer threads (8 warps)
 constexpr int kConsumerWarps = kConsumers / 32;
-constexpr int kResThreads = kConsumers + 32;     // + one producer warp
+constexpr int kResThreads = kConsumers + 64;     // + one producer warp + one copier warp
 constexpr int kMaxSlots = 32;
-constexpr int kBarBytes = 3 * kMaxSlots * 8;     // full[], empty[], done[] mbarriers
+constexpr int kBarBytes = 4 * kMaxSlots * 8;     // full[], empty[], done[], cpdone[] mbarriers
 
 struct ResPlan {
     int G;               // CTAs (at most one per SM)
@@ -65,6 +66,9 @@ struct ResPlan {
     int g, L;            // NCHW: planes per unit; lanes per plane
     int hints;           // 1: L2 eviction-priority hints on the bulk copies
     int stash_first;     // 1: the stash holds each thread's first rows, 0: its last
+    int stash_cp;        // 1: the copy engine (tcgen05.cp) fills the stash from the
+                         // landed slots (CPT 1, RP*VC = 256, first rows); 0: the
+                         // consumers store their registers
     int ncoef;           // NCHW: channels of the CTA's coefficient window kept in shared
                          // memory (scratch) for phase B; 0: read from global memory
     int stash;           // NHWC: rows per consumer thread kept in TMEM from phase A
@@ -199,6 +203,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxSlots;
     uint64_t* done = empty + kMaxSlots;
+    uint64_t* cpdone = done + kMaxSlots;   // TMEM copies out of a slot have finished
     __shared__ int s_fail;
     // gamma, beta (and, backward, the saved variance) of the first channel
     // each consumer warp finalizes, fetched while phase A streams
@@ -209,7 +214,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     unsigned char* slots = scratch + P.scratch_bytes;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const bool consumer = warp < kConsumerWarps;
     const bool producer = warp == kConsumerWarps;
+    const bool copier = warp == kConsumerWarps + 1;
     const int b = blockIdx.x;
     const int G = P.G;
     // Phase trace: 0 start, 1 phase A done, 2 merged, 3 barrier 1, 4 finalize,
@@ -262,6 +269,12 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     // being tile thi-1-j.
     const bool stash = LAYOUT == kNHWC && P.stash > 0;
     const bool sfirst = stash && P.stash_first != 0;
+    // copy-engine stash: tcgen05.cp moves each stashed row group (RP rows of
+    // RP*VC = 256 16-byte chunks, one tensor) from its landed slot into 8 TMEM
+    // columns, chunk L -> lane L (columns 0-3) and chunk L+128 -> lane L
+    // (columns 4-7): exactly what consumer thread L, resp. L+128, owns.
+    const bool scp = sfirst && P.stash_cp != 0;
+    const int tpg = P.tile_units / P.RP;   // row groups per tile (NHWC)
     const int64_t nrows = u1 - u0;
     const int Jc = stash ? (int)min((int64_t)P.stash, nrows / P.RP) : 0;
     const int64_t S = (int64_t)P.RP * Jc;
@@ -282,13 +295,14 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
             mbar_init(&done[s], kConsumerWarps);
+            mbar_init(&cpdone[s], 1);
         }
         mbar_init_fence();
         s_fail = 0;
     }
     // grid-barrier counter base of this launch (thread 0 only; see grid_barrier)
     const uint32_t bbase = tid == 0 ? bar_base(a.ctl) : 0u;
-    if (!producer && lane == 0) {
+    if (consumer && lane == 0) {
         const int64_t c = (int64_t)b * kConsumerWarps + warp;
         if (c < a.C) {
             cp_async4(&s_par[warp][0], a.gamma + c);
@@ -324,6 +338,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     uint32_t loaded = 0;      // slots that received at least one load
     uint32_t epar = 0;        // next empty[] phase to wait for, per ring slot
     uint32_t used = 0;        // ring slots holding a phase A tile not yet released
+    uint32_t cpp = 0;         // slots with a TMEM-copy commit not yet waited for
+    uint32_t cppar = 0;       // next cpdone[] phase to wait for, per slot
     uint64_t pol_keep = 0, pol_stream = 0;
     const bool pl = producer && lane == 0;
     if (pl) {
@@ -349,13 +365,22 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         fiss ^= 1u << s;
         loaded |= 1u << s;
     };
-    // Waits until the consumers released ring slot s after its phase A tile.
+    // Waits until the TMEM copies out of slot s have finished reading it.
+    auto wait_cp = [&](int s) -> bool {
+        if (!((cpp >> s) & 1u)) return true;
+        const bool ok = mbar_wait(&cpdone[s], (cppar >> s) & 1u, a.budget_ns, a.wait_prod);
+        cppar ^= 1u << s;
+        cpp &= ~(1u << s);
+        return ok;
+    };
+    // Waits until the consumers released ring slot s after its phase A tile
+    // (and any TMEM copy out of it finished).
     auto wait_empty = [&](int s) -> bool {
-        if (!((used >> s) & 1u)) return true;
+        if (!((used >> s) & 1u)) return wait_cp(s);
         const bool ok = mbar_wait(&empty[s], (epar >> s) & 1u, a.budget_ns, a.wait_prod);
         epar ^= 1u << s;
         used &= ~(1u << s);
-        return ok;
+        return ok && wait_cp(s);
     };
     if (pl) {
         for (int t = 0; t < n && !failed(); ++t) {
@@ -366,6 +391,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             }
             // tiles read again in phase B stay in L2; stashed or resident ones need not
             issue(t, s, (stash ? t >= tlo && t < thi : t < nring) ? pol_keep : pol_stream);
+            if (scp && t * tpg < Jc) cpp |= 1u << s;   // consumer warp 0 copies it to TMEM
         }
         // Phase B prefetch into the streamed slots as they free up: the j-th
         // streamed tile of phase B (tile thi-1-j) goes to slot j % ring.
@@ -374,6 +400,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             if (!wait_empty(j)) { set_failed(); break; }
             issue(thi - 1 - j, j, pol_stream);
         }
+        // every TMEM copy has finished before phase B reads TMEM
+        for (int s = 0; s < ring && scp && !failed(); ++s)
+            if (!wait_cp(s)) set_failed();
+        if (scp) tmem_fence_before_sync();
     }
 
     // ================================================================ consumers
@@ -404,12 +434,12 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         if (CPT == 1) {
             col[0] = tid % VC;
             phase = tid / VC;
-            colok[0] = !producer && phase < RP;
+            colok[0] = consumer && phase < RP;
         } else {
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
                 col[k] = tid + k * kConsumers;
-                colok[k] = !producer && col[k] < VC;
+                colok[k] = consumer && col[k] < VC;
             }
         }
     } else {
@@ -477,7 +507,32 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             }
     }
 
-    if (!producer) {
+    if (copier && lane == 0 && scp) {
+        // Each stashed tile, once landed: its row groups into TMEM (fwd: 8
+        // columns per group; bwd: z then dz, 16 columns per group), then a
+        // commit to cpdone[] that the producer waits for before refilling.
+        // The k-th tile of a slot completes full[] phase k; the producer does
+        // not reload the slot before this commit, so the parity cannot alias.
+        for (int t = 0; t < nring && t * tpg < Jc && !failed(); ++t) {
+            const int s = slotA(t);
+            if (!mbar_wait(&full[s], (uint32_t)((t / ring) & 1), a.budget_ns, a.wait_prod)) {
+                set_failed();
+                break;
+            }
+            const uint32_t sbase = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
+            for (int gi = 0; gi < tpg && t * tpg + gi < Jc; ++gi) {
+                const int i = t * tpg + gi;
+#pragma unroll
+                for (int k = 0; k < NT; ++k) {
+                    const uint32_t src = sbase + (uint32_t)(k * P.half_bytes) + (uint32_t)gi * 4096u;
+                    tmem_cp_128x256b(tmem_base + (uint32_t)(8 * (NT * i + k)),
+                                     smem_desc_plain(src, 2048u, 128u));
+                }
+            }
+            tmem_commit(&cpdone[s]);
+        }
+    }
+    if (consumer) {
         acct_start();
         for (int t = 0; t < n; ++t) {
             const int s = slotA(t);
@@ -502,7 +557,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                                 vz[u][k] = lds128(o);
                                 if (DIR == 1) vd[u][k] = lds128(o + (uint32_t)P.half_bytes);
                             }
-                        if (stash) {
+                        if (stash && !scp) {
                             // rows from ordinal js on also go to TMEM (warp-uniform:
                             // a warp's lanes share the row phase): a whole batch as
                             // one 16/32-column store, else vector by vector
@@ -709,9 +764,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             acct_work();
         }
         acct_flush(9);
-        if (stash) tmem_wait_st();   // this thread's stores land before its phase B loads
+        if (stash && !scp) tmem_wait_st();   // this thread's stores land before its loads
     }
     __syncthreads();
+    if (scp) tmem_fence_after_sync();   // the producer saw every TMEM copy complete
     stamp(1, tid == 0);
 
     // ------------------------------------------- per-CTA merge (NHWC)
@@ -770,8 +826,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     }
     grid_barrier(a.ctl, bbase + (uint32_t)G, a.budget_ns, &s_fail);
     stamp(3, tid == 0);
-    if (!producer && lane == 0) cp_async_wait_all();   // s_par (issued at launch)
-    if (!failed() && !producer) {
+    if (consumer && lane == 0) cp_async_wait_all();   // s_par (issued at launch)
+    if (!failed() && consumer) {
         // one consumer warp per channel over the whole grid, fp64, fixed order
         const int64_t nw = (int64_t)G * kConsumerWarps;
         const int64_t K = LAYOUT == kNHWC ? (int64_t)G : a.N;
@@ -908,7 +964,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int64_t ch0 = LAYOUT == kNCHW ? (u0 * P.g) % a.C : 0;
     float4* scoef = reinterpret_cast<float4*>(scratch);
     if (LAYOUT == kNCHW && P.ncoef > 0) {
-        if (!producer && !failed())
+        if (consumer && !failed())
             for (int i = tid; i < P.ncoef; i += kConsumers) {
                 const int64_t c = ch0 + i;
                 scoef[i] = a.coef[c >= a.C ? c - a.C : c];
@@ -935,7 +991,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             if (!ok) set_failed();
             stamp(7, true);
         }
-    } else if (!failed()) {
+    } else if (consumer && !failed()) {
         // coefficients of this thread's channels (NHWC)
         // c3/c4 are kept per channel only when a thread owns one column;
         // otherwise the backward forms them on the fly (register budget).
@@ -1144,7 +1200,27 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             }
         };
         acct_start();
-        if (stash && active) {
+        if (scp) {
+            // the stashed row groups first, four at a time: this thread's
+            // vector of group i is at column 8*(NT*i + tensor) + 4*(warp/4)
+            unsigned char* grow = a.dst + u0 * P.unit_bytes;
+            const uint32_t ta = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) +
+                                (uint32_t)(4 * ((warp >> 2) & 1));
+            for (int i0 = 0; i0 < Jc; i0 += 4) {
+                uint4 bz[4], bd[4];
+                tmem_ld4x4(ta + (uint32_t)(8 * NT * i0), (uint32_t)(8 * NT), bz);
+                if (NT == 2) tmem_ld4x4(ta + (uint32_t)(8 * NT * i0 + 8), (uint32_t)(8 * NT), bd);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (i0 + u >= Jc) continue;
+                    uint4 vz[CPT], vd[CPT];
+                    vz[0] = bz[u];
+                    vd[0] = NT == 2 ? bd[u] : bz[u];
+                    rewrite(vz, vd);
+                    stg128(grow + voff[0] + (size_t)(i0 + u) * vstep, DIR == 0 ? vz[0] : vd[0]);
+                }
+            }
+        } else if (stash && active) {
             // the stashed rows first: no wait for any tile
             unsigned char* grow = a.dst + u0 * P.unit_bytes;
             for (int i0 = 0; i0 < Jc; i0 += RB) {

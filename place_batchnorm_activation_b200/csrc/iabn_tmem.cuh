@@ -76,6 +76,46 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint4* v) {
         : "memory");
 }
 
+// Shared-memory matrix descriptor without swizzling (sm_100 format: start
+// address, LBO and SBO in 16-byte units, bits 46-47 = 1).  LBO strides the
+// two 16-byte halves of a 32-byte row, SBO the groups of 8 rows (each group:
+// 8 rows of 16 bytes, 128 contiguous bytes).
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Asynchronous copy of a 128-row x 32-byte matrix from shared memory into TMEM
+// lanes 0..127, 8 columns from taddr.  Issued by one thread; completion is
+// tracked with tmem_commit.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+// The mbarrier at bar (count 1) completes a phase once every tcgen05
+// operation the calling thread issued before has completed.
+__device__ __forceinline__ void tmem_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            (uint32_t)__cvta_generic_to_shared(bar))
+        : "memory");
+}
+
+// Four vectors at taddr + k*stride (k = 0..3) of the thread's lane, waited for.
+__device__ __forceinline__ void tmem_ld4x4(uint32_t taddr, uint32_t stride, uint4* v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%16];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [%17];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [%18];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%12, %13, %14, %15}, [%19];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0].x), "=r"(v[0].y), "=r"(v[0].z), "=r"(v[0].w), "=r"(v[1].x), "=r"(v[1].y),
+          "=r"(v[1].z), "=r"(v[1].w), "=r"(v[2].x), "=r"(v[2].y), "=r"(v[2].z), "=r"(v[2].w),
+          "=r"(v[3].x), "=r"(v[3].y), "=r"(v[3].z), "=r"(v[3].w)
+        : "r"(taddr), "r"(taddr + stride), "r"(taddr + 2 * stride), "r"(taddr + 3 * stride)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
