@@ -108,8 +108,8 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         // TMEM stash: 1 KB (64 vectors) per consumer thread; TMEM accesses are
         // warp-wide, so every warp must hold a single row phase
         if (env_long("IABN_TMEM_STASH", 1) != 0) {
-            if (cpt == 1 && P.RP * P.VC == kConsumers && env_long("IABN_STASH_CP", 1) != 0) {
-                P.stash = 64 / NT;   // copy engine: 8 columns per row group and tensor
+            if (P.RP * P.VC == kConsumers * cpt && env_long("IABN_STASH_CP", 1) != 0) {
+                P.stash = 64 / (cpt * NT);   // copy engine: 8 columns per 4 KB piece
                 P.stash_cp = 1;
             } else if (cpt > 1 || P.VC % 32 == 0) {
                 P.stash = 64 / (cpt * NT);

@@ -24,9 +24,10 @@
 //   barrier  grid-wide (bounded wait), a distributed fp64 finalize (one warp
 //            per channel, fixed order), a second grid barrier.
 //   phase B  tiles n-1..0: resident tiles first, then the streamed ones -- the
-//            most recently read first, while they are still in L2.  The
-//            consumers write their results straight to global memory with
-//            128-bit stores; the producer refills each freed streamed slot.
+//            most recently read first: the last one of each ring slot is still
+//            in the slot, the others are read back from L2.  The consumers
+//            write their results straight to global memory with 128-bit
+//            stores; the producer refills each freed ring slot.
 //
 // Method: "In-Place Activated BatchNorm for Memory-Optimized Training of
 // DNNs" (paperlayer.ai summary), section 3: "Batch Normalization Review",
@@ -269,10 +270,11 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     // being tile thi-1-j.
     const bool stash = LAYOUT == kNHWC && P.stash > 0;
     const bool sfirst = stash && P.stash_first != 0;
-    // copy-engine stash: tcgen05.cp moves each stashed row group (RP rows of
-    // RP*VC = 256 16-byte chunks, one tensor) from its landed slot into 8 TMEM
-    // columns, chunk L -> lane L (columns 0-3) and chunk L+128 -> lane L
-    // (columns 4-7): exactly what consumer thread L, resp. L+128, owns.
+    // copy-engine stash: tcgen05.cp moves each 4 KB piece of a stashed row
+    // group (RP rows holding RP*VC = 256*CPT 16-byte chunks; per tensor) from
+    // its landed slot into 8 TMEM columns, chunk L -> lane L (columns 0-3) and
+    // chunk L+128 -> lane L (columns 4-7): exactly what consumer thread L,
+    // resp. L+128, owns (its column k of the piece k).
     const bool scp = sfirst && P.stash_cp != 0;
     const int tpg = P.tile_units / P.RP;   // row groups per tile (NHWC)
     const int64_t nrows = u1 - u0;
@@ -328,6 +330,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         return (int)(r < P.tile_units ? r : P.tile_units);
     };
     auto slotA = [&](int t) -> int { return t < nring ? t % ring : ring + (t - nring); };
+    // Phase B streams tile t through ring slot t % ring too, so the last
+    // phase-A tile of each ring slot is still there when phase B wants it.
+    auto ring_resident = [&](int t) -> bool { return t < nring && t >= nring - ring; };
     auto slot_ptr = [&](int s) -> unsigned char* { return slots + (size_t)s * P.slot_bytes; };
     auto failed = [&]() -> bool { return *((volatile int*)&s_fail) != 0; };
     auto set_failed = [&]() { *((volatile int*)&s_fail) = 1; };
@@ -390,15 +395,19 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 used |= 1u << s;
             }
             // tiles read again in phase B stay in L2; stashed or resident ones need not
-            issue(t, s, (stash ? t >= tlo && t < thi : t < nring) ? pol_keep : pol_stream);
+            const bool again = (stash ? t >= tlo && t < thi : t < nring) && !ring_resident(t);
+            issue(t, s, again ? pol_keep : pol_stream);
             if (scp && t * tpg < Jc) cpp |= 1u << s;   // consumer warp 0 copies it to TMEM
         }
-        // Phase B prefetch into the streamed slots as they free up: the j-th
-        // streamed tile of phase B (tile thi-1-j) goes to slot j % ring.
+        // Phase B: the j-th streamed tile is t = thi-1-j, in slot t % ring.  The
+        // first one of each slot is either still there from phase A or is
+        // loaded as soon as phase A releases the slot.
         const int pro = min(ring, nB);
         for (int j = 0; j < pro && !failed(); ++j) {
-            if (!wait_empty(j)) { set_failed(); break; }
-            issue(thi - 1 - j, j, pol_stream);
+            const int t = thi - 1 - j;
+            if (ring_resident(t)) continue;
+            if (!wait_empty(t % ring)) { set_failed(); break; }
+            issue(t, t % ring, pol_stream);
         }
         // every TMEM copy has finished before phase B reads TMEM
         for (int s = 0; s < ring && scp && !failed(); ++s)
@@ -523,11 +532,14 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             for (int gi = 0; gi < tpg && t * tpg + gi < Jc; ++gi) {
                 const int i = t * tpg + gi;
 #pragma unroll
-                for (int k = 0; k < NT; ++k) {
-                    const uint32_t src = sbase + (uint32_t)(k * P.half_bytes) + (uint32_t)gi * 4096u;
-                    tmem_cp_128x256b(tmem_base + (uint32_t)(8 * (NT * i + k)),
-                                     smem_desc_plain(src, 2048u, 128u));
-                }
+                for (int kc = 0; kc < CPT; ++kc)
+#pragma unroll
+                    for (int k = 0; k < NT; ++k) {
+                        const uint32_t src = sbase + (uint32_t)(k * P.half_bytes) +
+                                             (uint32_t)(gi * CPT + kc) * 4096u;
+                        tmem_cp_128x256b(tmem_base + (uint32_t)(8 * (NT * (i * CPT + kc) + k)),
+                                         smem_desc_plain(src, 2048u, 128u));
+                    }
             }
             tmem_commit(&cpdone[s]);
         }
@@ -977,16 +989,17 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     if (producer) {
         if (pl && !failed()) {
             // The consumers write their results to global memory themselves;
-            // the producer refills each streamed slot with streamed tile
-            // j + ring once they are done with tile j.
+            // the producer loads streamed tile t into slot t % ring once they
+            // are done with the slot's previous phase-B tile, t + ring.
             uint32_t dpar = 0;
             bool ok = true;
-            for (int j = 0; j + ring < nB && ok; ++j) {
-                const int s = j % ring;
+            for (int j = ring; j < nB && ok; ++j) {
+                const int t = thi - 1 - j;
+                const int s = t % ring;
                 ok = mbar_wait(&done[s], (dpar >> s) & 1u, a.budget_ns, a.wait_prod);
                 dpar ^= 1u << s;
                 if (!ok) break;
-                issue(thi - 1 - (j + ring), s, pol_stream);
+                issue(t, s, pol_stream);
             }
             if (!ok) set_failed();
             stamp(7, true);
@@ -1201,23 +1214,26 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         };
         acct_start();
         if (scp) {
-            // the stashed row groups first, four at a time: this thread's
-            // vector of group i is at column 8*(NT*i + tensor) + 4*(warp/4)
+            // the stashed row groups first, RB at a time (four vectors per
+            // tensor): this thread's column k of group i is at TMEM column
+            // 8*(NT*(i*CPT + k) + tensor) + 4*(warp/4)
             unsigned char* grow = a.dst + u0 * P.unit_bytes;
             const uint32_t ta = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) +
                                 (uint32_t)(4 * ((warp >> 2) & 1));
-            for (int i0 = 0; i0 < Jc; i0 += 4) {
-                uint4 bz[4], bd[4];
-                tmem_ld4x4(ta + (uint32_t)(8 * NT * i0), (uint32_t)(8 * NT), bz);
-                if (NT == 2) tmem_ld4x4(ta + (uint32_t)(8 * NT * i0 + 8), (uint32_t)(8 * NT), bd);
+            for (int i0 = 0; i0 < Jc; i0 += RB) {
+                uint4 bz[RB * CPT], bd[RB * CPT];
+                const uint32_t f0 = (uint32_t)(i0 * CPT);
+                tmem_ld4x4(ta + 8u * NT * f0, 8u * NT, bz);
+                if (NT == 2) tmem_ld4x4(ta + 8u * NT * f0 + 8u, 8u * NT, bd);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < RB; ++u) {
                     if (i0 + u >= Jc) continue;
-                    uint4 vz[CPT], vd[CPT];
-                    vz[0] = bz[u];
-                    vd[0] = NT == 2 ? bd[u] : bz[u];
+                    uint4* vz = bz + u * CPT;
+                    uint4* vd = NT == 2 ? bd + u * CPT : bz + u * CPT;
                     rewrite(vz, vd);
-                    stg128(grow + voff[0] + (size_t)(i0 + u) * vstep, DIR == 0 ? vz[0] : vd[0]);
+#pragma unroll
+                    for (int k = 0; k < CPT; ++k)
+                        stg128(grow + voff[k] + (size_t)(i0 + u) * vstep, DIR == 0 ? vz[k] : vd[k]);
                 }
             }
         } else if (stash && active) {
@@ -1253,10 +1269,11 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
         acct_work();
         for (int j = 0; j < nB; ++j) {
-            const int s = j % ring;
-            if (!cwait(s)) break;
-            acct_wait();
             const int t = thi - 1 - j;
+            const int s = t % ring;
+            // a tile still in its slot from phase A needs no wait
+            if (!ring_resident(t) && !cwait(s)) break;
+            acct_wait();
             // skip the stashed rows: ordinals [js, js + Jc)
             const int qlo = stash && sfirst ? Jc - t * tile_ord : 0;
             const int qhi = stash && !sfirst ? js - t * tile_ord : INT_MAX;
