@@ -197,6 +197,14 @@ __device__ __forceinline__ double warp_sum(double v) {
     return __shfl_sync(0xffffffffu, v, 0);
 }
 
+// The same over each half of the warp (lanes 0-15, 16-31); every lane of the
+// warp must call it.
+__device__ __forceinline__ double half_warp_sum(double v) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o, 16);
+    return __shfl_sync(0xffffffffu, v, 0, 16);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);

@@ -206,9 +206,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     uint64_t* done = empty + kMaxSlots;
     uint64_t* cpdone = done + kMaxSlots;   // TMEM copies out of a slot have finished
     __shared__ int s_fail;
-    // gamma, beta (and, backward, the saved variance) of the first channel
-    // each consumer warp finalizes, fetched while phase A streams
-    __shared__ float s_par[kConsumerWarps][3];
+    // gamma, beta (and, backward, the saved variance; forward NHWC, the pivot
+    // word) of the first channel each consumer half-warp finalizes, fetched
+    // while phase A streams
+    __shared__ float s_par[kConsumerWarps][2][3];
 
     const ResPlan& P = a.P;
     unsigned char* scratch = smem + kBarBytes;
@@ -304,15 +305,16 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     }
     // grid-barrier counter base of this launch (thread 0 only; see grid_barrier)
     const uint32_t bbase = tid == 0 ? bar_base(a.ctl) : 0u;
-    if (consumer && lane == 0) {
-        const int64_t c = (int64_t)b * kConsumerWarps + warp;
+    if (consumer && (lane & 15) == 0) {
+        const int h = lane >> 4;
+        const int64_t c = ((int64_t)b * kConsumerWarps + warp) * 2 + h;
         if (c < a.C) {
-            cp_async4(&s_par[warp][0], a.gamma + c);
-            cp_async4(&s_par[warp][1], a.beta + c);
-            if (DIR == 1) cp_async4(&s_par[warp][2], a.var_in + c);
+            cp_async4(&s_par[warp][h][0], a.gamma + c);
+            cp_async4(&s_par[warp][h][1], a.beta + c);
+            if (DIR == 1) cp_async4(&s_par[warp][h][2], a.var_in + c);
             // forward NHWC: the aligned word holding the pivot x[0, c]
             if (DIR == 0 && LAYOUT == kNHWC)
-                cp_async4(&s_par[warp][2], a.src0 + ((c * (int64_t)sizeof(typename Storage<DT>::T)) & ~int64_t(3)));
+                cp_async4(&s_par[warp][h][2], a.src0 + ((c * (int64_t)sizeof(typename Storage<DT>::T)) & ~int64_t(3)));
         }
     }
     if (stash && warp == 0) {
@@ -838,13 +840,16 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     }
     grid_barrier(a.ctl, bbase + (uint32_t)G, a.budget_ns, &s_fail);
     stamp(3, tid == 0);
-    if (consumer && lane == 0) cp_async_wait_all();   // s_par (issued at launch)
+    if (consumer && (lane & 15) == 0) cp_async_wait_all();   // s_par (issued at launch)
     if (!failed() && consumer) {
-        // one consumer warp per channel over the whole grid, fp64, fixed order
+        // one consumer half-warp per channel over the whole grid, fp64, fixed
+        // order; a warp takes the channels 2cp and 2cp+1 (the loop is
+        // warp-uniform; a half without a channel computes on a stand-in)
+        const int hl = lane & 15, half = lane >> 4;
         const int64_t nw = (int64_t)G * kConsumerWarps;
         const int64_t K = LAYOUT == kNHWC ? (int64_t)G : a.N;
-        constexpr int KC = 5;   // partials cached per lane when K <= 160
-        const bool cached = K <= 32 * KC;
+        constexpr int KC = 10;   // partials cached per lane when K <= 160
+        const bool cached = K <= 16 * KC;
         const double hw = (double)a.HW;   // elements behind each NCHW partial
         // the pivot x[0, c] from the aligned 32-bit word that holds it
         auto pivot_of = [&](uint32_t w, int64_t c) -> float {
@@ -854,23 +859,24 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             return __half2float(__ushort_as_half((unsigned short)h));
         };
         bool first = true;
-        for (int64_t c = (int64_t)b * kConsumerWarps + warp; c < a.C; c += nw, first = false) {
+        for (int64_t cpair = (int64_t)b * kConsumerWarps + warp; cpair * 2 < a.C;
+             cpair += nw, first = false) {
+            const int64_t cw = cpair * 2 + half;
+            const bool cv = cw < a.C;
+            const int64_t c = cv ? cw : a.C - 1;
             double2 pk[KC];
-            double ck[KC];
 #pragma unroll
             for (int i = 0; i < KC; ++i) {
-                const int64_t k = lane + 32 * i;
-                const bool in = cached && k < K;
-                pk[i] = in ? a.part[k * a.C + c] : make_double2(0.0, 0.0);
-                ck[i] = in ? hw : 0.0;
+                const int64_t k = hl + 16 * i;
+                pk[i] = cached && k < K ? a.part[k * a.C + c] : make_double2(0.0, 0.0);
             }
-            // per-channel parameters (lane 0 uses them)
+            // per-channel parameters (lane 0 of the half uses them)
             float gmf = 0.f, btf = 0.f, vif = 0.f;
-            if (lane == 0) {
+            if (hl == 0) {
                 if (first) {
-                    gmf = s_par[warp][0];
-                    btf = s_par[warp][1];
-                    vif = s_par[warp][2];
+                    gmf = s_par[warp][half][0];
+                    btf = s_par[warp][half][1];
+                    vif = s_par[warp][half][2];
                 } else {
                     gmf = a.gamma[c];
                     btf = a.beta[c];
@@ -887,7 +893,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 //   s1 = sum n (mean_k - r),  s2 = sum M2_k + n (mean_k - r)^2.
                 double r = 0.0;
                 if (LAYOUT == kNCHW)
-                    r = __shfl_sync(0xffffffffu, cached ? pk[0].x : a.part[c].x, 0);
+                    r = __shfl_sync(0xffffffffu, cached ? pk[0].x : a.part[c].x, 0, 16);
                 double s1 = 0.0, s2 = 0.0;
                 if (cached) {
 #pragma unroll
@@ -896,13 +902,13 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                             s1 += pk[i].x;
                             s2 += pk[i].y;
                         } else {
-                            const double w = ck[i] * (pk[i].x - r);
+                            const double w = (hl + 16 * i < K ? hw : 0.0) * (pk[i].x - r);
                             s1 += w;
                             s2 += pk[i].y + w * (pk[i].x - r);
                         }
                     }
                 } else {
-                    for (int64_t k = lane; k < K; k += 32) {
+                    for (int64_t k = hl; k < K; k += 16) {
                         const double2 v = a.part[k * a.C + c];
                         if (LAYOUT == kNHWC) {
                             s1 += v.x;
@@ -914,10 +920,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         }
                     }
                 }
-                s1 = warp_sum(s1);
-                s2 = warp_sum(s2);
-                if (LAYOUT == kNHWC && lane == 0) r = (double)pivot_of(__float_as_uint(vif), c);
-                if (lane == 0) {
+                s1 = half_warp_sum(s1);
+                s2 = half_warp_sum(s2);
+                if (LAYOUT == kNHWC && hl == 0) r = (double)pivot_of(__float_as_uint(vif), c);
+                if (hl == 0 && cv) {
                     const double mean = r + s1 / a.M;
                     const double var = fmax((s2 - s1 * (s1 / a.M)) / a.M, 0.0);
                     a.out0[c] = (float)mean;
@@ -937,15 +943,15 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         sy += pk[i].y;
                     }
                 } else {
-                    for (int64_t k = lane; k < K; k += 32) {
+                    for (int64_t k = hl; k < K; k += 16) {
                         const double2 v = a.part[k * a.C + c];
                         s1 += v.x;
                         sy += v.y;
                     }
                 }
-                s1 = warp_sum(s1);
-                sy = warp_sum(sy);
-                if (lane == 0) {
+                s1 = half_warp_sum(s1);
+                sy = half_warp_sum(sy);
+                if (hl == 0 && cv) {
                     const double gm = gmf, bt = btf;
                     const double rstd = 1.0 / sqrt((double)vif + (double)a.eps);
                     if (!(fabs(gm) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN
