@@ -40,9 +40,9 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # profiles/k_resident_resnet_trunk.md).  Reported only while the CUDA sources
 # hash to the value they were captured on; otherwise "traffic" is null.
 NCU_TRAFFIC = {
-    "sources_sha256": "c6193880c60726217306a45d316e56ceb81f79eb404eb74c5219cd27633bbef9",
-    "backward": 287760640 + 34491392,
-    "forward": 110098176 + 23406336,
+    "sources_sha256": "4b6bf8830e9890cc4c95f874942cb477f957201d814cefc3f692c74d71aa3fd0",
+    "backward": 287329536 + 34717440,
+    "forward": 109736192 + 23128064,
 }
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
