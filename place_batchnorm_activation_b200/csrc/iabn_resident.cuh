@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             // tiles read again in phase B stay in L2; stashed or resident ones need not
             const bool again = (stash ? t >= tlo && t < thi : t < nring) && !ring_resident(t);
             issue(t, s, again ? pol_keep : pol_stream);
-            if (scp && t * tpg < Jc) cpp |= 1u << s;   // consumer warp 0 copies it to TMEM
+            if (scp && t * tpg < Jc) cpp |= 1u << s;   // the copier warp copies it to TMEM
         }
         // Phase B: the j-th streamed tile is t = thi-1-j, in slot t % ring.  The
         // first one of each slot is either still there from phase A or is
