@@ -40,7 +40,7 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # profiles/k_resident_resnet_trunk.md).  Reported only while the CUDA sources
 # hash to the value they were captured on; otherwise "traffic" is null.
 NCU_TRAFFIC = {
-    "sources_sha256": "fac35d2fe0c19686c916590c41760d83ed9ff523fa0dd6031c6546cb963c4439",
+    "sources_sha256": "69de1e4d13adfb6e1ad53f3e5dc9dacb52b16396833a8f25b117475ef07cd89b",
     "backward": 287329536 + 34717440,
     "forward": 109736192 + 23128064,
 }

@@ -154,6 +154,47 @@ iabn_status iabn_get_device_status(void* workspace, void* stream);
  * process so far (all devices, all threads).  Host-only; never fails. */
 uint64_t iabn_kernel_launches(void);
 
+/* Launch plans (see iabn_describe_plan). */
+typedef enum {
+    IABN_PLAN_TWOPHASE = 0,   /* statistics, finalize, apply: three plain launches */
+    IABN_PLAN_RESIDENT = 1    /* one cooperative persistent launch, one CTA per SM */
+} iabn_plan;
+
+/* Launch shape of one call; filled by iabn_describe_plan.  The fields after
+ * `launches` describe the resident plan and are 0 for the two-phase plan. */
+typedef struct {
+    int32_t plan;               /* iabn_plan */
+    int32_t launches;           /* kernels one iabn_forward / iabn_backward call launches */
+    int32_t grid;               /* CTAs (at most one per SM) */
+    int32_t threads;            /* threads per CTA */
+    int32_t smem_bytes;         /* dynamic shared memory per CTA */
+    int32_t tile_bytes;         /* bytes of each streamed tensor per full tile */
+    int32_t slots;              /* tile slots in shared memory */
+    int32_t ring;               /* slots the stream cycles through (<= slots) */
+    int32_t vectors_per_row;    /* NHWC: 16-byte vectors in a row of C channels; NCHW: 0 */
+    int32_t cols_per_thread;    /* NHWC: 16-byte columns each consumer thread owns */
+    int32_t row_phases;         /* NHWC: consumer threads sharing one column */
+    int32_t planes_per_unit;    /* NCHW: whole H*W planes per 16-byte aligned unit */
+    int32_t stash_rows;         /* NHWC: rows per consumer thread kept in Tensor Memory
+                                   between the two passes (0: none) */
+    int32_t stash_copy_engine;  /* 1: tcgen05.cp fills that stash from shared memory */
+} iabn_plan_info;
+
+/* Which plan iabn_forward (direction 0) or iabn_backward (direction 1)
+ * takes for descriptor d, and its launch shape, as decided on the host; the
+ * same environment settings apply (IABN_FORCE_PLAN=twophase, tile and ring
+ * sizes).  A resident launch the driver refuses at run time (e.g. too few
+ * co-resident CTAs) still falls back to the two-phase plan; that is not
+ * predicted here.
+ * sm_count, smem_optin: the device's SM count and opt-in shared memory per
+ * block in bytes (B200: 148 and 232448); both 0 = query the current device
+ * (IABN_ERR_CUDA if there is none).  With both given no CUDA call is made.
+ * Returns the descriptor errors of iabn_forward, IABN_ERR_INVALID_ARG for a
+ * null `out`, a direction other than 0/1 or a negative or half-given limit
+ * pair, else IABN_OK with *out filled. */
+iabn_status iabn_describe_plan(const iabn_desc* d, int32_t direction, int32_t sm_count,
+                               int32_t smem_optin, iabn_plan_info* out);
+
 /* iabn_forward without a caller-supplied workspace.  The paper has no
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory -- e.g. a plugin inside a framework whose own allocator owns

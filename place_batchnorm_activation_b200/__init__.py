@@ -10,7 +10,8 @@ Two levels:
     ``iabn_workspace_size``, ``iabn_get_device_status``: the C entry points
     with the same names and arguments (raw device pointers as ints).
   * ``forward``, ``backward``, ``update_running_stats``, ``workspace_size``,
-    ``get_device_status``: the same calls taking torch tensors.
+    ``get_device_status``: the same calls taking torch tensors;
+    ``describe_plan``: the launch plan of a descriptor, as a dict.
 """
 from __future__ import annotations
 
@@ -41,12 +42,22 @@ IABN_ACT_LEAKY_RELU, IABN_ACT_ELU, IABN_ACT_IDENTITY = 0, 1, 2
 # Symbols include/iabn.h declares (checked by the tests).
 EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_backward",
            "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches",
-           "iabn_forward_static_ws")
+           "iabn_forward_static_ws", "iabn_describe_plan")
+
+IABN_PLAN_TWOPHASE, IABN_PLAN_RESIDENT = 0, 1
+PLAN_NAMES = {IABN_PLAN_TWOPHASE: "twophase", IABN_PLAN_RESIDENT: "resident"}
 
 
 class IabnDesc(ctypes.Structure):
     _fields_ = [("n", ctypes.c_int64), ("c", ctypes.c_int64), ("h", ctypes.c_int64),
                 ("w", ctypes.c_int64), ("layout", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class IabnPlanInfo(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "plan", "launches", "grid", "threads", "smem_bytes", "tile_bytes", "slots", "ring",
+        "vectors_per_row", "cols_per_thread", "row_phases", "planes_per_unit", "stash_rows",
+        "stash_copy_engine")]
 
 
 class IabnError(RuntimeError):
@@ -86,6 +97,8 @@ def lib() -> ctypes.CDLL:
             L.iabn_kernel_launches.restype = ctypes.c_uint64
             L.iabn_forward_static_ws.argtypes = [pd, vp, vp, vp, f32, i32, f32, vp, vp, vp]
             L.iabn_forward_static_ws.restype = i32
+            L.iabn_describe_plan.argtypes = [pd, i32, i32, i32, ctypes.POINTER(IabnPlanInfo)]
+            L.iabn_describe_plan.restype = i32
             _lib = L
     return _lib
 
@@ -136,6 +149,11 @@ def iabn_forward_static_ws(desc, x_inout, gamma, beta, eps, act, act_param, save
                                             act_param, save_mean, save_var, stream))
 
 
+def iabn_describe_plan(desc, direction, sm_count, smem_optin, info) -> int:
+    return int(lib().iabn_describe_plan(ctypes.byref(desc), direction, sm_count, smem_optin,
+                                        ctypes.byref(info)))
+
+
 # ---------------------------------------------------------- tensor helpers
 
 def _dtype_code(t) -> int:
@@ -169,6 +187,19 @@ def _ok(status: int, what: str) -> None:
 
 def workspace_size(shape, layout: int, dtype: int) -> int:
     return iabn_workspace_size(make_desc(shape, layout, dtype))
+
+
+def describe_plan(shape, layout: int, dtype: int, direction: int, *, sm_count: int = 0,
+                  smem_optin: int = 0) -> dict:
+    """The launch plan and shape iabn_forward (direction 0) or iabn_backward
+    (direction 1) takes for this descriptor; sm_count and smem_optin describe
+    the device (both 0: the current device)."""
+    info = IabnPlanInfo()
+    _ok(iabn_describe_plan(make_desc(shape, layout, dtype), int(direction), int(sm_count),
+                           int(smem_optin), info), "iabn_describe_plan")
+    out = {name: int(getattr(info, name)) for name, _ in IabnPlanInfo._fields_}
+    out["plan"] = PLAN_NAMES[out["plan"]]
+    return out
 
 
 def new_workspace(shape, layout: int, dtype: int, device=None):

@@ -228,3 +228,47 @@ extern "C" iabn_status iabn_get_device_status(void* workspace, void* stream) {
 extern "C" uint64_t iabn_kernel_launches(void) {
     return g_launches.load(std::memory_order_relaxed);
 }
+
+extern "C" iabn_status iabn_describe_plan(const iabn_desc* d, int32_t direction,
+                                          int32_t sm_count, int32_t smem_optin,
+                                          iabn_plan_info* out) {
+    Geom g;
+    iabn_status st = make_geom(d, g);
+    if (st != IABN_OK) return st;
+    if (!out || (direction != 0 && direction != 1)) return IABN_ERR_INVALID_ARG;
+    if (sm_count < 0 || smem_optin < 0 || (sm_count == 0) != (smem_optin == 0))
+        return IABN_ERR_INVALID_ARG;
+    if (sm_count == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
+        int sms = 0, smem = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess)
+            return from_cuda(cudaErrorUnknown);
+        sm_count = sms;
+        smem_optin = smem;
+    }
+    memset(out, 0, sizeof(*out));
+    ResidentShape r;
+    if (forced_plan() != kTwoPhase && resident_shape(g, direction, sm_count, smem_optin, r)) {
+        out->plan = IABN_PLAN_RESIDENT;
+        out->launches = 1;
+        out->grid = r.grid;
+        out->threads = r.threads;
+        out->smem_bytes = r.smem_bytes;
+        out->tile_bytes = r.tile_bytes;
+        out->slots = r.slots;
+        out->ring = r.ring;
+        out->vectors_per_row = r.vectors_per_row;
+        out->cols_per_thread = r.cols_per_thread;
+        out->row_phases = r.row_phases;
+        out->planes_per_unit = r.planes_per_unit;
+        out->stash_rows = r.stash_rows;
+        out->stash_copy_engine = r.stash_copy_engine;
+    } else {
+        out->plan = IABN_PLAN_TWOPHASE;
+        out->launches = 3;
+    }
+    return IABN_OK;
+}

@@ -74,4 +74,17 @@ cudaError_t backward_resident(const Geom& g, const BwdArgs& a, const Workspace& 
                               cudaStream_t s);
 bool resident_supported(const Geom& g);
 
+// Launch shape of the resident plan in one direction (iabn_describe_plan).
+struct ResidentShape {
+    int grid, threads, smem_bytes, tile_bytes, slots, ring;
+    int vectors_per_row, cols_per_thread, row_phases, planes_per_unit;
+    int stash_rows, stash_copy_engine;
+};
+
+// True, with `out` filled for direction dir (0 forward, 1 backward), if the
+// calls on g take the resident plan on a device with `sms` SMs and
+// `smem_optin` bytes of opt-in shared memory per block (both directions must
+// qualify, as in resident_supported).  Host only: no CUDA call.
+bool resident_shape(const Geom& g, int dir, int sms, int smem_optin, ResidentShape& out);
+
 }  // namespace iabn

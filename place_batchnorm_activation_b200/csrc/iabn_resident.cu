@@ -205,6 +205,29 @@ bool resident_supported(const Geom& g) {
     return make_plan(g, 0, dl, P, cpt) && make_plan(g, 1, dl, P, cpt);
 }
 
+bool resident_shape(const Geom& g, int dir, int sms, int smem_optin, ResidentShape& out) {
+    DeviceLimits dl;
+    dl.sms = sms;
+    dl.smem_optin = smem_optin;
+    ResPlan P, Q;
+    int cpt, cpt_other;
+    if (!make_plan(g, dir, dl, P, cpt) || !make_plan(g, 1 - dir, dl, Q, cpt_other)) return false;
+    const bool nhwc = g.layout == kNHWC;
+    out.grid = P.G;
+    out.threads = kResThreads;
+    out.smem_bytes = P.smem_bytes;
+    out.tile_bytes = P.tile_bytes;
+    out.slots = P.nslots;
+    out.ring = P.ring;
+    out.vectors_per_row = nhwc ? P.VC : 0;
+    out.cols_per_thread = nhwc ? cpt : 0;
+    out.row_phases = nhwc ? P.RP : 0;
+    out.planes_per_unit = nhwc ? 0 : P.g;
+    out.stash_rows = P.stash;
+    out.stash_copy_engine = P.stash_cp;
+    return true;
+}
+
 cudaError_t forward_resident(const Geom& g, const FwdArgs& f, const Workspace& w,
                              cudaStream_t s) {
     const DeviceLimits dl = device_limits();
