@@ -40,7 +40,7 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # profiles/k_resident_resnet_trunk.md).  Reported only while the CUDA sources
 # hash to the value they were captured on; otherwise "traffic" is null.
 NCU_TRAFFIC = {
-    "sources_sha256": "69de1e4d13adfb6e1ad53f3e5dc9dacb52b16396833a8f25b117475ef07cd89b",
+    "sources_sha256": "3db1281b43e6e728f799c6579dc1efeb0cad3d4128120db3e5484f6b5c343786",
     "backward": 287329536 + 34717440,
     "forward": 109736192 + 23128064,
 }

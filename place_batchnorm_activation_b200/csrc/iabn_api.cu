@@ -49,7 +49,9 @@ static iabn_status make_geom(const iabn_desc* d, Geom& g) {
         return IABN_ERR_INVALID_ARG;
     const int64_t lim = (int64_t)1 << 40;
     if (d->n > lim || d->c > lim || d->h > lim || d->w > lim) return IABN_ERR_UNSUPPORTED;
-    if (d->c > ((int64_t)1 << 24)) return IABN_ERR_UNSUPPORTED;   // launch-grid limit
+    // launch-grid limit: the NHWC reductions of the two-phase plan put blocks of
+    // 256 channels on the grid's y dimension (at most 65535)
+    if (d->c > (int64_t)65535 * 256) return IABN_ERR_UNSUPPORTED;
     const __int128 hw = (__int128)d->h * d->w;
     const __int128 m = hw * d->n;
     const __int128 e = m * d->c;

@@ -12,10 +12,21 @@
 //
 // Determinism: every reduction runs in a fixed order (fixed partition of the
 // rows/planes, fixed trees), so results are bitwise reproducible.
+#include <atomic>
+
+#include "iabn_bulk.cuh"
 #include "iabn_device.cuh"
 #include "iabn_internal.h"
 
 namespace iabn {
+
+// Threads of the NHWC reductions: one column of W <= 256 channels per thread,
+// kTpRowThreads / W row phases, so several rows are read at once.
+constexpr int kTpRowThreads = 512;
+
+// Loads issued together by every thread of the reductions before the
+// values are used (the accumulation order stays row by row).
+constexpr int kTpBatch = 8;
 
 // Partial-summary slots per channel of the NHWC split statistics.
 static inline int nhwc_row_blocks(int64_t R) {
@@ -24,16 +35,25 @@ static inline int nhwc_row_blocks(int64_t R) {
 
 // ---------------------------------------------------------------- forward
 
+// Running Welford update of (n, mean, M2) with one value.
+__device__ __forceinline__ void welford_add(float v, float& n, float& mean, float& m2) {
+    n += 1.f;
+    const float d = v - mean;
+    mean += d / n;
+    m2 = fmaf(d, v - mean, m2);
+}
+
 // NHWC: block (rb, cb) owns rows [rb*R/RB, (rb+1)*R/RB) and columns
 // [cb*W, cb*W + W).  Thread t reads column t % W of rows phase, phase + RP,
-// ... (coalesced along the channel dimension) with a running Welford update,
-// then the RP row phases of each column merge in a fixed tree.
+// ... (coalesced along the channel dimension; kTpBatch rows loaded at once)
+// with a running Welford update, then the RP row phases of each column merge
+// in a fixed tree.
 template <int DT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kTpRowThreads, 2)
 k_tp_stats_nhwc(const typename Storage<DT>::T* __restrict__ x, int64_t R, int64_t C, int RB,
                 double2* __restrict__ part) {
     const int W = C < 256 ? (int)C : 256;
-    const int RP = 256 / W;
+    const int RP = kTpRowThreads / W;
     const int t = threadIdx.x;
     const int lc = t % W, phase = t / W;
     const int64_t col = (int64_t)blockIdx.y * W + lc;
@@ -41,15 +61,19 @@ k_tp_stats_nhwc(const typename Storage<DT>::T* __restrict__ x, int64_t R, int64_
     const int64_t r0 = rb * R / RB, r1 = (rb + 1) * R / RB;
     float n = 0.f, mean = 0.f, m2 = 0.f;
     if (phase < RP && col < C) {
-        for (int64_t r = r0 + phase; r < r1; r += RP) {
-            const float v = Storage<DT>::load(x + r * C + col);
-            n += 1.f;
-            const float d = v - mean;
-            mean += d / n;
-            m2 = fmaf(d, v - mean, m2);
+        const typename Storage<DT>::T* src = x + col;
+        int64_t r = r0 + phase;
+        for (; r + (kTpBatch - 1) * (int64_t)RP < r1; r += kTpBatch * (int64_t)RP) {
+            float v[kTpBatch];
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k)
+                v[k] = Storage<DT>::load(src + (r + (int64_t)k * RP) * C);
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k) welford_add(v[k], n, mean, m2);
         }
+        for (; r < r1; r += RP) welford_add(Storage<DT>::load(src + r * C), n, mean, m2);
     }
-    __shared__ float sn[256], sm[256], sq[256];
+    __shared__ float sn[kTpRowThreads], sm[kTpRowThreads], sq[kTpRowThreads];
     sn[t] = n; sm[t] = mean; sq[t] = m2;
     __syncthreads();
     for (int s = 1; s < RP; s <<= 1) {
@@ -81,13 +105,22 @@ k_tp_stats_nchw(const typename Storage<DT>::T* __restrict__ x, int64_t planes, i
     for (int64_t pl = gw; pl < planes; pl += nw) {
         const typename Storage<DT>::T* src = x + pl * HW;
         float n = 0.f, mean = 0.f, m2 = 0.f;
-        for (int64_t i = lane; i < HW; i += 32) {
-            const float v = Storage<DT>::load(src + i);
-            n += 1.f;
-            const float d = v - mean;
-            mean += d / n;
-            m2 = fmaf(d, v - mean, m2);
+        int64_t i = lane;
+        for (; i + 32 * (kTpBatch - 1) < HW; i += 32 * kTpBatch) {
+            float v[kTpBatch];
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k) v[k] = Storage<DT>::load(src + i + 32 * k);
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k) welford_add(v[k], n, mean, m2);
         }
+        // the rest of the plane: up to kTpBatch - 1 values per lane, all loaded first
+        float v[kTpBatch - 1];
+#pragma unroll
+        for (int k = 0; k < kTpBatch - 1; ++k)
+            v[k] = i + 32 * k < HW ? Storage<DT>::load(src + i + 32 * k) : 0.f;
+#pragma unroll
+        for (int k = 0; k < kTpBatch - 1; ++k)
+            if (i + 32 * k < HW) welford_add(v[k], n, mean, m2);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const float b0 = __shfl_down_sync(0xffffffffu, n, o);
@@ -185,18 +218,124 @@ k_tp_apply_fwd(typename Storage<DT>::T* __restrict__ x, int64_t E, int64_t C, in
     }
 }
 
+// Channel of a flat element index, moved without division: by one element
+// (step) or by the grid-stride loop's fixed stride (jump).  NHWC: c = i mod C;
+// NCHW: rem = i mod HW, c = (i div HW) mod C.
+struct ChannelPos {
+    int64_t c, rem;
+};
+
+template <int LAYOUT>
+struct ChannelStride {
+    int64_t C, HW, sc, sr, sq;
+    __device__ __forceinline__ void setup(int64_t stride, int64_t C_, int64_t HW_) {
+        C = C_;
+        HW = HW_;
+        sc = stride % C;
+        sr = stride % HW;
+        sq = (stride / HW) % C;
+    }
+    __device__ __forceinline__ ChannelPos at(int64_t i) const {
+        ChannelPos q;
+        if (LAYOUT == kNHWC) {
+            q.c = i % C;
+            q.rem = 0;
+        } else {
+            q.rem = i % HW;
+            q.c = (i / HW) % C;
+        }
+        return q;
+    }
+    __device__ __forceinline__ void jump(ChannelPos& q) const {
+        if (LAYOUT == kNHWC) {
+            q.c += sc;
+            if (q.c >= C) q.c -= C;
+        } else {
+            q.rem += sr;
+            int64_t carry = 0;
+            if (q.rem >= HW) {
+                q.rem -= HW;
+                carry = 1;
+            }
+            q.c += sq + carry;   // < 2C
+            if (q.c >= C) q.c -= C;
+        }
+    }
+    __device__ __forceinline__ void step(ChannelPos& q) const {
+        if (LAYOUT == kNHWC) {
+            if (++q.c == C) q.c = 0;
+        } else if (++q.rem == HW) {
+            q.rem = 0;
+            if (++q.c == C) q.c = 0;
+        }
+    }
+};
+
+// NCHW elementwise passes over 16-byte vectors (the tensors start on a
+// 16-byte boundary): thread t takes vectors t, t + nt, t + 2nt, ... two at a
+// time, both loaded before either is used; the last E mod VE elements go one
+// per thread to the first threads of the grid.  The eight (or four) values of
+// a vector lie in one or two planes, so the lanes of a warp read the
+// coefficients of a few neighbouring channels.  In NHWC they would read eight
+// channels each, 128 bytes apart across the lanes (one L1 wavefront per
+// element), so NHWC keeps the scalar pass above, whose lanes read
+// consecutive channels.
+template <int DT, int ACT, int LAYOUT>
+__global__ void __launch_bounds__(256)
+k_tp_apply_fwd_vec(typename Storage<DT>::T* __restrict__ x, int64_t E, int64_t C,
+                   int64_t HW, const float4* __restrict__ coef, float p) {
+    constexpr int VE = Vec<DT>::N;
+    const int64_t NV = E / VE;
+    const int64_t nt = (int64_t)gridDim.x * blockDim.x;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint4* xv = reinterpret_cast<uint4*>(x);
+    ChannelStride<LAYOUT> cs;
+    cs.setup(2 * nt * VE, C, HW);
+    auto apply = [&](uint4& u, ChannelPos q) {
+        float f[VE];
+        Vec<DT>::unpack(u, f);
+#pragma unroll
+        for (int k = 0; k < VE; ++k) {
+            const float4 kk = __ldg(coef + q.c);
+            f[k] = act_forward<ACT, DT>(fmaf(f[k] - kk.x, kk.y, kk.z), p);
+            cs.step(q);
+        }
+        u = Vec<DT>::pack(f);
+    };
+    ChannelPos q0 = cs.at(t * VE), q1 = cs.at((t + nt) * VE);
+    for (int64_t v = t; v < NV; v += 2 * nt) {
+        const bool two = v + nt < NV;
+        uint4 a = xv[v];
+        uint4 b = two ? xv[v + nt] : make_uint4(0u, 0u, 0u, 0u);
+        apply(a, q0);
+        xv[v] = a;
+        if (two) {
+            apply(b, q1);
+            xv[v + nt] = b;
+        }
+        cs.jump(q0);
+        cs.jump(q1);
+    }
+    const int64_t i = NV * VE + t;
+    if (i < E) {
+        const float4 kk = __ldg(coef + cs.at(i).c);
+        const float xi = Storage<DT>::load(x + i);
+        Storage<DT>::store(x + i, act_forward<ACT, DT>(fmaf(xi - kk.x, kk.y, kk.z), p));
+    }
+}
+
 // --------------------------------------------------------------- backward
 
 // Per-channel sums S1 = sum dy and S2 = sum dy*xhat, xhat = (y - beta)/gamma
 // recovered from z.  Same partition and merge order as the statistics.
 template <int DT, int ACT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kTpRowThreads, 2)
 k_tp_reduce_nhwc(const typename Storage<DT>::T* __restrict__ z,
                  const typename Storage<DT>::T* __restrict__ dz, int64_t R, int64_t C, int RB,
                  const float* __restrict__ gamma, const float* __restrict__ beta, float p,
                  float inv_p, double2* __restrict__ part) {
     const int W = C < 256 ? (int)C : 256;
-    const int RP = 256 / W;
+    const int RP = kTpRowThreads / W;
     const int t = threadIdx.x;
     const int lc = t % W, phase = t / W;
     const int64_t col = (int64_t)blockIdx.y * W + lc;
@@ -206,16 +345,30 @@ k_tp_reduce_nhwc(const typename Storage<DT>::T* __restrict__ z,
     if (phase < RP && col < C) {
         const float ig = 1.f / gamma[col];
         const float nb = -beta[col] * ig;
-        for (int64_t r = r0 + phase; r < r1; r += RP) {
-            const int64_t k = r * C + col;
+        auto add = [&](float zv, float dzv) {
             float y, dy;
-            act_backward<ACT, DT>(Storage<DT>::load(z + k), Storage<DT>::load(dz + k), p, inv_p,
-                                  y, dy);
+            act_backward<ACT, DT>(zv, dzv, p, inv_p, y, dy);
             s1 += dy;
             s2 = fmaf(dy, fmaf(y, ig, nb), s2);
+        };
+        int64_t r = r0 + phase;
+        for (; r + (kTpBatch - 1) * (int64_t)RP < r1; r += kTpBatch * (int64_t)RP) {
+            float zv[kTpBatch], dzv[kTpBatch];
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k) {
+                const int64_t e = (r + (int64_t)k * RP) * C + col;
+                zv[k] = Storage<DT>::load(z + e);
+                dzv[k] = Storage<DT>::load(dz + e);
+            }
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k) add(zv[k], dzv[k]);
+        }
+        for (; r < r1; r += RP) {
+            const int64_t e = r * C + col;
+            add(Storage<DT>::load(z + e), Storage<DT>::load(dz + e));
         }
     }
-    __shared__ float a[256], b[256];
+    __shared__ float a[kTpRowThreads], b[kTpRowThreads];
     a[t] = s1; b[t] = s2;
     __syncthreads();
     for (int s = 1; s < RP; s <<= 1) {
@@ -243,14 +396,36 @@ k_tp_reduce_nchw(const typename Storage<DT>::T* __restrict__ z,
         const float ig = 1.f / gamma[c];
         const float nb = -beta[c] * ig;
         float s1 = 0.f, s2 = 0.f;
-        for (int64_t i = lane; i < HW; i += 32) {
-            const int64_t k = pl * HW + i;
+        auto add = [&](float zv, float dzv) {
             float y, dy;
-            act_backward<ACT, DT>(Storage<DT>::load(z + k), Storage<DT>::load(dz + k), p, inv_p,
-                                  y, dy);
+            act_backward<ACT, DT>(zv, dzv, p, inv_p, y, dy);
             s1 += dy;
             s2 = fmaf(dy, fmaf(y, ig, nb), s2);
+        };
+        const typename Storage<DT>::T* zp = z + pl * HW;
+        const typename Storage<DT>::T* dzp = dz + pl * HW;
+        int64_t i = lane;
+        for (; i + 32 * (kTpBatch - 1) < HW; i += 32 * kTpBatch) {
+            float zv[kTpBatch], dzv[kTpBatch];
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k) {
+                zv[k] = Storage<DT>::load(zp + i + 32 * k);
+                dzv[k] = Storage<DT>::load(dzp + i + 32 * k);
+            }
+#pragma unroll
+            for (int k = 0; k < kTpBatch; ++k) add(zv[k], dzv[k]);
         }
+        // the rest of the plane: up to kTpBatch - 1 pairs per lane, all loaded first
+        float zv[kTpBatch - 1], dzv[kTpBatch - 1];
+#pragma unroll
+        for (int k = 0; k < kTpBatch - 1; ++k) {
+            const bool in = i + 32 * k < HW;
+            zv[k] = in ? Storage<DT>::load(zp + i + 32 * k) : 0.f;
+            dzv[k] = in ? Storage<DT>::load(dzp + i + 32 * k) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kTpBatch - 1; ++k)
+            if (i + 32 * k < HW) add(zv[k], dzv[k]);
         s1 = warp_sum(s1);
         s2 = warp_sum(s2);
         if (lane == 0) part[pl] = make_double2(s1, s2);
@@ -319,6 +494,60 @@ k_tp_apply_bwd(const typename Storage<DT>::T* __restrict__ z, typename Storage<D
     }
 }
 
+template <int DT, int ACT, int LAYOUT>
+__global__ void __launch_bounds__(256)
+k_tp_apply_bwd_vec(const typename Storage<DT>::T* __restrict__ z,
+                   typename Storage<DT>::T* dz, int64_t E, int64_t C, int64_t HW,
+                   const float4* __restrict__ coef, float p, float inv_p) {
+    constexpr int VE = Vec<DT>::N;
+    const int64_t NV = E / VE;
+    const int64_t nt = (int64_t)gridDim.x * blockDim.x;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint4* zv = reinterpret_cast<const uint4*>(z);
+    uint4* dzv = reinterpret_cast<uint4*>(dz);
+    ChannelStride<LAYOUT> cs;
+    cs.setup(2 * nt * VE, C, HW);
+    auto apply = [&](const uint4& uz, uint4& ud, ChannelPos q) {
+        float fz[VE], fd[VE];
+        Vec<DT>::unpack(uz, fz);
+        Vec<DT>::unpack(ud, fd);
+#pragma unroll
+        for (int k = 0; k < VE; ++k) {
+            const float4 kk = __ldg(coef + q.c);
+            float y, dy;
+            act_backward<ACT, DT>(fz[k], fd[k], p, inv_p, y, dy);
+            fd[k] = fmaf(kk.x, dy, fmaf(kk.y, y, kk.z));
+            cs.step(q);
+        }
+        ud = Vec<DT>::pack(fd);
+    };
+    ChannelPos q0 = cs.at(t * VE), q1 = cs.at((t + nt) * VE);
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t v = t; v < NV; v += 2 * nt) {
+        const bool two = v + nt < NV;
+        const uint4 za = __ldg(zv + v);
+        uint4 da = dzv[v];
+        const uint4 zb = two ? __ldg(zv + v + nt) : zero;
+        uint4 db = two ? dzv[v + nt] : zero;
+        apply(za, da, q0);
+        dzv[v] = da;
+        if (two) {
+            apply(zb, db, q1);
+            dzv[v + nt] = db;
+        }
+        cs.jump(q0);
+        cs.jump(q1);
+    }
+    const int64_t i = NV * VE + t;
+    if (i < E) {
+        const float4 kk = __ldg(coef + cs.at(i).c);
+        float y, dy;
+        act_backward<ACT, DT>(Storage<DT>::load(z + i), Storage<DT>::load(dz + i), p, inv_p, y,
+                              dy);
+        Storage<DT>::store(dz + i, fmaf(kk.x, dy, fmaf(kk.y, y, kk.z)));
+    }
+}
+
 // ------------------------------------------------------------ running stats
 
 __global__ void k_running_update(int64_t C, float unbias, const float* __restrict__ mean,
@@ -339,12 +568,41 @@ static int grid_for(int64_t work, int per_block, int cap) {
     return (int)g;
 }
 
+// CTAs of `kern` (`threads` threads, no dynamic shared memory) resident on
+// one SM, queried once per kernel; the grid-stride kernels are sized to one
+// full wave of them (a second, partial wave would run its whole share alone).
+template <typename Kern>
+static int ctas_per_sm(Kern kern, int threads, std::atomic<int>& cache) {
+    int nb = cache.load(std::memory_order_relaxed);
+    if (nb > 0) return nb;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, threads, 0) != cudaSuccess ||
+        nb < 1) {
+        cudaGetLastError();
+        return 4;
+    }
+    cache.store(nb, std::memory_order_relaxed);
+    return nb;
+}
+
+// Grid of an elementwise pass: two 16-byte vectors per thread per step.
+static int apply_grid(const Geom& g, int sms, int per_sm) {
+    const int64_t nv = g.E / (16 / g.esize);
+    return grid_for(nv, 2 * 256, sms * per_sm);
+}
+
 template <int DT, int ACT, int LAYOUT>
 static cudaError_t fwd_apply(const Geom& g, void* x, const float4* coef, float p,
                              cudaStream_t s, int sms) {
     using T = typename Storage<DT>::T;
-    k_tp_apply_fwd<DT, ACT, LAYOUT><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
-        static_cast<T*>(x), g.E, g.C, g.HW, coef, p);
+    if (LAYOUT == kNHWC) {
+        k_tp_apply_fwd<DT, ACT, kNHWC><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
+            static_cast<T*>(x), g.E, g.C, g.HW, coef, p);
+    } else {
+        static std::atomic<int> occ{0};
+        auto kern = k_tp_apply_fwd_vec<DT, ACT, kNCHW>;
+        kern<<<apply_grid(g, sms, ctas_per_sm(kern, 256, occ)), 256, 0, s>>>(
+            static_cast<T*>(x), g.E, g.C, g.HW, coef, p);
+    }
     count_launches(1);
     return cudaGetLastError();
 }
@@ -360,13 +618,15 @@ static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Worksp
         RB = nhwc_row_blocks(g.R);
         const int W = g.C < 256 ? (int)g.C : 256;
         dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
-        k_tp_stats_nhwc<DT><<<grid, 256, 0, s>>>(x, g.R, g.C, RB, w.part);
+        k_tp_stats_nhwc<DT><<<grid, kTpRowThreads, 0, s>>>(x, g.R, g.C, RB, w.part);
         K = RB;
         count_launches(1);
     } else {
         const int64_t planes = g.N * g.C;
-        k_tp_stats_nchw<DT><<<grid_for(planes, 8, sms * 16), 256, 0, s>>>(x, planes, g.HW,
-                                                                          w.part);
+        static std::atomic<int> occ{0};
+        const int per_sm = ctas_per_sm(k_tp_stats_nchw<DT>, 256, occ);
+        k_tp_stats_nchw<DT><<<grid_for(planes, 8, sms * per_sm), 256, 0, s>>>(x, planes, g.HW,
+                                                                              w.part);
         K = g.N;
         count_launches(1);
     }
@@ -416,13 +676,15 @@ static cudaError_t bwd_twophase_act(const Geom& g, const BwdArgs& a, const Works
         const int RB = nhwc_row_blocks(g.R);
         const int W = g.C < 256 ? (int)g.C : 256;
         dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
-        k_tp_reduce_nhwc<DT, ACT><<<grid, 256, 0, s>>>(z, dz, g.R, g.C, RB, a.gamma, a.beta, p,
-                                                       inv_p, w.part);
+        k_tp_reduce_nhwc<DT, ACT><<<grid, kTpRowThreads, 0, s>>>(z, dz, g.R, g.C, RB, a.gamma,
+                                                                 a.beta, p, inv_p, w.part);
         K = RB;
         count_launches(1);
     } else {
         const int64_t planes = g.N * g.C;
-        k_tp_reduce_nchw<DT, ACT><<<grid_for(planes, 8, sms * 16), 256, 0, s>>>(
+        static std::atomic<int> occ{0};
+        const int per_sm = ctas_per_sm(k_tp_reduce_nchw<DT, ACT>, 256, occ);
+        k_tp_reduce_nchw<DT, ACT><<<grid_for(planes, 8, sms * per_sm), 256, 0, s>>>(
             z, dz, planes, g.C, g.HW, a.gamma, a.beta, p, inv_p, w.part);
         K = g.N;
         count_launches(1);
@@ -435,13 +697,15 @@ static cudaError_t bwd_twophase_act(const Geom& g, const BwdArgs& a, const Works
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int grid = grid_for(g.E, 256, sms * 8);
-    if (g.layout == kNHWC)
-        k_tp_apply_bwd<DT, ACT, kNHWC><<<grid, 256, 0, s>>>(z, dz, g.E, g.C, g.HW, w.coef, p,
-                                                            inv_p);
-    else
-        k_tp_apply_bwd<DT, ACT, kNCHW><<<grid, 256, 0, s>>>(z, dz, g.E, g.C, g.HW, w.coef, p,
-                                                            inv_p);
+    if (g.layout == kNHWC) {
+        k_tp_apply_bwd<DT, ACT, kNHWC><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
+            z, dz, g.E, g.C, g.HW, w.coef, p, inv_p);
+    } else {
+        static std::atomic<int> occ{0};
+        auto kern = k_tp_apply_bwd_vec<DT, ACT, kNCHW>;
+        kern<<<apply_grid(g, sms, ctas_per_sm(kern, 256, occ)), 256, 0, s>>>(
+            z, dz, g.E, g.C, g.HW, w.coef, p, inv_p);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

@@ -177,6 +177,13 @@ def test_describe_rejects_bad_arguments():
     assert iabn.iabn_describe_plan(bad, 0, 148, 232448, info) == iabn.IABN_ERR_INVALID_ARG
     huge = iabn.make_desc((1, 1 << 25, 1, 2), wl.NHWC, wl.BF16)    # beyond the grid limit
     assert iabn.iabn_describe_plan(huge, 0, 148, 232448, info) == iabn.IABN_ERR_UNSUPPORTED
+    # channels: at most 65535 blocks of 256 on the grid's y dimension
+    edge = iabn.make_desc((1, 65535 * 256, 1, 2), wl.NHWC, wl.BF16)
+    assert iabn.iabn_describe_plan(edge, 0, 148, 232448, info) == iabn.IABN_OK
+    assert info.plan == iabn.IABN_PLAN_TWOPHASE
+    over = iabn.make_desc((1, 65535 * 256 + 8, 1, 2), wl.NHWC, wl.BF16)
+    assert iabn.iabn_describe_plan(over, 0, 148, 232448, info) == iabn.IABN_ERR_UNSUPPORTED
+    assert iabn.iabn_workspace_size(over) == 0
     lib = iabn.lib()
     assert lib.iabn_describe_plan(iabn.ctypes.byref(d), 0, 148, 232448, None) == \
         iabn.IABN_ERR_INVALID_ARG
