@@ -67,6 +67,8 @@ def _load():
                 f = getattr(lib, name)
                 f.argtypes = geom + [pd, pd, pd, pd, pd, d, i32, d, pd, pd, pd]
                 f.restype = i32
+            lib.orc_inference.argtypes = geom + [pd, pd, pd, pd, pd, d, i32, d, pd]
+            lib.orc_inference.restype = i32
             lib.orc_running_update.argtypes = [i64, i64, pd, pd, d, pd, pd]
             lib.orc_running_update.restype = i32
             _lib = lib
@@ -158,6 +160,17 @@ def backward_inplace(shape, layout, z, dz, gamma, beta, var, eps, kind, p, form:
     _check(fn(n, c, h, w, int(layout), _p(z), _p(dz), _p(g), _p(b), _p(v), float(eps),
               int(kind), float(p), _p(dx), _p(dg), _p(db)), f"backward_inplace_{form}")
     return {"dx": dx, "dgamma": dg, "dbeta": db}
+
+
+def inference(shape, layout, x, gamma, beta, running_mean, running_var, eps, kind, p):
+    """Evaluation-mode z (fp64) from fixed statistics; x in the given layout."""
+    n, c, h, w = (int(v) for v in shape)
+    x, g, b = _f64(x), _f64(gamma), _f64(beta)
+    rm, rv = _f64(running_mean), _f64(running_var)
+    z = np.empty_like(x)
+    _check(_load().orc_inference(n, c, h, w, int(layout), _p(x), _p(g), _p(b), _p(rm), _p(rv),
+                                 float(eps), int(kind), float(p), _p(z)), "inference")
+    return z
 
 
 def running_update(count, mean, var, momentum, running_mean, running_var):

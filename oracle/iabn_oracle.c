@@ -277,6 +277,30 @@ int orc_backward_inplace_2(int64_t n, int64_t c, int64_t h, int64_t w, int layou
 }
 
 /* ----------------------------------------------------- running statistics */
+/* ------------------------------------------------------------ inference */
+/* [BN] Algorithm 2 (the inference network): the batch statistics are
+ * replaced by fixed estimates of the population's, here the running
+ * averages; then the same scale, shift and activation as in training. */
+
+int orc_inference(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
+                  const double* x, const double* gamma, const double* beta,
+                  const double* running_mean, const double* running_var,
+                  double eps, int act, double act_param, double* z_out) {
+    if (check_geom(n, c, h, w, layout)) return -1;
+    const int64_t HW = h * w;
+    for (int64_t ch = 0; ch < c; ++ch) {
+        double rstd = 1.0 / sqrt(running_var[ch] + eps);
+        for (int64_t i = 0; i < n; ++i)
+            for (int64_t p = 0; p < HW; ++p) {
+                int64_t k = at(layout, c, HW, i, ch, p);
+                double xhat = (x[k] - running_mean[ch]) * rstd;
+                double y = gamma[ch] * xhat + beta[ch];
+                z_out[k] = orc_act(y, act, act_param);
+            }
+    }
+    return 0;
+}
+
 /* [BN] Algorithm 2 uses the unbiased variance for inference; the momentum
  * form of the running average is the usual framework convention. */
 int orc_running_update(int64_t c, int64_t count, const double* mean, const double* var,

@@ -100,6 +100,18 @@ int orc_backward_inplace_2(int64_t n, int64_t c, int64_t h, int64_t w, int layou
                            const double* var, double eps, int act, double act_param,
                            double* dx, double* dgamma, double* dbeta);
 
+/* Inference (evaluation mode): the layer with fixed statistics in place of
+ * the batch's ([BN] Algorithm 2, the inference network: normalise with the
+ * population mean and variance the running averages estimate; [ABN] section
+ * 3, "Batch Normalization Review": scale and shift by gamma and beta):
+ *   xhat = (x - running_mean) / sqrt(running_var + eps),
+ *   y = gamma*xhat + beta,  z = phi(y).
+ * Returns 0, or -1 on a bad argument. */
+int orc_inference(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
+                  const double* x, const double* gamma, const double* beta,
+                  const double* running_mean, const double* running_var,
+                  double eps, int act, double act_param, double* z_out);
+
 /* Running statistics (momentum form, unbiased running variance), in place. */
 int orc_running_update(int64_t c, int64_t count, const double* mean, const double* var,
                        double momentum, double* running_mean, double* running_var);

@@ -197,6 +197,71 @@ def test_forward_invariants():
     np.testing.assert_array_equal(wl.logical_view(znhwc, shape, 1), zr.reshape(shape))
 
 
+# -------------------------------------------------------------- inference
+
+def _torch_inference(xl, g, b, rm, rv, eps, act, p):
+    """PyTorch fp64 batch_norm in evaluation mode, then the activation."""
+    y = torch.nn.functional.batch_norm(torch.tensor(xl), torch.tensor(rm), torch.tensor(rv),
+                                       torch.tensor(g), torch.tensor(b), training=False,
+                                       eps=eps)
+    if act == oracle.LEAKY_RELU:
+        return torch.nn.functional.leaky_relu(y, p).numpy()
+    if act == oracle.ELU:
+        return torch.nn.functional.elu(y, p).numpy()
+    return y.numpy()
+
+
+@pytest.mark.parametrize("layout", [oracle.NCHW, oracle.NHWC])
+@pytest.mark.parametrize("act,p", ACTS)
+def test_inference_matches_torch_eval_batch_norm(layout, act, p):
+    rng = np.random.default_rng(40 + layout)
+    shape = (3, 5, 4, 6)
+    xl, g, b, _ = _rand_layer(rng, shape, layout)
+    rm = rng.uniform(-2, 2, shape[1])
+    rv = rng.uniform(0.25, 9, shape[1])
+    ref = _torch_inference(xl, g, b, rm, rv, 1e-5, act, p)
+    z = oracle.inference(shape, layout, _flat(xl, layout), g, b, rm, rv, 1e-5, act, p)
+    _close(z, _flat(ref, layout), rel=1e-12, abs_=1e-14)
+
+
+def test_inference_with_the_batch_statistics_is_the_training_forward():
+    """Fed the batch's own mean and biased variance, evaluation mode gives
+    the training-mode z bit for bit (same formula, same precision)."""
+    rng = np.random.default_rng(42)
+    for layout in (oracle.NCHW, oracle.NHWC):
+        shape = (2, 7, 3, 5)
+        xl, g, b, _ = _rand_layer(rng, shape, layout)
+        for act, p in ACTS:
+            fw = oracle.forward(shape, layout, _flat(xl, layout), g, b, 1e-5, act, p)
+            z = oracle.inference(shape, layout, _flat(xl, layout), g, b, fw["mean"], fw["var"],
+                                 1e-5, act, p)
+            np.testing.assert_array_equal(z, fw["z"])
+
+
+def test_inference_closed_forms():
+    """Dyadic statistics make every step exact: with running_var + eps = 4
+    the layer is z = phi(gamma*(x - m)/2 + beta) exactly; with m = 0, v = 1,
+    eps = 0, gamma = 1 and beta = 0 it is phi itself."""
+    rng = np.random.default_rng(43)
+    shape = (2, 3, 2, 4)
+    xl = rng.integers(-64, 64, shape) / 8.0
+    for act, p in ((oracle.LEAKY_RELU, 0.25), (oracle.IDENTITY, 0.0)):
+        g = np.array([1.0, -0.5, 2.0])
+        b = np.array([0.25, 0.0, -1.0])
+        m = np.array([0.5, -1.0, 0.0])
+        v = np.array([3.75, 3.75, 3.75])
+        z = oracle.inference(shape, oracle.NCHW, _flat(xl, 0), g, b, m, v, 0.25, act, p)
+        y = g[None, :, None, None] * (xl - m[None, :, None, None]) / 2 + b[None, :, None, None]
+        want = np.where(y > 0, y, p * y) if act == oracle.LEAKY_RELU else y
+        np.testing.assert_array_equal(z.reshape(shape), want)
+    one = np.ones(3)
+    zero = np.zeros(3)
+    z = oracle.inference(shape, oracle.NHWC, _flat(xl, 1), one, zero, zero, one, 0.0,
+                         oracle.ELU, 1.0)
+    np.testing.assert_array_equal(z, np.where(_flat(xl, 1) > 0, _flat(xl, 1),
+                                              np.expm1(_flat(xl, 1))))
+
+
 # --------------------------------------------------------------- backward
 
 @pytest.mark.parametrize("layout", [oracle.NCHW, oracle.NHWC])
