@@ -40,7 +40,7 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # profiles/k_resident_resnet_trunk.md).  Reported only while the CUDA sources
 # hash to the value they were captured on; otherwise "traffic" is null.
 NCU_TRAFFIC = {
-    "sources_sha256": "3db1281b43e6e728f799c6579dc1efeb0cad3d4128120db3e5484f6b5c343786",
+    "sources_sha256": "3f329c8647407bf0f144fbd15a039b5083c86d7822a943c50809dc7cfbefd2eb",
     "backward": 287329536 + 34717440,
     "forward": 109736192 + 23128064,
 }
@@ -425,6 +425,46 @@ def bench_other_workloads(flush, steps, warmup, hbm_peak, device):
     return out
 
 
+def bench_inference(flush, steps, warmup, hbm_peak, device):
+    """Evaluation mode (iabn_inference) on the ResNet-trunk layer, with the
+    running statistics of three training steps; L2 flushed before every
+    call, x restored between calls (outside the timed events).  Traffic:
+    read x, write z = 2*E*s."""
+    import torch
+    import workloads as wl
+    sp = wl.spec(1)
+    L = Layer(sp, sp.seed, device)
+    for _ in range(3):
+        L.restore()
+        L.fwd()
+        L.run()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    recs = []
+    l0 = L.iabn.iabn_kernel_launches()
+    for i in range(warmup + steps):
+        L.restore()
+        flush.zero_()
+        a, b = ev(), ev()
+        a.record()
+        L.iabn.inference(L.x, L.gamma, L.beta, L.rmean, L.rvar, L.ws, shape=sp.shape,
+                         layout=sp.layout, eps=sp.eps, act=sp.act, act_param=sp.act_param)
+        b.record()
+        if i >= warmup:
+            recs.append((a, b))
+    torch.cuda.synchronize()
+    calls = warmup + steps
+    launches = (L.iabn.iabn_kernel_launches() - l0) / calls
+    t = statistics.median(a.elapsed_time(b) for a, b in recs)
+    nbytes = 2 * sp.numel * sp.itemsize
+    gbs = nbytes / (t * 1e-3) / 1e9
+    del L
+    torch.cuda.empty_cache()
+    return {"us": round(t * 1e3, 2), "gbs": round(gbs, 1),
+            "frac_measured_hbm": round(gbs / hbm_peak, 4), "bytes_per_call": nbytes,
+            "launches_per_call": launches,
+            "plan": "two launches: per-channel coefficients, then the elementwise pass"}
+
+
 # ------------------------------------------------------------ CPU (oracle)
 
 def oracle_pass(sp_sample):
@@ -603,6 +643,11 @@ def main():
     extra = {}
     if not args.no_extra and world == 1:
         extra = bench_other_workloads(flush, max(5, args.steps // 5), 3, hbm_peak, device)
+        try:
+            extra["inference_resnet_trunk"] = bench_inference(flush, max(5, args.steps // 5), 3,
+                                                              hbm_peak, device)
+        except Exception as e:  # reported in the line; never fatal for the headline
+            extra["inference_resnet_trunk"] = {"error": f"{type(e).__name__}: {e}"}
 
     if rank == 0:
         bwd_bytes = 3 * sp.numel * sp.itemsize

@@ -85,8 +85,10 @@ typedef struct {
     int32_t dtype;
 } iabn_desc;
 
-/* Bytes of workspace the forward and backward calls need for descriptor `d`
- * (a multiple of 256).  Returns 0 if the descriptor is invalid.  Host-only. */
+/* Bytes of workspace the forward, backward and inference calls need for
+ * descriptor `d` (a multiple of 256).  Returns 0 if the descriptor is
+ * invalid; M = 1 is valid here (iabn_inference takes it, the training calls
+ * do not).  Host-only. */
 size_t iabn_workspace_size(const iabn_desc* d);
 
 /* Forward, training mode ([ABN] section 3, "Batch Normalization Review" and
@@ -129,6 +131,25 @@ iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz_inout,
                           int32_t act, float act_param,
                           float* dgamma, float* dbeta,
                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Inference, i.e. evaluation mode ([BN] Algorithm 2, the inference network;
+ * [ABN] section 3, "Batch Normalization Review" for the scale and shift):
+ *   xhat = (x - running_mean_c) / sqrt(running_var_c + eps),
+ *   z = phi(gamma_c*xhat + beta_c), written over x_inout.
+ * No statistics are computed or written; M >= 1.
+ * x_inout   [N,C,H,W] in `d->layout`/`d->dtype`: x on entry, z on return.
+ * gamma, beta, running_mean, running_var [C] float32; running_var_c + eps
+ *           must be > 0.
+ * eps >= 0; act, act_param as for iabn_forward.
+ * workspace, ws_bytes: scratch of at least iabn_workspace_size(d) bytes (its
+ *           coefficient area is written); it need not be zero-filled.
+ * Launches two kernels: the per-channel coefficients, then the forward's
+ * elementwise pass.  Arguments are checked as for iabn_forward. */
+iabn_status iabn_inference(const iabn_desc* d, void* x_inout,
+                           const float* gamma, const float* beta,
+                           const float* running_mean, const float* running_var, float eps,
+                           int32_t act, float act_param,
+                           void* workspace, size_t ws_bytes, void* stream);
 
 /* Running statistics ([BN] Algorithm 2 uses the unbiased variance for
  * inference; the momentum form is the usual framework convention):

@@ -6,10 +6,11 @@ memory and streams.  There is no CPU fallback: if the library is missing or
 no GPU is present, calls raise.
 
 Two levels:
-  * ``iabn_forward``, ``iabn_backward``, ``iabn_update_running_stats``,
-    ``iabn_workspace_size``, ``iabn_get_device_status``: the C entry points
-    with the same names and arguments (raw device pointers as ints).
-  * ``forward``, ``backward``, ``update_running_stats``, ``workspace_size``,
+  * ``iabn_forward``, ``iabn_backward``, ``iabn_inference``,
+    ``iabn_update_running_stats``, ``iabn_workspace_size``,
+    ``iabn_get_device_status``: the C entry points with the same names and
+    arguments (raw device pointers as ints).
+  * ``forward``, ``backward``, ``inference``, ``update_running_stats``, ``workspace_size``,
     ``get_device_status``: the same calls taking torch tensors;
     ``describe_plan``: the launch plan of a descriptor, as a dict.
 """
@@ -42,7 +43,7 @@ IABN_ACT_LEAKY_RELU, IABN_ACT_ELU, IABN_ACT_IDENTITY = 0, 1, 2
 # Symbols include/iabn.h declares (checked by the tests).
 EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_backward",
            "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches",
-           "iabn_forward_static_ws", "iabn_describe_plan")
+           "iabn_forward_static_ws", "iabn_describe_plan", "iabn_inference")
 
 IABN_PLAN_TWOPHASE, IABN_PLAN_RESIDENT = 0, 1
 PLAN_NAMES = {IABN_PLAN_TWOPHASE: "twophase", IABN_PLAN_RESIDENT: "resident"}
@@ -89,6 +90,9 @@ def lib() -> ctypes.CDLL:
             L.iabn_backward.argtypes = [pd, vp, vp, vp, vp, vp, f32, i32, f32, vp, vp, vp,
                                         ctypes.c_size_t, vp]
             L.iabn_backward.restype = i32
+            L.iabn_inference.argtypes = [pd, vp, vp, vp, vp, vp, f32, i32, f32, vp,
+                                         ctypes.c_size_t, vp]
+            L.iabn_inference.restype = i32
             L.iabn_update_running_stats.argtypes = [i64, i64, vp, vp, vp, vp, f32, vp]
             L.iabn_update_running_stats.restype = i32
             L.iabn_get_device_status.argtypes = [vp, vp]
@@ -125,6 +129,13 @@ def iabn_backward(desc, z, dz_inout, gamma, beta, save_var, eps, act, act_param,
     return int(lib().iabn_backward(ctypes.byref(desc), z, dz_inout, gamma, beta, save_var,
                                    eps, act, act_param, dgamma, dbeta, workspace, ws_bytes,
                                    stream))
+
+
+def iabn_inference(desc, x_inout, gamma, beta, running_mean, running_var, eps, act, act_param,
+                   workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_inference(ctypes.byref(desc), x_inout, gamma, beta, running_mean,
+                                    running_var, eps, act, act_param, workspace, ws_bytes,
+                                    stream))
 
 
 def iabn_update_running_stats(c, count, save_mean, save_var, running_mean, running_var,
@@ -226,6 +237,17 @@ def backward(z, dz, gamma, beta, save_var, dgamma, dbeta, workspace, *, shape, l
                       float(eps), int(act), float(act_param), _ptr(dgamma), _ptr(dbeta),
                       _ptr(workspace), workspace.numel() * workspace.element_size(),
                       _stream_ptr(stream)), "iabn_backward")
+
+
+def inference(x, gamma, beta, running_mean, running_var, workspace, *, shape, layout: int,
+              eps: float, act: int, act_param: float, stream=None) -> None:
+    """Evaluation mode: x is overwritten with z computed from the running
+    statistics."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    _ok(iabn_inference(desc, _ptr(x), _ptr(gamma), _ptr(beta), _ptr(running_mean),
+                       _ptr(running_var), float(eps), int(act), float(act_param),
+                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                       _stream_ptr(stream)), "iabn_inference")
 
 
 def update_running_stats(save_mean, save_var, running_mean, running_var, *, count: int,

@@ -40,8 +40,10 @@ static size_t workspace_bytes(const Geom& g) {
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Checks the descriptor; fills g.  Returns IABN_OK or the error.
-static iabn_status make_geom(const iabn_desc* d, Geom& g) {
+// Checks the descriptor; fills g.  Returns IABN_OK or the error.  min_m is
+// the least number of values per channel the call accepts: 2 for the
+// training calls (a variance needs two values), 1 for inference.
+static iabn_status make_geom(const iabn_desc* d, Geom& g, int64_t min_m = 2) {
     if (!d) return IABN_ERR_INVALID_ARG;
     if (d->n <= 0 || d->c <= 0 || d->h <= 0 || d->w <= 0) return IABN_ERR_INVALID_ARG;
     if (d->layout != IABN_NCHW && d->layout != IABN_NHWC) return IABN_ERR_INVALID_ARG;
@@ -56,7 +58,7 @@ static iabn_status make_geom(const iabn_desc* d, Geom& g) {
     const __int128 m = hw * d->n;
     const __int128 e = m * d->c;
     if (e * 4 > (__int128)INT64_MAX / 2) return IABN_ERR_UNSUPPORTED;
-    if (m < 2) return IABN_ERR_INVALID_ARG;
+    if (m < min_m) return IABN_ERR_INVALID_ARG;
     // Partial slots and the count of values per channel must stay exact.
     if ((__int128)d->n * d->c > ((__int128)1 << 40)) return IABN_ERR_UNSUPPORTED;
     if (m > ((__int128)1 << 52)) return IABN_ERR_UNSUPPORTED;
@@ -138,7 +140,7 @@ using namespace iabn;
 
 extern "C" size_t iabn_workspace_size(const iabn_desc* d) {
     Geom g;
-    if (make_geom(d, g) != IABN_OK) return 0;
+    if (make_geom(d, g, 1) != IABN_OK) return 0;
     return workspace_bytes(g);
 }
 
@@ -197,6 +199,28 @@ extern "C" iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz
         cudaGetLastError();
     }
     return from_cuda(backward_twophase(g, a, w, s, device_sms(dev)));
+}
+
+extern "C" iabn_status iabn_inference(const iabn_desc* d, void* x_inout, const float* gamma,
+                                      const float* beta, const float* running_mean,
+                                      const float* running_var, float eps, int32_t act,
+                                      float act_param, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+    Geom g;
+    iabn_status st = make_geom(d, g, 1);
+    if (st != IABN_OK) return st;
+    if (!x_inout || !gamma || !beta || !running_mean || !running_var) return IABN_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !isfinite(eps)) return IABN_ERR_INVALID_ARG;
+    if ((st = check_act(act, act_param)) != IABN_OK) return st;
+    if (!aligned16(x_inout)) return IABN_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < workspace_bytes(g) || !aligned16(workspace))
+        return IABN_ERR_WORKSPACE;
+    InfArgs a{x_inout, gamma, beta, running_mean, running_var, eps, (int)act, act_param};
+    const Workspace w = carve(workspace, g);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
+    return from_cuda(inference_twophase(g, a, w, static_cast<cudaStream_t>(stream),
+                                        device_sms(dev)));
 }
 
 extern "C" iabn_status iabn_update_running_stats(int64_t c, int64_t count,

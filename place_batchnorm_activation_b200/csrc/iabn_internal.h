@@ -53,6 +53,17 @@ struct BwdArgs {
     float* dbeta;
 };
 
+struct InfArgs {
+    void* x;
+    const float* gamma;
+    const float* beta;
+    const float* running_mean;
+    const float* running_var;
+    float eps;
+    int act;
+    float act_param;
+};
+
 // Host-side count of kernel launches (diagnostics; see iabn_kernel_launches).
 void count_launches(int n);
 
@@ -63,6 +74,10 @@ cudaError_t forward_twophase(const Geom& g, const FwdArgs& a, const Workspace& w
                              cudaStream_t s, int sms);
 cudaError_t backward_twophase(const Geom& g, const BwdArgs& a, const Workspace& w,
                               cudaStream_t s, int sms);
+// Evaluation mode: coefficients from the running statistics, then the
+// forward's elementwise pass (two launches).
+cudaError_t inference_twophase(const Geom& g, const InfArgs& a, const Workspace& w,
+                               cudaStream_t s, int sms);
 cudaError_t running_update(int64_t C, int64_t count, const float* mean, const float* var,
                            float* rmean, float* rvar, float momentum, cudaStream_t s);
 

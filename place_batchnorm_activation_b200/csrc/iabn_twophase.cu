@@ -548,6 +548,22 @@ k_tp_apply_bwd_vec(const typename Storage<DT>::T* __restrict__ z,
     }
 }
 
+// ------------------------------------------------------------ inference
+
+// Evaluation mode ([BN] Algorithm 2, the inference network): the running
+// averages stand in for the batch statistics.  The coefficients take the
+// training forward's form (mean, gamma*rstd, beta), so the forward's
+// elementwise pass applies them unchanged.
+__global__ void k_eval_coef(int64_t C, const float* __restrict__ gamma,
+                            const float* __restrict__ beta, const float* __restrict__ rmean,
+                            const float* __restrict__ rvar, float eps,
+                            float4* __restrict__ coef) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    const double rstd = 1.0 / sqrt((double)rvar[c] + (double)eps);
+    coef[c] = make_float4(rmean[c], (float)((double)gamma[c] * rstd), beta[c], 0.f);
+}
+
 // ------------------------------------------------------------ running stats
 
 __global__ void k_running_update(int64_t C, float unbias, const float* __restrict__ mean,
@@ -726,6 +742,39 @@ cudaError_t backward_twophase(const Geom& g, const BwdArgs& a, const Workspace& 
     case kF32: return bwd_twophase_dt<kF32>(g, a, w, s, sms);
     case kBF16: return bwd_twophase_dt<kBF16>(g, a, w, s, sms);
     default: return bwd_twophase_dt<kF16>(g, a, w, s, sms);
+    }
+}
+
+template <int DT>
+static cudaError_t inference_dt(const Geom& g, const InfArgs& a, const float4* coef,
+                                cudaStream_t s, int sms) {
+    void* x = a.x;
+    const float p = a.act_param;
+    if (g.layout == kNHWC) {
+        switch (a.act) {
+        case kLeaky: return fwd_apply<DT, kLeaky, kNHWC>(g, x, coef, p, s, sms);
+        case kElu: return fwd_apply<DT, kElu, kNHWC>(g, x, coef, p, s, sms);
+        default: return fwd_apply<DT, kIdent, kNHWC>(g, x, coef, p, s, sms);
+        }
+    }
+    switch (a.act) {
+    case kLeaky: return fwd_apply<DT, kLeaky, kNCHW>(g, x, coef, p, s, sms);
+    case kElu: return fwd_apply<DT, kElu, kNCHW>(g, x, coef, p, s, sms);
+    default: return fwd_apply<DT, kIdent, kNCHW>(g, x, coef, p, s, sms);
+    }
+}
+
+cudaError_t inference_twophase(const Geom& g, const InfArgs& a, const Workspace& w,
+                               cudaStream_t s, int sms) {
+    k_eval_coef<<<(unsigned)((g.C + 255) / 256), 256, 0, s>>>(
+        g.C, a.gamma, a.beta, a.running_mean, a.running_var, a.eps, w.coef);
+    count_launches(1);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    switch (g.dtype) {
+    case kF32: return inference_dt<kF32>(g, a, w.coef, s, sms);
+    case kBF16: return inference_dt<kBF16>(g, a, w.coef, s, sms);
+    default: return inference_dt<kF16>(g, a, w.coef, s, sms);
     }
 }
 

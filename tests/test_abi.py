@@ -51,8 +51,10 @@ def test_workspace_size():
     assert n >= 256 + 256 * 256 * 16 + 256 * 16
     d2 = iabn.make_desc((128, 2048, 7, 7), iabn.IABN_NCHW, iabn.IABN_F16)
     assert iabn.iabn_workspace_size(d2) >= 256 + 128 * 2048 * 16 + 2048 * 16
-    for bad in [(0, 1, 1, 2), (1, 0, 2, 2), (1, 1, 1, 1), (-1, 2, 2, 2)]:
+    for bad in [(0, 1, 1, 2), (1, 0, 2, 2), (-1, 2, 2, 2)]:
         assert iabn.iabn_workspace_size(iabn.make_desc(bad, 0, 0)) == 0
+    # one value per channel is a valid descriptor for inference
+    assert iabn.iabn_workspace_size(iabn.make_desc((1, 1, 1, 1), 0, 0)) > 0
     assert iabn.iabn_workspace_size(iabn.make_desc((2, 2, 2, 2), 2, 0)) == 0
     assert iabn.iabn_workspace_size(iabn.make_desc((2, 2, 2, 2), 0, 3)) == 0
 
@@ -116,6 +118,32 @@ def test_backward_rejects_bad_arguments():
     assert _bwd(dz=FAKE + 4096 + 8) == E.IABN_ERR_MISALIGNED
     assert _bwd(z=FAKE + 1) == E.IABN_ERR_MISALIGNED
     assert _bwd(ws_bytes=16) == E.IABN_ERR_WORKSPACE
+
+
+def _inf(desc=None, x=FAKE, eps=1e-5, act=0, p=0.01, ws=FAKE + 8192, ws_bytes=None,
+         rm=FAKE, rv=FAKE):
+    desc = desc or iabn.make_desc((2, 4, 3, 3), iabn.IABN_NHWC, iabn.IABN_F16)
+    if ws_bytes is None:
+        ws_bytes = iabn.iabn_workspace_size(desc)
+    return iabn.iabn_inference(desc, x, FAKE, FAKE, rm, rv, eps, act, p, ws, ws_bytes, None)
+
+
+@no_gpu_only
+def test_inference_rejects_bad_arguments():
+    E = iabn
+    assert _inf(desc=iabn.make_desc((0, 4, 1, 1), 0, 0)) == E.IABN_ERR_INVALID_ARG
+    assert _inf(desc=iabn.make_desc((1, 4, 1, 1), 0, 3)) == E.IABN_ERR_INVALID_ARG
+    assert _inf(x=None) == E.IABN_ERR_INVALID_ARG
+    assert _inf(rm=None) == E.IABN_ERR_INVALID_ARG
+    assert _inf(rv=None) == E.IABN_ERR_INVALID_ARG
+    assert _inf(eps=-1.0) == E.IABN_ERR_INVALID_ARG
+    assert _inf(act=E.IABN_ACT_ELU, p=0.0) == E.IABN_ERR_INVALID_ARG
+    assert _inf(x=FAKE + 8) == E.IABN_ERR_MISALIGNED
+    assert _inf(ws=None) == E.IABN_ERR_WORKSPACE
+    assert _inf(ws_bytes=16) == E.IABN_ERR_WORKSPACE
+    # M = 1 passes the host checks (and then finds no device here)
+    assert _inf(desc=iabn.make_desc((1, 4, 1, 1), 0, 0)) == E.IABN_ERR_CUDA
+    assert _inf() == E.IABN_ERR_CUDA
 
 
 @no_gpu_only
