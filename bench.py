@@ -692,6 +692,12 @@ def main():
             "clocks": sampler.summary(),
             "timed_wall_s": round(wall, 4),
         }
+        try:   # host-side description of the launches timed above
+            line["launch_plan"] = {
+                d: layer.iabn.describe_plan(sp.shape, sp.layout, sp.dtype, i)
+                for i, d in enumerate(("forward", "backward"))}
+        except Exception as e:
+            line["launch_plan"] = {"error": f"{type(e).__name__}: {e}"}
         if extra:
             line["workloads"] = extra
         if not args.no_extra and world == 1:
