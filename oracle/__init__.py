@@ -67,6 +67,11 @@ def _load():
                 f = getattr(lib, name)
                 f.argtypes = geom + [pd, pd, pd, pd, pd, d, i32, d, pd, pd, pd]
                 f.restype = i32
+            lib.orc_backward_checkpoint.argtypes = geom + [pd, pd, pd, pd, pd, d, i32, d, pd,
+                                                           pd, pd]
+            lib.orc_backward_checkpoint.restype = i32
+            lib.orc_checkpoint_recompute.argtypes = geom + [pd, pd, pd, i32, d, pd]
+            lib.orc_checkpoint_recompute.restype = i32
             lib.orc_inference.argtypes = geom + [pd, pd, pd, pd, pd, d, i32, d, pd]
             lib.orc_inference.restype = i32
             lib.orc_running_update.argtypes = [i64, i64, pd, pd, d, pd, pd]
@@ -160,6 +165,29 @@ def backward_inplace(shape, layout, z, dz, gamma, beta, var, eps, kind, p, form:
     _check(fn(n, c, h, w, int(layout), _p(z), _p(dz), _p(g), _p(b), _p(v), float(eps),
               int(kind), float(p), _p(dx), _p(dg), _p(db)), f"backward_inplace_{form}")
     return {"dx": dx, "dgamma": dg, "dbeta": db}
+
+
+def backward_checkpoint(shape, layout, xhat, dz, gamma, beta, var, eps, kind, p):
+    """Optimized-checkpointing backward from the stored xhat (and dz)."""
+    n, c, h, w = (int(v) for v in shape)
+    xh, dz, g, b, v = _f64(xhat), _f64(dz), _f64(gamma), _f64(beta), _f64(var)
+    dx = np.empty_like(xh)
+    dg = np.empty(c)
+    db = np.empty(c)
+    _check(_load().orc_backward_checkpoint(n, c, h, w, int(layout), _p(xh), _p(dz), _p(g),
+                                           _p(b), _p(v), float(eps), int(kind), float(p),
+                                           _p(dx), _p(dg), _p(db)), "backward_checkpoint")
+    return {"dx": dx, "dgamma": dg, "dbeta": db}
+
+
+def checkpoint_recompute(shape, layout, xhat, gamma, beta, kind, p):
+    """z = phi(gamma*xhat + beta) from the stored xhat (fp64)."""
+    n, c, h, w = (int(v) for v in shape)
+    xh, g, b = _f64(xhat), _f64(gamma), _f64(beta)
+    z = np.empty_like(xh)
+    _check(_load().orc_checkpoint_recompute(n, c, h, w, int(layout), _p(xh), _p(g), _p(b),
+                                            int(kind), float(p), _p(z)), "checkpoint_recompute")
+    return z
 
 
 def inference(shape, layout, x, gamma, beta, running_mean, running_var, eps, kind, p):

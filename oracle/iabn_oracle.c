@@ -276,6 +276,57 @@ int orc_backward_inplace_2(int64_t n, int64_t c, int64_t h, int64_t w, int layou
     return 0;
 }
 
+/* --------------------------------------------------- checkpointing (xhat) */
+/* [ABN] section 3, "Proposed Checkpointing": the stored buffer is xhat; the
+ * backward reaches y through the scale and shift only and uses the stored
+ * xhat in the BN backward as it stands. */
+
+int orc_backward_checkpoint(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
+                            const double* xhat, const double* dz,
+                            const double* gamma, const double* beta,
+                            const double* var, double eps, int act, double act_param,
+                            double* dx, double* dgamma, double* dbeta) {
+    if (check_geom(n, c, h, w, layout)) return -1;
+    const int64_t HW = h * w;
+    const double M = (double)(n * HW);
+    for (int64_t ch = 0; ch < c; ++ch) {
+        double rstd = 1.0 / sqrt(var[ch] + eps);
+        double s1 = 0.0, s2 = 0.0;
+        for (int64_t i = 0; i < n; ++i)
+            for (int64_t p = 0; p < HW; ++p) {
+                int64_t k = at(layout, c, HW, i, ch, p);
+                double y = gamma[ch] * xhat[k] + beta[ch];           /* scale and shift */
+                double dy = dz[k] * orc_act_deriv_from_y(y, act, act_param);
+                s1 += dy;
+                s2 += dy * xhat[k];
+            }
+        dbeta[ch] = s1;
+        dgamma[ch] = s2;
+        for (int64_t i = 0; i < n; ++i)
+            for (int64_t p = 0; p < HW; ++p) {
+                int64_t k = at(layout, c, HW, i, ch, p);
+                double y = gamma[ch] * xhat[k] + beta[ch];
+                double dy = dz[k] * orc_act_deriv_from_y(y, act, act_param);
+                dx[k] = gamma[ch] * rstd * (dy - s1 / M - xhat[k] * s2 / M);
+            }
+    }
+    return 0;
+}
+
+int orc_checkpoint_recompute(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
+                             const double* xhat, const double* gamma, const double* beta,
+                             int act, double act_param, double* z_out) {
+    if (check_geom(n, c, h, w, layout)) return -1;
+    const int64_t HW = h * w;
+    for (int64_t ch = 0; ch < c; ++ch)
+        for (int64_t i = 0; i < n; ++i)
+            for (int64_t p = 0; p < HW; ++p) {
+                int64_t k = at(layout, c, HW, i, ch, p);
+                z_out[k] = orc_act(gamma[ch] * xhat[k] + beta[ch], act, act_param);
+            }
+    return 0;
+}
+
 /* ----------------------------------------------------- running statistics */
 /* ------------------------------------------------------------ inference */
 /* [BN] Algorithm 2 (the inference network): the batch statistics are

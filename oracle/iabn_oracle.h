@@ -100,6 +100,27 @@ int orc_backward_inplace_2(int64_t n, int64_t c, int64_t h, int64_t w, int layou
                            const double* var, double eps, int act, double act_param,
                            double* dx, double* dgamma, double* dbeta);
 
+/* Optimized checkpointing ([ABN] section 3, "Proposed Checkpointing"): the
+ * layer keeps the normalised xhat (the forward's xhat_out) instead of x.  The
+ * backward recovers y = gamma*xhat + beta by the scale and shift alone,
+ * dy = dz*phi'(y), and runs the BN backward on the stored xhat (nothing is
+ * recomputed from x):
+ *   dbeta = sum dy,  dgamma = sum dy*xhat,
+ *   dx = gamma*rstd*(dy - dbeta/M - xhat*dgamma/M),  rstd from the saved
+ *   (biased) variance. */
+int orc_backward_checkpoint(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
+                            const double* xhat, const double* dz,
+                            const double* gamma, const double* beta,
+                            const double* var, double eps, int act, double act_param,
+                            double* dx, double* dgamma, double* dbeta);
+
+/* The activation output the layer after it needs, recovered from the stored
+ * xhat ([ABN] "Proposed Checkpointing": scale and shift, then the
+ * activation):  z = phi(gamma*xhat + beta). */
+int orc_checkpoint_recompute(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
+                             const double* xhat, const double* gamma, const double* beta,
+                             int act, double act_param, double* z_out);
+
 /* Inference (evaluation mode): the layer with fixed statistics in place of
  * the batch's ([BN] Algorithm 2, the inference network: normalise with the
  * population mean and variance the running averages estimate; [ABN] section

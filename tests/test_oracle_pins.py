@@ -299,6 +299,72 @@ def test_inplace_backward_equals_standard(layout, act, p):
         _close(ip["dbeta"], std["dbeta"], rel=1e-9, abs_=1e-10)
 
 
+def _torch_xhat_var(xl, eps):
+    """xhat = (x - mean)/sqrt(var + eps) and the biased variance, from PyTorch."""
+    x = torch.tensor(xl, dtype=torch.float64)
+    var, mean = torch.var_mean(x, dim=(0, 2, 3), unbiased=False)
+    xh = (x - mean[None, :, None, None]) / torch.sqrt(var + eps)[None, :, None, None]
+    return xh.numpy(), var.numpy()
+
+
+@pytest.mark.parametrize("layout", [oracle.NCHW, oracle.NHWC])
+@pytest.mark.parametrize("act,p", ACTS + [(oracle.LEAKY_RELU, 0.2)])
+def test_checkpoint_backward_matches_torch_autograd(layout, act, p):
+    """Optimized checkpointing: the backward from the stored xhat (here taken
+    from PyTorch, not from the oracle's forward) gives PyTorch's autograd
+    gradients of BN + activation with respect to x, gamma and beta."""
+    rng = np.random.default_rng(60 + layout)
+    shape = (3, 4, 5, 3)
+    xl, g, b, dzl = _rand_layer(rng, shape, layout, gamma_lo=0.05)
+    ref = _torch_reference(xl, g, b, dzl, 1e-5, act, p)
+    xh, var = _torch_xhat_var(xl, 1e-5)
+    out = oracle.backward_checkpoint(shape, layout, _flat(xh, layout), _flat(dzl, layout), g, b,
+                                     var, 1e-5, act, p)
+    scale = np.abs(ref["dx"]).max()
+    _close(out["dx"], _flat(ref["dx"], layout), rel=1e-10, abs_=1e-12 * scale)
+    _close(out["dgamma"], ref["dgamma"], rel=1e-10, abs_=1e-12)
+    _close(out["dbeta"], ref["dbeta"], rel=1e-10, abs_=1e-12)
+    z = oracle.checkpoint_recompute(shape, layout, _flat(xh, layout), g, b, act, p)
+    _close(z, _flat(ref["z"], layout), rel=1e-12, abs_=1e-14)
+
+
+@pytest.mark.parametrize("layout", [oracle.NCHW, oracle.NHWC])
+@pytest.mark.parametrize("act,p", ACTS + [(oracle.ELU, 0.5)])
+def test_checkpoint_backward_equals_standard(layout, act, p):
+    """From the unrounded xhat, the checkpointing backward equals the standard
+    backward from x, and the recomputed z is the forward's z bit for bit
+    (same scale, shift and activation in the same precision)."""
+    rng = np.random.default_rng(70 + layout)
+    shape = (5, 7, 3, 4)
+    xl, g, b, dzl = _rand_layer(rng, shape, layout, gamma_lo=0.05)
+    x, dz = _flat(xl, layout), _flat(dzl, layout)
+    fw = oracle.forward(shape, layout, x, g, b, 1e-5, act, p, want_xhat_y=True)
+    std = oracle.backward_standard(shape, layout, x, dz, g, b, 1e-5, act, p)
+    ck = oracle.backward_checkpoint(shape, layout, fw["xhat"], dz, g, b, fw["var"], 1e-5, act, p)
+    scale = np.abs(std["dx"]).max()
+    _close(ck["dx"], std["dx"], rel=1e-10, abs_=1e-11 * scale)
+    _close(ck["dgamma"], std["dgamma"], rel=1e-10, abs_=1e-11)
+    _close(ck["dbeta"], std["dbeta"], rel=1e-10, abs_=1e-11)
+    z = oracle.checkpoint_recompute(shape, layout, fw["xhat"], g, b, act, p)
+    np.testing.assert_array_equal(z, fw["z"])
+
+
+def test_checkpoint_backward_needs_no_invertible_gamma():
+    """The stored xhat carries what gamma = 0 would erase: the checkpointing
+    backward stays finite there and matches PyTorch (dx = 0 for the channel)."""
+    rng = np.random.default_rng(80)
+    shape = (2, 3, 3, 2)
+    xl, g, b, dzl = _rand_layer(rng, shape, oracle.NCHW)
+    g[1] = 0.0
+    ref = _torch_reference(xl, g, b, dzl, 1e-5, oracle.LEAKY_RELU, 0.01)
+    xh, var = _torch_xhat_var(xl, 1e-5)
+    out = oracle.backward_checkpoint(shape, 0, _flat(xh, 0), _flat(dzl, 0), g, b, var, 1e-5,
+                                     oracle.LEAKY_RELU, 0.01)
+    assert np.isfinite(out["dx"]).all() and np.isfinite(out["dgamma"]).all()
+    assert np.all(out["dx"].reshape(shape)[:, 1] == 0.0)
+    _close(out["dgamma"], ref["dgamma"], rel=1e-10, abs_=1e-12)
+
+
 def test_bn_backward_invariants():
     """Per channel: sum dx = 0, and sum dx*xhat = gamma*rstd*dgamma*eps/(var+eps)
     (zero for eps = 0: the gradient is orthogonal to the directions that
@@ -422,10 +488,14 @@ def test_hand_derived_examples():
             _close(fw[k], e[k], rel=1e-14, abs_=1e-15)
         std = oracle.backward_standard(shape, lay, case["x"], case["dz"], case["gamma"],
                                        case["beta"], eps, act, p)
+        fwx = oracle.forward(shape, lay, case["x"], case["gamma"], case["beta"], eps, act, p,
+                             want_xhat_y=True)
+        ck = oracle.backward_checkpoint(shape, lay, fwx["xhat"], case["dz"], case["gamma"],
+                                        case["beta"], fw["var"], eps, act, p)
         for form in (1, 2):
             ip = oracle.backward_inplace(shape, lay, fw["z"], case["dz"], case["gamma"],
                                          case["beta"], fw["var"], eps, act, p, form=form)
-            for res in (std, ip):
+            for res in (std, ip, ck):
                 for k in ("dx", "dgamma", "dbeta"):
                     _close(res[k], e[k], rel=1e-13, abs_=1e-14)
         rm, rv = oracle.running_update(shape[0] * shape[2] * shape[3], fw["mean"], fw["var"],
