@@ -257,6 +257,11 @@ class L2Flush:
         if not self.write_only:
             self.r.sum()
 
+    def read_(self):
+        """The clean-read half alone: reading 2x L2 of other data evicts every
+        line the previous kernel left in L2 (dirty ones are written back)."""
+        self.r.sum()
+
 
 def timed_layer_steps(layer, flush, steps, warmup, dist_barrier=None, sampler=None):
     """Warm-up, then `steps` timed steps; returns per-step event times (ms) of
@@ -349,6 +354,136 @@ def e2e_steps(layer, steps, warmup):
     d2h = (hz.numel() * hz.element_size() + hdx.numel() * hdx.element_size()
            + hg.numel() * 4 + hb.numel() * 4)
     return ms, h2d, d2h
+
+
+def drained_steps(layer, flush, steps, warmup):
+    """The same steps with each call's dirty output drained inside its own
+    events: call, then the clean-read half of the flush (which writes back
+    whatever the call left dirty in L2), minus that read's time on an L2 that
+    holds only clean lines.  Returns (fwd_ms, bwd_ms, read_ms) medians."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    recs = []
+    for i in range(warmup + steps):
+        layer.restore()
+        r = [ev() for _ in range(6)]
+        flush.zero_()
+        r[0].record()
+        flush.read_()
+        r[1].record()
+        flush.zero_()
+        r[2].record()
+        layer.fwd()
+        flush.read_()
+        r[3].record()
+        flush.zero_()
+        r[4].record()
+        layer.bwd()
+        flush.read_()
+        r[5].record()
+        layer.run()
+        if i >= warmup:
+            recs.append(r)
+    torch.cuda.synchronize()
+    rd = statistics.median(r[0].elapsed_time(r[1]) for r in recs)
+    f = statistics.median(r[2].elapsed_time(r[3]) for r in recs) - rd
+    b = statistics.median(r[4].elapsed_time(r[5]) for r in recs) - rd
+    return f, b, rd
+
+
+class LayerVariants(Layer):
+    """One workload's buffers for the three layers the pages compare: the
+    in-place layer (keeps z), the standard BN+ACT layer (keeps x and z) and
+    the optimized-checkpointing layer (keeps xhat)."""
+
+    def __init__(self, sp, seed, device):
+        import torch
+        super().__init__(sp, seed, device)
+        self.z = torch.empty_like(self.x)
+
+    def kw(self):
+        sp = self.sp
+        return dict(shape=sp.shape, layout=sp.layout, eps=sp.eps, act=sp.act,
+                    act_param=sp.act_param)
+
+    def calls(self, variant):
+        """(name, callable) of one step of `variant`, in order."""
+        io = self.iabn
+        if variant == "inplace":
+            return [("fwd", self.fwd), ("bwd", self.bwd)]
+        if variant == "standard":
+            return [("fwd", lambda: io.forward_standard(self.x, self.z, self.gamma, self.beta,
+                                                        self.mean, self.var, self.ws,
+                                                        **self.kw())),
+                    ("bwd", lambda: io.backward_standard(self.x, self.dz, self.gamma, self.beta,
+                                                         self.mean, self.var, self.dgamma,
+                                                         self.dbeta, self.ws, **self.kw()))]
+        kw = self.kw()
+        return [("fwd", lambda: io.forward_checkpoint(self.x, self.z, self.gamma, self.beta,
+                                                      self.mean, self.var, self.ws, **kw)),
+                ("recompute", lambda: io.checkpoint_recompute(
+                    self.x, self.z, self.gamma, self.beta, shape=kw["shape"],
+                    layout=kw["layout"], act=kw["act"], act_param=kw["act_param"])),
+                ("bwd", lambda: io.backward_checkpoint(self.x, self.dz, self.gamma, self.beta,
+                                                       self.var, self.dgamma, self.dbeta,
+                                                       self.ws, **kw))]
+
+
+# bytes each layer reads and writes per step, in units of E*s
+LAYER_TRAFFIC = {"inplace": {"fwd": 2, "bwd": 3}, "standard": {"fwd": 2, "bwd": 3},
+                 "checkpoint": {"fwd": 3, "recompute": 2, "bwd": 3}}
+# activation buffers a layer keeps from its forward to its backward, in units of E*s
+LAYER_KEPT = {"inplace": 1, "standard": 2, "checkpoint": 1}
+
+
+def bench_layer_variants(flush, steps, warmup, device):
+    """The in-place layer against the standard BN+ACT layer and the
+    optimized-checkpointing layer on workloads 1-3 (same protocol: L2
+    flushed before every call, inputs restored before every step)."""
+    import torch
+    import workloads as wl
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    out = {}
+    for wid in (1, 2, 3):
+        sp = wl.spec(wid)
+        L = LayerVariants(sp, sp.seed, device)
+        es = sp.numel * sp.itemsize
+        res = {}
+        for variant in ("inplace", "standard", "checkpoint"):
+            calls = L.calls(variant)
+            times = {name: [] for name, _ in calls}
+            for i in range(warmup + steps):
+                L.restore()
+                for name, fn in calls:
+                    flush.zero_()
+                    a, b = ev(), ev()
+                    a.record()
+                    fn()
+                    b.record()
+                    if i >= warmup:
+                        times[name].append((a, b))
+            torch.cuda.synchronize()
+            us = {k: statistics.median(a.elapsed_time(b) for a, b in v) * 1e3
+                  for k, v in times.items()}
+            total = sum(us.values())
+            nbytes = sum(LAYER_TRAFFIC[variant].values()) * es
+            res[variant] = {**{f"{k}_us": round(v, 2) for k, v in us.items()},
+                            "step_us": round(total, 2),
+                            "compulsory_bytes": nbytes,
+                            "gbs": round(nbytes / (total * 1e-6) / 1e9, 1),
+                            "kept_for_backward_bytes": LAYER_KEPT[variant] * es}
+        std = res["standard"]
+        for variant in ("inplace", "checkpoint"):
+            r = res[variant]
+            r["time_vs_standard_pct"] = round(100.0 * (r["step_us"] / std["step_us"] - 1.0), 2)
+            r["memory_saving_vs_standard_pct"] = round(
+                100.0 * (1.0 - r["kept_for_backward_bytes"] / std["kept_for_backward_bytes"]), 1)
+        out[sp.name] = res
+        del L
+        torch.cuda.empty_cache()
+    out["pages"] = ("InPlace-ABN vs standard BN+ACT on 4x Titan Xp (Pascal): up to 50% training "
+                    "memory saved, 0.8-2% more computation time (whole networks)")
+    return out
 
 
 # -------------------------------------------------------- other workloads
@@ -465,6 +600,32 @@ def bench_inference(flush, steps, warmup, hbm_peak, device):
             "plan": "two launches: per-channel coefficients, then the elementwise pass"}
 
 
+def bench_twophase(flush, steps, warmup, hbm_peak, device):
+    """The fallback plan (three launches per call, for the shapes the
+    resident plan declines) forced on the ResNet-trunk layer, same protocol."""
+    import torch
+    import workloads as wl
+    old = os.environ.get("IABN_FORCE_PLAN")
+    os.environ["IABN_FORCE_PLAN"] = "twophase"
+    try:
+        sp = wl.spec(1)
+        L = Layer(sp, sp.seed, device)
+        f, b, u, launches, _ = timed_layer_steps(L, flush, steps, warmup)
+    finally:
+        if old is None:
+            os.environ.pop("IABN_FORCE_PLAN", None)
+        else:
+            os.environ["IABN_FORCE_PLAN"] = old
+    tf, tb = statistics.median(f), statistics.median(b)
+    gbs = L.bytes / ((tf + tb) * 1e-3) / 1e9
+    del L
+    torch.cuda.empty_cache()
+    return {"fwd_us": round(tf * 1e3, 2), "bwd_us": round(tb * 1e3, 2), "gbs": round(gbs, 1),
+            "frac_measured_hbm": round(gbs / hbm_peak, 4),
+            "launches_per_step": launches / max(1, steps),
+            "plan": "IABN_FORCE_PLAN=twophase"}
+
+
 # ------------------------------------------------------------ CPU (oracle)
 
 def oracle_pass(sp_sample):
@@ -486,26 +647,57 @@ def oracle_pass(sp_sample):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(batch: int):
+def host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def cpu_baseline():
+    """The fp64 C oracle on the bench workload itself (N=64), one
+    fwd+bwd+running update: the -fopenmp build on all host cores (the
+    reported value) and the plain build on one core."""
+    import oracle
     import workloads as wl
-    sp = wl.spec(1).with_(n=batch)
-    t = oracle_pass(sp)
-    gbs = 5 * sp.numel * sp.itemsize / t / 1e9
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"resnet_trunk workload with N={batch} instead of 64 "
-                      f"({sp.numel} elements), one fwd+bwd+running update, "
-                      f"single-threaded fp64 C oracle, {t:.2f} s"}
+    sp = wl.spec(1)
+    cores, model = host_cpu()
+    nbytes = 5 * sp.numel * sp.itemsize
+    oracle.openmp(True)
+    try:
+        t_all = oracle_pass(sp)
+    finally:
+        oracle.openmp(False)
+    t_one = oracle_pass(sp)
+    return {"value": round(nbytes / t_all / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle", "cpu_model": model,
+            "sample": f"the resnet_trunk workload itself (N=64, {sp.numel} elements), one "
+                      f"fwd+bwd+running update of the fp64 C oracle built with -fopenmp, "
+                      f"channel loops over all {cores} host threads: {t_all:.2f} s",
+            "single_thread": {"value": round(nbytes / t_one / 1e9, 4), "unit": "GB/s",
+                              "cores": 1, "seconds": round(t_one, 2)}}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    import oracle
     import workloads as wl
-    sp = wl.spec(1).with_(n=1)
+    sp = wl.spec(1).with_(n=8)
+    cores, model = host_cpu()
+    oracle.openmp(True)
     for _ in range(args.warmup):
         oracle_pass(sp)
     times = [oracle_pass(sp) for _ in range(args.steps)]
+    oracle.openmp(False)
     t = statistics.mean(times)
     gbs = 5 * sp.numel * sp.itemsize / t / 1e9
     line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
@@ -513,12 +705,13 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": "resnet_trunk NHWC bf16 N=64 C=256 H=W=56 leaky_relu 0.01, "
-                                   "fwd+bwd+running stats; each step a bounded sample N=1",
+                                   "fwd+bwd+running stats; each step a bounded sample N=8",
                        "sample_elements": sp.numel},
-            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
-                             "kind": "oracle",
-                             "sample": f"N=1 slice of the resnet_trunk workload "
-                                       f"({sp.numel} elements) per step"},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "cpu_model": model,
+                             "sample": f"N=8 slice of the resnet_trunk workload "
+                                       f"({sp.numel} elements) per step, fp64 C oracle built "
+                                       f"with -fopenmp on all {cores} host threads"},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -634,6 +827,9 @@ def main():
     t_max = reduce_max(mean_ms, world, device)
     value = whole_job_gbs(layer.bytes, world, t_max)
     fwd_us, bwd_us = statistics.mean(f) * 1e3, statistics.mean(b) * 1e3
+    # the same steps with each call's dirty output written back inside its events
+    df, db, drd = drained_steps(layer, flush, max(5, args.steps // 5), 2)
+    d_ms = reduce_max(df + db + statistics.mean(u), world, device)
 
     # e2e through host buffers
     e_ms, h2d, d2h = e2e_steps(layer, max(3, args.steps // 10), 2)
@@ -648,6 +844,16 @@ def main():
                                                               hbm_peak, device)
         except Exception as e:  # reported in the line; never fatal for the headline
             extra["inference_resnet_trunk"] = {"error": f"{type(e).__name__}: {e}"}
+        try:
+            extra["twophase_resnet_trunk"] = bench_twophase(flush, max(5, args.steps // 5), 3,
+                                                            hbm_peak, device)
+        except Exception as e:
+            extra["twophase_resnet_trunk"] = {"error": f"{type(e).__name__}: {e}"}
+        try:
+            extra["layers_vs_standard"] = bench_layer_variants(flush, max(5, args.steps // 5), 3,
+                                                               device)
+        except Exception as e:
+            extra["layers_vs_standard"] = {"error": f"{type(e).__name__}: {e}"}
 
     if rank == 0:
         bwd_bytes = 3 * sp.numel * sp.itemsize
@@ -671,6 +877,12 @@ def main():
                        "plan": os.environ.get("IABN_FORCE_PLAN", "auto")},
             "elements_per_s": world * sp.numel / (t_max * 1e-3),
             "value_write_only_flush": round(whole_job_gbs(layer.bytes, world, wf_ms), 1),
+            "value_drained": round(whole_job_gbs(layer.bytes, world, d_ms), 1),
+            "drained": {"fwd_us": round(df * 1e3, 2), "bwd_us": round(db * 1e3, 2),
+                        "flush_read_us": round(drd * 1e3, 2),
+                        "how": "each call followed, inside its events, by a read of 2x L2 of "
+                               "other data (which writes back what the call left dirty), "
+                               "minus that read's time on an L2 holding only clean lines"},
             "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
             "running_update_us": round(statistics.mean(u) * 1e3, 2),
             "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
@@ -701,7 +913,7 @@ def main():
         if extra:
             line["workloads"] = extra
         if not args.no_extra and world == 1:
-            line["cpu_baseline"] = cpu_baseline(32)
+            line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -24,8 +24,10 @@
  *
  * Conventions for every call
  *   - Every pointer argument except `stream` is a DEVICE pointer to memory
- *     owned by the caller.  The library allocates nothing and keeps no state
- *     between calls other than per-device launch settings.
+ *     owned by the caller.  No call allocates memory.  Between calls the
+ *     library keeps only per-device launch settings, and one 8 MiB array of
+ *     device memory on every GPU that loads it: the scratch of
+ *     iabn_forward_static_ws, held until the process exits.
  *   - All calls are asynchronous and ordered on `stream` (a cudaStream_t;
  *     NULL means the legacy default stream), except iabn_get_device_status.
  *   - Arguments are checked on the host before anything is launched; a
@@ -85,7 +87,7 @@ typedef struct {
     int32_t dtype;
 } iabn_desc;
 
-/* Bytes of workspace the forward, backward and inference calls need for
+/* Bytes of workspace the forward and backward calls of every layer need for
  * descriptor `d` (a multiple of 256).  Returns 0 if the descriptor is
  * invalid; M = 1 is valid here (iabn_inference takes it, the training calls
  * do not).  Host-only. */
@@ -132,6 +134,87 @@ iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz_inout,
                           float* dgamma, float* dbeta,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The standard BN+ACT layer ([ABN] section 3, "Standard and Checkpointed
+ * Computation"): it keeps both its input x (for the BN backward) and its
+ * output z (for the activation's and the next layer's backward) -- the
+ * layer InPlace-ABN is measured against.  Same statistics, arithmetic and
+ * rounding as iabn_forward / iabn_backward; only what is stored differs.
+ * ------------------------------------------------------------------------ */
+
+/* Standard forward: as iabn_forward, but x is only read and z is written to
+ * its own buffer.
+ * x      [N,C,H,W] input, not modified.
+ * z_out  [N,C,H,W] output; must not overlap x (IABN_ERR_INVALID_ARG) and
+ *        must start on a 16-byte boundary (IABN_ERR_MISALIGNED).
+ * Other arguments, errors and the workspace as for iabn_forward. */
+iabn_status iabn_forward_standard(const iabn_desc* d, const void* x, void* z_out,
+                                  const float* gamma, const float* beta, float eps,
+                                  int32_t act, float act_param,
+                                  float* save_mean, float* save_var,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Standard backward from the stored input x ([BN] backward; [ABN]
+ * "Standard and Checkpointed Computation"):
+ *   rstd = 1/sqrt(save_var_c + eps),  xhat = (x - save_mean_c)*rstd,
+ *   y = gamma_c*xhat + beta_c,  dy = dz*phi'(y),
+ *   dbeta_c = sum dy,  dgamma_c = sum dy*xhat,
+ *   dx = gamma_c*rstd*(dy - dbeta_c/M - xhat*dgamma_c/M), written over dz.
+ * x         [N,C,H,W]: the forward's input (not modified).
+ * dz_inout  [N,C,H,W]: dL/dz on entry, dL/dx on return; must not overlap x.
+ * save_mean, save_var [C]: as returned by the forward.
+ * gamma may be zero here (nothing is divided by it).  Other arguments and
+ * errors as for iabn_backward. */
+iabn_status iabn_backward_standard(const iabn_desc* d, const void* x, void* dz_inout,
+                                   const float* gamma, const float* beta,
+                                   const float* save_mean, const float* save_var, float eps,
+                                   int32_t act, float act_param,
+                                   float* dgamma, float* dbeta,
+                                   void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * The optimized-checkpointing layer ([ABN] section 3, "Proposed
+ * Checkpointing"): it keeps the normalised xhat in place of x; the backward
+ * reaches y by the scale and shift alone and uses xhat in the BN backward as
+ * it stands; z, which the next layer's backward needs, is recomputed from
+ * xhat (iabn_checkpoint_recompute).
+ * ------------------------------------------------------------------------ */
+
+/* Checkpointing forward: the statistics of iabn_forward, then
+ *   xhat = (x - mean_c)*rstd, written over x (storage type, one rounding),
+ *   z = phi(gamma_c*xhat + beta_c), written to z_out.
+ * x_inout [N,C,H,W]: x on entry, xhat on return.
+ * z_out   [N,C,H,W]: must not overlap x_inout; 16-byte aligned.
+ * Other arguments, errors and the workspace as for iabn_forward. */
+iabn_status iabn_forward_checkpoint(const iabn_desc* d, void* x_inout, void* z_out,
+                                    const float* gamma, const float* beta, float eps,
+                                    int32_t act, float act_param,
+                                    float* save_mean, float* save_var,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* z = phi(gamma_c*xhat + beta_c) from the stored xhat, for the layer that
+ * follows (one elementwise pass; no statistics, no workspace).  M >= 1.
+ * xhat    [N,C,H,W]: not modified unless z_out is the same buffer.
+ * z_out   [N,C,H,W]: xhat itself or a buffer that does not overlap it. */
+iabn_status iabn_checkpoint_recompute(const iabn_desc* d, const void* xhat, void* z_out,
+                                      const float* gamma, const float* beta,
+                                      int32_t act, float act_param, void* stream);
+
+/* Checkpointing backward from the stored xhat:
+ *   y = gamma_c*xhat + beta_c,  dy = dz*phi'(y),
+ *   dbeta_c = sum dy,  dgamma_c = sum dy*xhat,
+ *   dx = gamma_c*rstd*(dy - dbeta_c/M - xhat*dgamma_c/M), written over dz,
+ *   rstd = 1/sqrt(save_var_c + eps).
+ * xhat      [N,C,H,W]: as the checkpointing forward left it (not modified).
+ * dz_inout  [N,C,H,W]: dL/dz on entry, dL/dx on return; must not overlap xhat.
+ * gamma may be zero.  Other arguments and errors as for iabn_backward. */
+iabn_status iabn_backward_checkpoint(const iabn_desc* d, const void* xhat, void* dz_inout,
+                                     const float* gamma, const float* beta,
+                                     const float* save_var, float eps,
+                                     int32_t act, float act_param,
+                                     float* dgamma, float* dbeta,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
 /* Inference, i.e. evaluation mode ([BN] Algorithm 2, the inference network;
  * [ABN] section 3, "Batch Normalization Review" for the scale and shift):
  *   xhat = (x - running_mean_c) / sqrt(running_var_c + eps),
@@ -141,10 +224,9 @@ iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz_inout,
  * gamma, beta, running_mean, running_var [C] float32; running_var_c + eps
  *           must be > 0.
  * eps >= 0; act, act_param as for iabn_forward.
- * workspace, ws_bytes: scratch of at least iabn_workspace_size(d) bytes (its
- *           coefficient area is written); it need not be zero-filled.
- * Launches two kernels: the per-channel coefficients, then the forward's
- * elementwise pass.  Arguments are checked as for iabn_forward. */
+ * workspace, ws_bytes: checked as for iabn_forward but not used (the pass
+ *           forms its coefficients itself).
+ * One kernel launch.  Arguments are checked as for iabn_forward. */
 iabn_status iabn_inference(const iabn_desc* d, void* x_inout,
                            const float* gamma, const float* beta,
                            const float* running_mean, const float* running_var, float eps,
@@ -175,6 +257,16 @@ iabn_status iabn_get_device_status(void* workspace, void* stream);
  * process so far (all devices, all threads).  Host-only; never fails. */
 uint64_t iabn_kernel_launches(void);
 
+/* The calls iabn_describe_plan describes. */
+typedef enum {
+    IABN_CALL_FORWARD = 0,              /* iabn_forward */
+    IABN_CALL_BACKWARD = 1,             /* iabn_backward */
+    IABN_CALL_FORWARD_STANDARD = 2,     /* iabn_forward_standard */
+    IABN_CALL_BACKWARD_STANDARD = 3,    /* iabn_backward_standard */
+    IABN_CALL_FORWARD_CHECKPOINT = 4,   /* iabn_forward_checkpoint */
+    IABN_CALL_BACKWARD_CHECKPOINT = 5   /* iabn_backward_checkpoint */
+} iabn_call;
+
 /* Launch plans (see iabn_describe_plan). */
 typedef enum {
     IABN_PLAN_TWOPHASE = 0,   /* statistics, finalize, apply: three plain launches */
@@ -201,19 +293,19 @@ typedef struct {
     int32_t stash_copy_engine;  /* 1: tcgen05.cp fills that stash from shared memory */
 } iabn_plan_info;
 
-/* Which plan iabn_forward (direction 0) or iabn_backward (direction 1)
- * takes for descriptor d, and its launch shape, as decided on the host; the
- * same environment settings apply (IABN_FORCE_PLAN=twophase, tile and ring
- * sizes).  A resident launch the driver refuses at run time (e.g. too few
+/* Which plan the training call `call` (an iabn_call value) takes for
+ * descriptor d, and its launch shape, as decided on the host; the same
+ * environment settings apply (IABN_FORCE_PLAN=twophase, tile and ring
+ * sizes).  A layer's two calls take the same plan.  A resident launch the driver refuses at run time (e.g. too few
  * co-resident CTAs) still falls back to the two-phase plan; that is not
  * predicted here.
  * sm_count, smem_optin: the device's SM count and opt-in shared memory per
  * block in bytes (B200: 148 and 232448); both 0 = query the current device
  * (IABN_ERR_CUDA if there is none).  With both given no CUDA call is made.
  * Returns the descriptor errors of iabn_forward, IABN_ERR_INVALID_ARG for a
- * null `out`, a direction other than 0/1 or a negative or half-given limit
- * pair, else IABN_OK with *out filled. */
-iabn_status iabn_describe_plan(const iabn_desc* d, int32_t direction, int32_t sm_count,
+ * null `out`, an unknown call or a negative or half-given limit pair, else
+ * IABN_OK with *out filled. */
+iabn_status iabn_describe_plan(const iabn_desc* d, int32_t call, int32_t sm_count,
                                int32_t smem_optin, iabn_plan_info* out);
 
 /* iabn_forward without a caller-supplied workspace.  The paper has no
@@ -228,7 +320,10 @@ iabn_status iabn_describe_plan(const iabn_desc* d, int32_t direction, int32_t sm
  *     rejected with IABN_ERR_WORKSPACE before anything is launched; other
  *     argument errors are reported as by iabn_forward.
  *   - The first call on a device (that device current) looks up the array's
- *     device address; make that first call before any stream capture.
+ *     device address and keeps it for the life of the process; make that
+ *     first call before any stream capture.  A cudaDeviceReset of the device
+ *     discards the array: do not call this entry point on that device after
+ *     one.
  *   - All calls on a device share the one array: calls that overlap on the
  *     GPU (other streams, other host threads) race and give wrong results.
  *     Each call zeroes the array's control block on `stream` before its

@@ -21,33 +21,45 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "iabn_oracle.c")
 _HDR = os.path.join(_HERE, "iabn_oracle.h")
 _LIB = os.path.join(_HERE, "libiabn_oracle.so")
+# the same source built with -fopenmp: its channel loops run on all host cores
+# (identical results; used only for the multi-core CPU baseline)
+_LIB_OMP = os.path.join(_HERE, "libiabn_oracle_omp.so")
 
 NCHW, NHWC = 0, 1
 F32, BF16, F16 = 0, 1, 2
 LEAKY_RELU, ELU, IDENTITY = 0, 1, 2
 
 _lock = threading.Lock()
-_lib = None
+_libs = {}
+_use_omp = False
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle into ``libiabn_oracle.so`` (gcc, -O2, strict IEEE)."""
-    stale = (not os.path.exists(_LIB)) or any(
-        os.path.getmtime(p) > os.path.getmtime(_LIB) for p in (_SRC, _HDR))
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile the oracle into ``libiabn_oracle.so`` (gcc, -O2, strict IEEE),
+    or with ``openmp`` into ``libiabn_oracle_omp.so`` (also -fopenmp)."""
+    lib = _LIB_OMP if openmp else _LIB
+    stale = (not os.path.exists(lib)) or any(
+        os.path.getmtime(p) > os.path.getmtime(lib) for p in (_SRC, _HDR))
     if force or stale:
-        tmp = _LIB + f".tmp{os.getpid()}"
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-               "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+               "-fno-fast-math", *(["-fopenmp"] if openmp else []), "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, _LIB)
-    return _LIB
+        os.replace(tmp, lib)
+    return lib
+
+
+def openmp(enabled: bool) -> None:
+    """Route the calls below to the -fopenmp build (True) or the plain one."""
+    global _use_omp
+    _use_omp = bool(enabled)
 
 
 def _load():
-    global _lib
     with _lock:
-        if _lib is None:
-            lib = ctypes.CDLL(build())
+        key = _use_omp
+        if key not in _libs:
+            lib = ctypes.CDLL(build(openmp=key))
             d, i64, i32 = ctypes.c_double, ctypes.c_int64, ctypes.c_int
             pd = ctypes.POINTER(ctypes.c_double)
             for name in ("orc_act", "orc_act_inv", "orc_act_deriv_from_y"):
@@ -76,8 +88,8 @@ def _load():
             lib.orc_inference.restype = i32
             lib.orc_running_update.argtypes = [i64, i64, pd, pd, d, pd, pd]
             lib.orc_running_update.restype = i32
-            _lib = lib
-    return _lib
+            _libs[key] = lib
+        return _libs[key]
 
 
 def _f64(a) -> np.ndarray:

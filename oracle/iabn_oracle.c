@@ -13,6 +13,16 @@
 #include <math.h>
 #include <stdlib.h>
 
+/* Built with -fopenmp (the benchmark's multi-core CPU baseline), the loops
+ * over channels (and over the elements of orc_round) are split across the
+ * host's cores.  Every iteration writes only its own channel's outputs, in
+ * the same order, so both builds give identical bits. */
+#ifdef _OPENMP
+#define ORC_PARALLEL_FOR _Pragma("omp parallel for schedule(static)")
+#else
+#define ORC_PARALLEL_FOR
+#endif
+
 /* ---------------------------------------------------------------- layout */
 
 static int64_t at(int layout, int64_t C, int64_t HW, int64_t n, int64_t c, int64_t p) {
@@ -107,6 +117,7 @@ int orc_round(const double* in, double* out, int64_t count, int dtype) {
     case ORC_F16:  prec = 11; emin = -14;  emax = 15;  break;
     default: return -1;
     }
+    ORC_PARALLEL_FOR
     for (int64_t i = 0; i < count; ++i) out[i] = round_format(in[i], prec, emin, emax);
     return 0;
 }
@@ -139,6 +150,7 @@ int orc_forward(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
                 double* xhat_out, double* y_out, double* z_out) {
     if (check_geom(n, c, h, w, layout)) return -1;
     const int64_t HW = h * w;
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch) {
         double mu, var;
         channel_stats(n, c, HW, layout, x, ch, &mu, &var);
@@ -168,6 +180,7 @@ int orc_backward_standard(int64_t n, int64_t c, int64_t h, int64_t w, int layout
     if (check_geom(n, c, h, w, layout)) return -1;
     const int64_t HW = h * w;
     const double M = (double)(n * HW);
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch) {
         double mu, var;
         channel_stats(n, c, HW, layout, x, ch, &mu, &var);
@@ -204,6 +217,7 @@ int orc_backward_inplace_1(int64_t n, int64_t c, int64_t h, int64_t w, int layou
     if (check_geom(n, c, h, w, layout)) return -1;
     const int64_t HW = h * w;
     const double M = (double)(n * HW);
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch) {
         double rstd = 1.0 / sqrt(var[ch] + eps);
         double s1 = 0.0, s2 = 0.0;
@@ -244,6 +258,7 @@ int orc_backward_inplace_2(int64_t n, int64_t c, int64_t h, int64_t w, int layou
     if (check_geom(n, c, h, w, layout)) return -1;
     const int64_t HW = h * w;
     const double M = (double)(n * HW);
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch) {
         double rstd = 1.0 / sqrt(var[ch] + eps);
         double s1 = 0.0, sy = 0.0;
@@ -289,6 +304,7 @@ int orc_backward_checkpoint(int64_t n, int64_t c, int64_t h, int64_t w, int layo
     if (check_geom(n, c, h, w, layout)) return -1;
     const int64_t HW = h * w;
     const double M = (double)(n * HW);
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch) {
         double rstd = 1.0 / sqrt(var[ch] + eps);
         double s1 = 0.0, s2 = 0.0;
@@ -318,6 +334,7 @@ int orc_checkpoint_recompute(int64_t n, int64_t c, int64_t h, int64_t w, int lay
                              int act, double act_param, double* z_out) {
     if (check_geom(n, c, h, w, layout)) return -1;
     const int64_t HW = h * w;
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch)
         for (int64_t i = 0; i < n; ++i)
             for (int64_t p = 0; p < HW; ++p) {
@@ -339,6 +356,7 @@ int orc_inference(int64_t n, int64_t c, int64_t h, int64_t w, int layout,
                   double eps, int act, double act_param, double* z_out) {
     if (check_geom(n, c, h, w, layout)) return -1;
     const int64_t HW = h * w;
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch) {
         double rstd = 1.0 / sqrt(running_var[ch] + eps);
         for (int64_t i = 0; i < n; ++i)
@@ -358,6 +376,7 @@ int orc_running_update(int64_t c, int64_t count, const double* mean, const doubl
                        double momentum, double* running_mean, double* running_var) {
     if (c <= 0 || count < 2) return -1;
     const double unbias = (double)count / (double)(count - 1);
+    ORC_PARALLEL_FOR
     for (int64_t ch = 0; ch < c; ++ch) {
         running_mean[ch] = (1.0 - momentum) * running_mean[ch] + momentum * mean[ch];
         running_var[ch] = (1.0 - momentum) * running_var[ch] + momentum * var[ch] * unbias;

@@ -6,13 +6,17 @@ memory and streams.  There is no CPU fallback: if the library is missing or
 no GPU is present, calls raise.
 
 Two levels:
-  * ``iabn_forward``, ``iabn_backward``, ``iabn_inference``,
-    ``iabn_update_running_stats``, ``iabn_workspace_size``,
+  * ``iabn_forward``, ``iabn_backward``, ``iabn_forward_standard``,
+    ``iabn_backward_standard``, ``iabn_forward_checkpoint``,
+    ``iabn_backward_checkpoint``, ``iabn_checkpoint_recompute``,
+    ``iabn_inference``, ``iabn_update_running_stats``, ``iabn_workspace_size``,
     ``iabn_get_device_status``: the C entry points with the same names and
     arguments (raw device pointers as ints).
-  * ``forward``, ``backward``, ``inference``, ``update_running_stats``, ``workspace_size``,
+  * ``forward``, ``backward``, ``forward_standard``, ``backward_standard``,
+    ``forward_checkpoint``, ``backward_checkpoint``, ``checkpoint_recompute``,
+    ``inference``, ``update_running_stats``, ``workspace_size``,
     ``get_device_status``: the same calls taking torch tensors;
-    ``describe_plan``: the launch plan of a descriptor, as a dict.
+    ``describe_plan``: the launch plan of a call on a descriptor, as a dict.
 """
 from __future__ import annotations
 
@@ -43,7 +47,13 @@ IABN_ACT_LEAKY_RELU, IABN_ACT_ELU, IABN_ACT_IDENTITY = 0, 1, 2
 # Symbols include/iabn.h declares (checked by the tests).
 EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_backward",
            "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches",
-           "iabn_forward_static_ws", "iabn_describe_plan", "iabn_inference")
+           "iabn_forward_static_ws", "iabn_describe_plan", "iabn_inference",
+           "iabn_forward_standard", "iabn_backward_standard", "iabn_forward_checkpoint",
+           "iabn_backward_checkpoint", "iabn_checkpoint_recompute")
+
+# iabn_call values (iabn_describe_plan)
+(IABN_CALL_FORWARD, IABN_CALL_BACKWARD, IABN_CALL_FORWARD_STANDARD, IABN_CALL_BACKWARD_STANDARD,
+ IABN_CALL_FORWARD_CHECKPOINT, IABN_CALL_BACKWARD_CHECKPOINT) = range(6)
 
 IABN_PLAN_TWOPHASE, IABN_PLAN_RESIDENT = 0, 1
 PLAN_NAMES = {IABN_PLAN_TWOPHASE: "twophase", IABN_PLAN_RESIDENT: "resident"}
@@ -90,6 +100,20 @@ def lib() -> ctypes.CDLL:
             L.iabn_backward.argtypes = [pd, vp, vp, vp, vp, vp, f32, i32, f32, vp, vp, vp,
                                         ctypes.c_size_t, vp]
             L.iabn_backward.restype = i32
+            L.iabn_forward_standard.argtypes = [pd, vp, vp, vp, vp, f32, i32, f32, vp, vp, vp,
+                                                ctypes.c_size_t, vp]
+            L.iabn_forward_standard.restype = i32
+            L.iabn_forward_checkpoint.argtypes = [pd, vp, vp, vp, vp, f32, i32, f32, vp, vp, vp,
+                                                  ctypes.c_size_t, vp]
+            L.iabn_forward_checkpoint.restype = i32
+            L.iabn_backward_standard.argtypes = [pd, vp, vp, vp, vp, vp, vp, f32, i32, f32, vp,
+                                                 vp, vp, ctypes.c_size_t, vp]
+            L.iabn_backward_standard.restype = i32
+            L.iabn_backward_checkpoint.argtypes = [pd, vp, vp, vp, vp, vp, f32, i32, f32, vp, vp,
+                                                   vp, ctypes.c_size_t, vp]
+            L.iabn_backward_checkpoint.restype = i32
+            L.iabn_checkpoint_recompute.argtypes = [pd, vp, vp, vp, vp, i32, f32, vp]
+            L.iabn_checkpoint_recompute.restype = i32
             L.iabn_inference.argtypes = [pd, vp, vp, vp, vp, vp, f32, i32, f32, vp,
                                          ctypes.c_size_t, vp]
             L.iabn_inference.restype = i32
@@ -131,6 +155,39 @@ def iabn_backward(desc, z, dz_inout, gamma, beta, save_var, eps, act, act_param,
                                    stream))
 
 
+def iabn_forward_standard(desc, x, z_out, gamma, beta, eps, act, act_param, save_mean, save_var,
+                          workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_forward_standard(ctypes.byref(desc), x, z_out, gamma, beta, eps, act,
+                                           act_param, save_mean, save_var, workspace, ws_bytes,
+                                           stream))
+
+
+def iabn_backward_standard(desc, x, dz_inout, gamma, beta, save_mean, save_var, eps, act,
+                           act_param, dgamma, dbeta, workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_backward_standard(ctypes.byref(desc), x, dz_inout, gamma, beta,
+                                            save_mean, save_var, eps, act, act_param, dgamma,
+                                            dbeta, workspace, ws_bytes, stream))
+
+
+def iabn_forward_checkpoint(desc, x_inout, z_out, gamma, beta, eps, act, act_param, save_mean,
+                            save_var, workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_forward_checkpoint(ctypes.byref(desc), x_inout, z_out, gamma, beta,
+                                             eps, act, act_param, save_mean, save_var, workspace,
+                                             ws_bytes, stream))
+
+
+def iabn_backward_checkpoint(desc, xhat, dz_inout, gamma, beta, save_var, eps, act, act_param,
+                             dgamma, dbeta, workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_backward_checkpoint(ctypes.byref(desc), xhat, dz_inout, gamma, beta,
+                                              save_var, eps, act, act_param, dgamma, dbeta,
+                                              workspace, ws_bytes, stream))
+
+
+def iabn_checkpoint_recompute(desc, xhat, z_out, gamma, beta, act, act_param, stream) -> int:
+    return int(lib().iabn_checkpoint_recompute(ctypes.byref(desc), xhat, z_out, gamma, beta,
+                                               act, act_param, stream))
+
+
 def iabn_inference(desc, x_inout, gamma, beta, running_mean, running_var, eps, act, act_param,
                    workspace, ws_bytes, stream) -> int:
     return int(lib().iabn_inference(ctypes.byref(desc), x_inout, gamma, beta, running_mean,
@@ -160,8 +217,8 @@ def iabn_forward_static_ws(desc, x_inout, gamma, beta, eps, act, act_param, save
                                             act_param, save_mean, save_var, stream))
 
 
-def iabn_describe_plan(desc, direction, sm_count, smem_optin, info) -> int:
-    return int(lib().iabn_describe_plan(ctypes.byref(desc), direction, sm_count, smem_optin,
+def iabn_describe_plan(desc, call, sm_count, smem_optin, info) -> int:
+    return int(lib().iabn_describe_plan(ctypes.byref(desc), call, sm_count, smem_optin,
                                         ctypes.byref(info)))
 
 
@@ -200,13 +257,13 @@ def workspace_size(shape, layout: int, dtype: int) -> int:
     return iabn_workspace_size(make_desc(shape, layout, dtype))
 
 
-def describe_plan(shape, layout: int, dtype: int, direction: int, *, sm_count: int = 0,
+def describe_plan(shape, layout: int, dtype: int, call: int, *, sm_count: int = 0,
                   smem_optin: int = 0) -> dict:
-    """The launch plan and shape iabn_forward (direction 0) or iabn_backward
-    (direction 1) takes for this descriptor; sm_count and smem_optin describe
-    the device (both 0: the current device)."""
+    """The launch plan and shape the training call ``call`` (IABN_CALL_*; 0 is
+    iabn_forward, 1 iabn_backward) takes for this descriptor; sm_count and
+    smem_optin describe the device (both 0: the current device)."""
     info = IabnPlanInfo()
-    _ok(iabn_describe_plan(make_desc(shape, layout, dtype), int(direction), int(sm_count),
+    _ok(iabn_describe_plan(make_desc(shape, layout, dtype), int(call), int(sm_count),
                            int(smem_optin), info), "iabn_describe_plan")
     out = {name: int(getattr(info, name)) for name, _ in IabnPlanInfo._fields_}
     out["plan"] = PLAN_NAMES[out["plan"]]
@@ -237,6 +294,60 @@ def backward(z, dz, gamma, beta, save_var, dgamma, dbeta, workspace, *, shape, l
                       float(eps), int(act), float(act_param), _ptr(dgamma), _ptr(dbeta),
                       _ptr(workspace), workspace.numel() * workspace.element_size(),
                       _stream_ptr(stream)), "iabn_backward")
+
+
+def forward_standard(x, z, gamma, beta, save_mean, save_var, workspace, *, shape, layout: int,
+                     eps: float, act: int, act_param: float, stream=None) -> None:
+    """Standard BN+ACT forward: x is kept, z is written to its own buffer."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    _ok(iabn_forward_standard(desc, _ptr(x), _ptr(z), _ptr(gamma), _ptr(beta), float(eps),
+                              int(act), float(act_param), _ptr(save_mean), _ptr(save_var),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream_ptr(stream)), "iabn_forward_standard")
+
+
+def backward_standard(x, dz, gamma, beta, save_mean, save_var, dgamma, dbeta, workspace, *,
+                      shape, layout: int, eps: float, act: int, act_param: float,
+                      stream=None) -> None:
+    """Standard backward from the stored x: dz is overwritten with dx."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    _ok(iabn_backward_standard(desc, _ptr(x), _ptr(dz), _ptr(gamma), _ptr(beta),
+                               _ptr(save_mean), _ptr(save_var), float(eps), int(act),
+                               float(act_param), _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(),
+                               _stream_ptr(stream)), "iabn_backward_standard")
+
+
+def forward_checkpoint(x, z, gamma, beta, save_mean, save_var, workspace, *, shape,
+                       layout: int, eps: float, act: int, act_param: float,
+                       stream=None) -> None:
+    """Checkpointing forward: x is overwritten with xhat, z written to its own buffer."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    _ok(iabn_forward_checkpoint(desc, _ptr(x), _ptr(z), _ptr(gamma), _ptr(beta), float(eps),
+                                int(act), float(act_param), _ptr(save_mean), _ptr(save_var),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream_ptr(stream)), "iabn_forward_checkpoint")
+
+
+def backward_checkpoint(xhat, dz, gamma, beta, save_var, dgamma, dbeta, workspace, *, shape,
+                        layout: int, eps: float, act: int, act_param: float,
+                        stream=None) -> None:
+    """Checkpointing backward from the stored xhat: dz is overwritten with dx."""
+    desc = make_desc(shape, layout, _dtype_code(xhat))
+    _ok(iabn_backward_checkpoint(desc, _ptr(xhat), _ptr(dz), _ptr(gamma), _ptr(beta),
+                                 _ptr(save_var), float(eps), int(act), float(act_param),
+                                 _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(),
+                                 _stream_ptr(stream)), "iabn_backward_checkpoint")
+
+
+def checkpoint_recompute(xhat, z, gamma, beta, *, shape, layout: int, act: int,
+                         act_param: float, stream=None) -> None:
+    """z = phi(gamma*xhat + beta) from the stored xhat."""
+    desc = make_desc(shape, layout, _dtype_code(xhat))
+    _ok(iabn_checkpoint_recompute(desc, _ptr(xhat), _ptr(z), _ptr(gamma), _ptr(beta), int(act),
+                                  float(act_param), _stream_ptr(stream)),
+        "iabn_checkpoint_recompute")
 
 
 def inference(x, gamma, beta, running_mean, running_var, workspace, *, shape, layout: int,

@@ -34,11 +34,18 @@ static size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 static size_t workspace_bytes(const Geom& g) {
     return round_up(sizeof(Control) + kTraceBytes + (size_t)partial_slots(g) * sizeof(double2) +
-                        (size_t)g.C * sizeof(float4),
+                        2 * (size_t)g.C * sizeof(float4),
                     256);
 }
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// True if the two activation tensors of g at a and b share any byte.
+static bool overlap(const Geom& g, const void* a, const void* b) {
+    const uintptr_t n = (uintptr_t)g.E * (uintptr_t)g.esize;
+    const uintptr_t pa = (uintptr_t)a, pb = (uintptr_t)b;
+    return pa < pb + n && pb < pa + n;
+}
 
 // Checks the descriptor; fills g.  Returns IABN_OK or the error.  min_m is
 // the least number of values per channel the call accepts: 2 for the
@@ -144,31 +151,115 @@ extern "C" size_t iabn_workspace_size(const iabn_desc* d) {
     return workspace_bytes(g);
 }
 
-extern "C" iabn_status iabn_forward(const iabn_desc* d, void* x_inout, const float* gamma,
-                                    const float* beta, float eps, int32_t act, float act_param,
-                                    float* save_mean, float* save_var, void* workspace,
-                                    size_t ws_bytes, void* stream) {
-    Geom g;
+// Checks shared by the training forward calls; fills g.  z_out: the separate
+// output of the standard and checkpointing forwards (nullptr for the in-place
+// one, which writes over x).
+static iabn_status check_forward(const iabn_desc* d, Geom& g, const void* x, const void* z_out,
+                                 bool separate_out, const float* gamma, const float* beta,
+                                 float eps, int32_t act, float act_param,
+                                 const float* save_mean, const float* save_var,
+                                 const void* workspace, size_t ws_bytes) {
     iabn_status st = make_geom(d, g);
     if (st != IABN_OK) return st;
-    if (!x_inout || !gamma || !beta || !save_mean || !save_var) return IABN_ERR_INVALID_ARG;
+    if (!x || !gamma || !beta || !save_mean || !save_var) return IABN_ERR_INVALID_ARG;
+    if (separate_out && (!z_out || overlap(g, x, z_out))) return IABN_ERR_INVALID_ARG;
     if (!(eps >= 0.f) || !isfinite(eps)) return IABN_ERR_INVALID_ARG;
     if ((st = check_act(act, act_param)) != IABN_OK) return st;
-    if (!aligned16(x_inout)) return IABN_ERR_MISALIGNED;
+    if (!aligned16(x) || (separate_out && !aligned16(z_out))) return IABN_ERR_MISALIGNED;
     if (!workspace || ws_bytes < workspace_bytes(g) || !aligned16(workspace))
         return IABN_ERR_WORKSPACE;
-    FwdArgs a{x_inout, gamma, beta, eps, (int)act, act_param, save_mean, save_var};
+    return IABN_OK;
+}
+
+// Checks shared by the backward calls; fills g.  src is z, x or xhat.
+static iabn_status check_backward(const iabn_desc* d, Geom& g, const void* src, const void* dz,
+                                  const float* gamma, const float* beta, const float* save_var,
+                                  float eps, int32_t act, float act_param, const float* dgamma,
+                                  const float* dbeta, const void* workspace, size_t ws_bytes,
+                                  bool need_mean = false, const float* save_mean = nullptr) {
+    iabn_status st = make_geom(d, g);
+    if (st != IABN_OK) return st;
+    if (!src || !dz || !gamma || !beta || !save_var || !dgamma || !dbeta)
+        return IABN_ERR_INVALID_ARG;
+    if (need_mean && !save_mean) return IABN_ERR_INVALID_ARG;
+    if (overlap(g, src, dz)) return IABN_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !isfinite(eps)) return IABN_ERR_INVALID_ARG;
+    if ((st = check_act(act, act_param)) != IABN_OK) return st;
+    if (!aligned16(src) || !aligned16(dz)) return IABN_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < workspace_bytes(g) || !aligned16(workspace))
+        return IABN_ERR_WORKSPACE;
+    return IABN_OK;
+}
+
+// The resident plan when both calls of the layer qualify, else (or when the
+// driver declines the launch) the two-phase plan.
+static iabn_status run_forward(const Geom& g, const FwdArgs& a, void* workspace,
+                               cudaStream_t s) {
     const Workspace w = carve(workspace, g);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
     const Plan plan = forced_plan();
-    if (plan != kTwoPhase && resident_supported(g)) {
+    if (plan != kTwoPhase && resident_supported(g, a.layer)) {
         cudaError_t e = forward_resident(g, a, w, s);
         if (e == cudaSuccess || plan == kResident || !resident_declined(e)) return from_cuda(e);
         cudaGetLastError();
     }
     return from_cuda(forward_twophase(g, a, w, s, device_sms(dev)));
+}
+
+static iabn_status run_backward(const Geom& g, const BwdArgs& a, void* workspace,
+                                cudaStream_t s) {
+    const Workspace w = carve(workspace, g);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
+    const Plan plan = forced_plan();
+    if (plan != kTwoPhase && resident_supported(g, a.layer)) {
+        cudaError_t e = backward_resident(g, a, w, s);
+        if (e == cudaSuccess || plan == kResident || !resident_declined(e)) return from_cuda(e);
+        cudaGetLastError();
+    }
+    return from_cuda(backward_twophase(g, a, w, s, device_sms(dev)));
+}
+
+extern "C" iabn_status iabn_forward(const iabn_desc* d, void* x_inout, const float* gamma,
+                                    const float* beta, float eps, int32_t act, float act_param,
+                                    float* save_mean, float* save_var, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+    Geom g;
+    const iabn_status st = check_forward(d, g, x_inout, nullptr, false, gamma, beta, eps, act,
+                                         act_param, save_mean, save_var, workspace, ws_bytes);
+    if (st != IABN_OK) return st;
+    const FwdArgs a{x_inout, x_inout, nullptr, kModeFwd, kLayerInPlace, gamma, beta, eps,
+                    (int)act, act_param, save_mean, save_var};
+    return run_forward(g, a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" iabn_status iabn_forward_standard(const iabn_desc* d, const void* x, void* z_out,
+                                             const float* gamma, const float* beta, float eps,
+                                             int32_t act, float act_param, float* save_mean,
+                                             float* save_var, void* workspace, size_t ws_bytes,
+                                             void* stream) {
+    Geom g;
+    const iabn_status st = check_forward(d, g, x, z_out, true, gamma, beta, eps, act, act_param,
+                                         save_mean, save_var, workspace, ws_bytes);
+    if (st != IABN_OK) return st;
+    const FwdArgs a{x, z_out, nullptr, kModeFwd, kLayerStandard, gamma, beta, eps, (int)act,
+                    act_param, save_mean, save_var};
+    return run_forward(g, a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" iabn_status iabn_forward_checkpoint(const iabn_desc* d, void* x_inout, void* z_out,
+                                               const float* gamma, const float* beta, float eps,
+                                               int32_t act, float act_param, float* save_mean,
+                                               float* save_var, void* workspace,
+                                               size_t ws_bytes, void* stream) {
+    Geom g;
+    const iabn_status st = check_forward(d, g, x_inout, z_out, true, gamma, beta, eps, act,
+                                         act_param, save_mean, save_var, workspace, ws_bytes);
+    if (st != IABN_OK) return st;
+    const FwdArgs a{x_inout, x_inout, z_out, kModeFwdCkpt, kLayerCkpt, gamma, beta, eps,
+                    (int)act, act_param, save_mean, save_var};
+    return run_forward(g, a, workspace, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz_inout,
@@ -177,28 +268,60 @@ extern "C" iabn_status iabn_backward(const iabn_desc* d, const void* z, void* dz
                                      float act_param, float* dgamma, float* dbeta,
                                      void* workspace, size_t ws_bytes, void* stream) {
     Geom g;
-    iabn_status st = make_geom(d, g);
+    const iabn_status st = check_backward(d, g, z, dz_inout, gamma, beta, save_var, eps, act,
+                                          act_param, dgamma, dbeta, workspace, ws_bytes);
     if (st != IABN_OK) return st;
-    if (!z || !dz_inout || !gamma || !beta || !save_var || !dgamma || !dbeta)
-        return IABN_ERR_INVALID_ARG;
-    if (z == dz_inout) return IABN_ERR_INVALID_ARG;
-    if (!(eps >= 0.f) || !isfinite(eps)) return IABN_ERR_INVALID_ARG;
+    const BwdArgs a{z, dz_inout, kModeBwdZ, kLayerInPlace, gamma, beta, nullptr, save_var, eps,
+                    (int)act, act_param, dgamma, dbeta};
+    return run_backward(g, a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" iabn_status iabn_backward_standard(const iabn_desc* d, const void* x, void* dz_inout,
+                                              const float* gamma, const float* beta,
+                                              const float* save_mean, const float* save_var,
+                                              float eps, int32_t act, float act_param,
+                                              float* dgamma, float* dbeta, void* workspace,
+                                              size_t ws_bytes, void* stream) {
+    Geom g;
+    const iabn_status st = check_backward(d, g, x, dz_inout, gamma, beta, save_var, eps, act,
+                                          act_param, dgamma, dbeta, workspace, ws_bytes, true,
+                                          save_mean);
+    if (st != IABN_OK) return st;
+    const BwdArgs a{x, dz_inout, kModeBwdX, kLayerStandard, gamma, beta, save_mean, save_var,
+                    eps, (int)act, act_param, dgamma, dbeta};
+    return run_backward(g, a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" iabn_status iabn_backward_checkpoint(const iabn_desc* d, const void* xhat,
+                                                void* dz_inout, const float* gamma,
+                                                const float* beta, const float* save_var,
+                                                float eps, int32_t act, float act_param,
+                                                float* dgamma, float* dbeta, void* workspace,
+                                                size_t ws_bytes, void* stream) {
+    Geom g;
+    const iabn_status st = check_backward(d, g, xhat, dz_inout, gamma, beta, save_var, eps, act,
+                                          act_param, dgamma, dbeta, workspace, ws_bytes);
+    if (st != IABN_OK) return st;
+    const BwdArgs a{xhat, dz_inout, kModeBwdXhat, kLayerCkpt, gamma, beta, nullptr, save_var,
+                    eps, (int)act, act_param, dgamma, dbeta};
+    return run_backward(g, a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" iabn_status iabn_checkpoint_recompute(const iabn_desc* d, const void* xhat,
+                                                 void* z_out, const float* gamma,
+                                                 const float* beta, int32_t act,
+                                                 float act_param, void* stream) {
+    Geom g;
+    iabn_status st = make_geom(d, g, 1);
+    if (st != IABN_OK) return st;
+    if (!xhat || !z_out || !gamma || !beta) return IABN_ERR_INVALID_ARG;
     if ((st = check_act(act, act_param)) != IABN_OK) return st;
-    if (!aligned16(z) || !aligned16(dz_inout)) return IABN_ERR_MISALIGNED;
-    if (!workspace || ws_bytes < workspace_bytes(g) || !aligned16(workspace))
-        return IABN_ERR_WORKSPACE;
-    BwdArgs a{z, dz_inout, gamma, beta, save_var, eps, (int)act, act_param, dgamma, dbeta};
-    const Workspace w = carve(workspace, g);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!aligned16(xhat) || !aligned16(z_out)) return IABN_ERR_MISALIGNED;
+    if (xhat != z_out && overlap(g, xhat, z_out)) return IABN_ERR_INVALID_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
-    const Plan plan = forced_plan();
-    if (plan != kTwoPhase && resident_supported(g)) {
-        cudaError_t e = backward_resident(g, a, w, s);
-        if (e == cudaSuccess || plan == kResident || !resident_declined(e)) return from_cuda(e);
-        cudaGetLastError();
-    }
-    return from_cuda(backward_twophase(g, a, w, s, device_sms(dev)));
+    return from_cuda(recompute_pass(g, xhat, z_out, gamma, beta, (int)act, act_param,
+                                    static_cast<cudaStream_t>(stream), device_sms(dev)));
 }
 
 extern "C" iabn_status iabn_inference(const iabn_desc* d, void* x_inout, const float* gamma,
@@ -216,11 +339,9 @@ extern "C" iabn_status iabn_inference(const iabn_desc* d, void* x_inout, const f
     if (!workspace || ws_bytes < workspace_bytes(g) || !aligned16(workspace))
         return IABN_ERR_WORKSPACE;
     InfArgs a{x_inout, gamma, beta, running_mean, running_var, eps, (int)act, act_param};
-    const Workspace w = carve(workspace, g);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
-    return from_cuda(inference_twophase(g, a, w, static_cast<cudaStream_t>(stream),
-                                        device_sms(dev)));
+    return from_cuda(inference_pass(g, a, static_cast<cudaStream_t>(stream), device_sms(dev)));
 }
 
 extern "C" iabn_status iabn_update_running_stats(int64_t c, int64_t count,
@@ -255,13 +376,14 @@ extern "C" uint64_t iabn_kernel_launches(void) {
     return g_launches.load(std::memory_order_relaxed);
 }
 
-extern "C" iabn_status iabn_describe_plan(const iabn_desc* d, int32_t direction,
-                                          int32_t sm_count, int32_t smem_optin,
-                                          iabn_plan_info* out) {
+extern "C" iabn_status iabn_describe_plan(const iabn_desc* d, int32_t call, int32_t sm_count,
+                                          int32_t smem_optin, iabn_plan_info* out) {
     Geom g;
     iabn_status st = make_geom(d, g);
     if (st != IABN_OK) return st;
-    if (!out || (direction != 0 && direction != 1)) return IABN_ERR_INVALID_ARG;
+    if (!out || call < IABN_CALL_FORWARD || call > IABN_CALL_BACKWARD_CHECKPOINT)
+        return IABN_ERR_INVALID_ARG;
+    const int layer = call / 2, direction = call % 2;
     if (sm_count < 0 || smem_optin < 0 || (sm_count == 0) != (smem_optin == 0))
         return IABN_ERR_INVALID_ARG;
     if (sm_count == 0) {
@@ -277,7 +399,8 @@ extern "C" iabn_status iabn_describe_plan(const iabn_desc* d, int32_t direction,
     }
     memset(out, 0, sizeof(*out));
     ResidentShape r;
-    if (forced_plan() != kTwoPhase && resident_shape(g, direction, sm_count, smem_optin, r)) {
+    if (forced_plan() != kTwoPhase &&
+        resident_shape(g, layer, direction, sm_count, smem_optin, r)) {
         out->plan = IABN_PLAN_RESIDENT;
         out->launches = 1;
         out->grid = r.grid;

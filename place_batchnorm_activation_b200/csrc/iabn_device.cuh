@@ -19,6 +19,16 @@ enum : int { kNCHW = 0, kNHWC = 1 };
 enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 enum : int { kLeaky = 0, kElu = 1, kIdent = 2 };
 
+// What one call computes.  The in-place layer keeps only z; the standard
+// BN+ACT layer keeps x (and z); the optimized-checkpointing layer keeps xhat.
+//   kModeFwd       read x, write z (over x for the in-place layer, to its
+//                  own buffer for the standard one)
+//   kModeFwdCkpt   read x, write xhat over x and z to its own buffer
+//   kModeBwdZ      read z and dz, write dx over dz (INPLACE-ABN)
+//   kModeBwdX      read x and dz, write dx over dz (standard)
+//   kModeBwdXhat   read xhat and dz, write dx over dz (checkpointing)
+enum : int { kModeFwd = 0, kModeFwdCkpt = 1, kModeBwdZ = 2, kModeBwdX = 3, kModeBwdXhat = 4 };
+
 // Sticky status bits written by kernels into the workspace control block.
 constexpr uint32_t kStTimeout = 1u << 0;
 constexpr uint32_t kStSingular = 1u << 1;
@@ -117,6 +127,46 @@ __device__ __forceinline__ void act_backward(float z, float dz, float p, float i
     }
 }
 
+// dy = dz * phi'(y) from the pre-activation y itself (the standard and the
+// checkpointing layers, which recompute y): 1 on the positive branch, the
+// slope a, or alpha*e^y for the ELU (y <= 0 there).
+template <int ACT, int DT>
+__device__ __forceinline__ float act_dy_from_y(float y, float dz, float p) {
+    if (ACT == kLeaky) return y > 0.f ? dz : dz * p;
+    if (ACT == kElu) {
+        const float e = DT == kF32 ? expf(fminf(y, 0.f)) : __expf(fminf(y, 0.f));
+        return y > 0.f ? dz : dz * (p * e);
+    }
+    return dz;
+}
+
+// Per-channel constants with which the standard and the checkpointing
+// backward recover, from the stored value a (x or xhat),
+//   xhat = a*xs + xb   and   y = a*ys + yb.
+// Standard (from x, with the saved mean and variance): rstd =
+// 1/sqrt(var + eps) and A = gamma*rstd in fp64, then xs = rstd,
+// xb = -mean*rstd, ys = A, yb = beta - mean*A, each rounded once to fp32.
+// Checkpointing (from xhat): xs = 1, xb = 0, ys = gamma, yb = beta.  Every
+// kernel that recomputes y from a takes these same four floats, so its sign
+// (the activation's branch) is decided identically in every pass.
+template <int MODE>
+__device__ __forceinline__ void src_affine(float g, float b, float mean, float var, float eps,
+                                           float& xs, float& xb, float& ys, float& yb) {
+    if (MODE == kModeBwdX) {
+        const double r = 1.0 / sqrt((double)var + (double)eps);
+        const double A = (double)g * r;
+        xs = (float)r;
+        xb = (float)(-(double)mean * r);
+        ys = (float)A;
+        yb = (float)((double)b - (double)mean * A);
+    } else {
+        xs = 1.f;
+        xb = 0.f;
+        ys = g;
+        yb = b;
+    }
+}
+
 // ------------------------------------------------------------ small helpers
 
 __device__ __forceinline__ unsigned long long global_ns() {
@@ -188,6 +238,88 @@ __device__ __forceinline__ bool grid_barrier(Control* ctl, uint32_t target,
 __device__ __forceinline__ void bar_pad(Control* ctl, uint32_t G, uint32_t nbar) {
     atomicAdd(&ctl->bar_count, 2u * kBarStride - nbar * G);
 }
+
+// ------------------------------------------------ channel of a flat index
+
+// The channel of element i of a flat grid-stride loop, tracked incrementally
+// (NHWC: i mod C; NCHW: (i div HW) mod C) so the loop has no division.
+template <int LAYOUT>
+struct ChannelWalker {
+    int64_t c, rem, sc, sr, sq, C, HW;
+    __device__ __forceinline__ void init(int64_t i, int64_t stride, int64_t C_, int64_t HW_) {
+        C = C_; HW = HW_;
+        if (LAYOUT == kNHWC) {
+            c = i % C; sc = stride % C;
+        } else {
+            rem = i % HW; c = (i / HW) % C; sr = stride % HW; sq = (stride / HW) % C;
+        }
+    }
+    __device__ __forceinline__ void advance() {
+        if (LAYOUT == kNHWC) {
+            c += sc;
+            if (c >= C) c -= C;
+        } else {
+            rem += sr;
+            int64_t carry = 0;
+            if (rem >= HW) { rem -= HW; carry = 1; }
+            c += sq + carry;
+            if (c >= C) c -= C;
+        }
+    }
+};
+
+// Channel of a flat element index, moved without division: by one element
+// (step) or by the grid-stride loop's fixed stride (jump).  NHWC: c = i mod C;
+// NCHW: rem = i mod HW, c = (i div HW) mod C.
+struct ChannelPos {
+    int64_t c, rem;
+};
+
+template <int LAYOUT>
+struct ChannelStride {
+    int64_t C, HW, sc, sr, sq;
+    __device__ __forceinline__ void setup(int64_t stride, int64_t C_, int64_t HW_) {
+        C = C_;
+        HW = HW_;
+        sc = stride % C;
+        sr = stride % HW;
+        sq = (stride / HW) % C;
+    }
+    __device__ __forceinline__ ChannelPos at(int64_t i) const {
+        ChannelPos q;
+        if (LAYOUT == kNHWC) {
+            q.c = i % C;
+            q.rem = 0;
+        } else {
+            q.rem = i % HW;
+            q.c = (i / HW) % C;
+        }
+        return q;
+    }
+    __device__ __forceinline__ void jump(ChannelPos& q) const {
+        if (LAYOUT == kNHWC) {
+            q.c += sc;
+            if (q.c >= C) q.c -= C;
+        } else {
+            q.rem += sr;
+            int64_t carry = 0;
+            if (q.rem >= HW) {
+                q.rem -= HW;
+                carry = 1;
+            }
+            q.c += sq + carry;   // < 2C
+            if (q.c >= C) q.c -= C;
+        }
+    }
+    __device__ __forceinline__ void step(ChannelPos& q) const {
+        if (LAYOUT == kNHWC) {
+            if (++q.c == C) q.c = 0;
+        } else if (++q.rem == HW) {
+            q.rem = 0;
+            if (++q.c == C) q.c = 0;
+        }
+    }
+};
 
 // Deterministic warp reductions (fixed shuffle-down tree; lane 0 holds the
 // result, which is then broadcast so every lane sees the same bits).

@@ -21,7 +21,8 @@ struct Geom {
     int esize;       // bytes per stored element
 };
 
-// Workspace carve-up: [Control | trace | partials (double2) | coef (float4)].
+// Workspace carve-up: [Control | trace | partials (double2) | coef (2 float4
+// records per channel)].
 struct Workspace {
     Control* ctl;
     unsigned long long* trace;
@@ -29,8 +30,18 @@ struct Workspace {
     float4* coef;
 };
 
+// Layers: which buffer each keeps for its backward.
+//   kLayerInPlace   z only (INPLACE-ABN): forward kModeFwd over x, backward kModeBwdZ
+//   kLayerStandard  x and z: forward kModeFwd into its own buffer, backward kModeBwdX
+//   kLayerCkpt      xhat: forward kModeFwdCkpt, backward kModeBwdXhat
+enum : int { kLayerInPlace = 0, kLayerStandard = 1, kLayerCkpt = 2 };
+
 struct FwdArgs {
-    void* x;
+    const void* x;
+    void* dst;            // z (kModeFwd) or xhat (kModeFwdCkpt)
+    void* dst2;           // kModeFwdCkpt: z
+    int mode;             // kModeFwd or kModeFwdCkpt
+    int layer;            // kLayer*
     const float* gamma;
     const float* beta;
     float eps;
@@ -41,10 +52,13 @@ struct FwdArgs {
 };
 
 struct BwdArgs {
-    const void* z;
+    const void* src;      // z (kModeBwdZ), x (kModeBwdX) or xhat (kModeBwdXhat)
     void* dz;
+    int mode;
+    int layer;
     const float* gamma;
     const float* beta;
+    const float* save_mean;   // kModeBwdX
     const float* save_var;
     float eps;
     int act;
@@ -74,9 +88,14 @@ cudaError_t forward_twophase(const Geom& g, const FwdArgs& a, const Workspace& w
                              cudaStream_t s, int sms);
 cudaError_t backward_twophase(const Geom& g, const BwdArgs& a, const Workspace& w,
                               cudaStream_t s, int sms);
-// Evaluation mode: coefficients from the running statistics, then the
-// forward's elementwise pass (two launches).
-cudaError_t inference_twophase(const Geom& g, const InfArgs& a, const Workspace& w,
+// One-launch elementwise passes (iabn_elementwise.cu): evaluation mode from
+// the running statistics; the checkpointing layer's z = phi(gamma*xhat +
+// beta); the two-phase forward's apply from its finalize's coefficients.
+cudaError_t inference_pass(const Geom& g, const InfArgs& a, cudaStream_t s, int sms);
+cudaError_t recompute_pass(const Geom& g, const void* xhat, void* z, const float* gamma,
+                           const float* beta, int act, float act_param, cudaStream_t s,
+                           int sms);
+cudaError_t forward_apply_pass(const Geom& g, const FwdArgs& f, const float4* coef,
                                cudaStream_t s, int sms);
 cudaError_t running_update(int64_t C, int64_t count, const float* mean, const float* var,
                            float* rmean, float* rvar, float momentum, cudaStream_t s);
@@ -87,7 +106,8 @@ cudaError_t forward_resident(const Geom& g, const FwdArgs& a, const Workspace& w
                              cudaStream_t s);
 cudaError_t backward_resident(const Geom& g, const BwdArgs& a, const Workspace& w,
                               cudaStream_t s);
-bool resident_supported(const Geom& g);
+// Both calls of the layer qualify for the resident plan on the current device.
+bool resident_supported(const Geom& g, int layer);
 
 // Launch shape of the resident plan in one direction (iabn_describe_plan).
 struct ResidentShape {
@@ -96,10 +116,11 @@ struct ResidentShape {
     int stash_rows, stash_copy_engine;
 };
 
-// True, with `out` filled for direction dir (0 forward, 1 backward), if the
-// calls on g take the resident plan on a device with `sms` SMs and
-// `smem_optin` bytes of opt-in shared memory per block (both directions must
-// qualify, as in resident_supported).  Host only: no CUDA call.
-bool resident_shape(const Geom& g, int dir, int sms, int smem_optin, ResidentShape& out);
+// True, with `out` filled for direction dir (0 forward, 1 backward) of
+// `layer`, if the calls on g take the resident plan on a device with `sms`
+// SMs and `smem_optin` bytes of opt-in shared memory per block (both calls of
+// the layer must qualify, as in resident_supported).  Host only: no CUDA call.
+bool resident_shape(const Geom& g, int layer, int dir, int sms, int smem_optin,
+                    ResidentShape& out);
 
 }  // namespace iabn

@@ -12,7 +12,9 @@
 // that loads this library until the process exits.  Host code may not use
 // the symbol itself as a device address, so the first call on each device
 // (with that device current) looks the address up with cudaGetSymbolAddress
-// and caches it.
+// and caches it for the life of the process (a cudaDeviceReset discards the
+// array, so callers must not use this entry point on that device after one).
+// Every call on a device shares the array: calls that overlap on the GPU race.
 #include <cuda_runtime.h>
 
 #include <mutex>

@@ -13,6 +13,7 @@
 // Tuning knobs read from the environment (defaults in brackets):
 //   IABN_L2_HINTS [1]       L2 evict-last on tiles phase B reloads, evict-first
 //                           on the rest; 0 = no hints.
+//   IABN_STORE_HINT [1]     phase B's stores evict-first in L2 (needs IABN_L2_HINTS).
 //   IABN_TILE_KB_FWD, IABN_TILE_KB_BWD [48, 24] KiB per tensor per tile.
 //   IABN_RING_FWD, IABN_RING_BWD       [4, 4]   slots cycled by the stream.
 //   IABN_BARRIER_BUDGET_NS  [1e9] time budget of each bounded wait.
@@ -77,10 +78,19 @@ int gcd_int(int64_t a, int64_t b) {
 
 int round_up_int(int v, int a) { return (v + a - 1) / a * a; }
 
-// Fills P for direction dir (0 forward, 1 backward); false if the shape does
-// not qualify or the device cannot hold the tiles.
-bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& cpt) {
+int layer_mode(int layer, int dir) {
+    if (layer == kLayerStandard) return dir == 0 ? kModeFwd : kModeBwdX;
+    if (layer == kLayerCkpt) return dir == 0 ? kModeFwdCkpt : kModeBwdXhat;
+    return dir == 0 ? kModeFwd : kModeBwdZ;
+}
+
+// Fills P for call mode `mode`; false if the shape does not qualify or the
+// device cannot hold the tiles.
+bool make_plan(const Geom& g, int mode, const DeviceLimits& dl, ResPlan& P, int& cpt) {
     if (dl.sms <= 0 || dl.smem_optin <= 0) return false;
+    const int dir = mode == kModeFwd || mode == kModeFwdCkpt ? 0 : 1;
+    // coefficient records per channel in phase B
+    const int nrec = mode == kModeBwdX || mode == kModeBwdXhat ? 2 : 1;
     const int s = g.esize;
     const int NT = dir == 0 ? 1 : 2;
     const int target =
@@ -94,6 +104,9 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         if (rby % 16 != 0 || rby > 16 * 4 * kConsumers) return false;
         P.VC = (int)(rby / 16);
         cpt = P.VC <= kConsumers ? 1 : (P.VC <= 2 * kConsumers ? 2 : 4);
+        // the standard backward and the checkpointing calls run with one
+        // 16-byte column per thread
+        if (cpt > 1 && mode != kModeFwd && mode != kModeBwdZ) return false;
         P.RP = cpt == 1 ? kConsumers / P.VC : 1;
         P.unit_bytes = (int)rby;
         P.units = g.R;
@@ -103,8 +116,9 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
         P.tile_units = tr;
         P.g = 1;
         P.L = 1;
-        // merge: RP-1 row phases x VC columns x one 16-byte float4 per pair
-        if (cpt == 1 && P.RP > 1) scratch = (P.RP - 1) * P.VC * (8 / s) * 16;
+        // merge: RP-1 row phases x VC columns x per channel pair, forward two
+        // double2 (mean, M2), backward one float4 (sum dy, sum dy*y)
+        if (cpt == 1 && P.RP > 1) scratch = (P.RP - 1) * P.VC * (8 / s) * (dir == 0 ? 32 : 16);
         // TMEM stash: 1 KB (64 vectors) per consumer thread; TMEM accesses are
         // warp-wide, so every warp must hold a single row phase
         if (env_long("IABN_TMEM_STASH", 1) != 0) {
@@ -142,11 +156,12 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     if (ring < 2) ring = 2;
     if (g.layout == kNCHW) {
         // phase B coefficients of the CTA's channel window, if they fit next to
-        // the ring: min(C, planes of the largest CTA range) float4s
+        // the ring: min(C, planes of the largest CTA range) records of nrec
+        // float4s
         const int64_t G0 = g.N * g.C / P.g < dl.sms ? g.N * g.C / P.g : dl.sms;
         const int64_t planes = (P.units + G0 - 1) / G0 * P.g;
         const int64_t w = planes < g.C ? planes : g.C;
-        const int64_t bytes = round_up_int((int)std::min<int64_t>(w * 16, 1 << 20), 128);
+        const int64_t bytes = round_up_int((int)std::min<int64_t>(w * 16 * nrec, 1 << 20), 128);
         if (env_long("IABN_NCHW_SMEM_COEF", 1) != 0 &&
             1024 + kBarBytes + bytes + (int64_t)ring * P.slot_bytes <= dl.smem_optin) {
             P.ncoef = (int)w;
@@ -165,16 +180,26 @@ bool make_plan(const Geom& g, int dir, const DeviceLimits& dl, ResPlan& P, int& 
     P.smem_bytes = kBarBytes + P.scratch_bytes + nslots * P.slot_bytes;
     P.G = (int)(P.units < dl.sms ? P.units : dl.sms);
     if (P.G > kMaxPartialBlocks) P.G = kMaxPartialBlocks;
+    // the kernel counts a CTA's units in 32 bits
+    if ((P.units + P.G - 1) / P.G >= ((int64_t)1 << 31)) return false;
     P.hints = env_long("IABN_L2_HINTS", 1) != 0 ? 1 : 0;
+    P.store_hint = P.hints && env_long("IABN_STORE_HINT", 1) != 0 ? 1 : 0;
     return true;
 }
 
-cudaError_t launch(const Geom& g, const ResArgs& a, int cpt, int act, int dir, int smem_optin,
+cudaError_t launch(const Geom& g, const ResArgs& a, int cpt, int act, int mode, int smem_optin,
                    cudaStream_t s) {
+    const bool fwd = mode == kModeFwd || mode == kModeFwdCkpt;
     switch (g.dtype) {
-    case kF32: return launch_resident_f32(a, g.layout, cpt, act, dir, smem_optin, s);
-    case kBF16: return launch_resident_bf16(a, g.layout, cpt, act, dir, smem_optin, s);
-    default: return launch_resident_f16(a, g.layout, cpt, act, dir, smem_optin, s);
+    case kF32:
+        return fwd ? launch_resident_f32_fwd(a, g.layout, cpt, act, mode, smem_optin, s)
+                   : launch_resident_f32_bwd(a, g.layout, cpt, act, mode, smem_optin, s);
+    case kBF16:
+        return fwd ? launch_resident_bf16_fwd(a, g.layout, cpt, act, mode, smem_optin, s)
+                   : launch_resident_bf16_bwd(a, g.layout, cpt, act, mode, smem_optin, s);
+    default:
+        return fwd ? launch_resident_f16_fwd(a, g.layout, cpt, act, mode, smem_optin, s)
+                   : launch_resident_f16_bwd(a, g.layout, cpt, act, mode, smem_optin, s);
     }
 }
 
@@ -198,20 +223,24 @@ ResArgs base_args(const Geom& g, const Workspace& w) {
 
 }  // namespace
 
-bool resident_supported(const Geom& g) {
+bool resident_supported(const Geom& g, int layer) {
     const DeviceLimits dl = device_limits();
     ResPlan P;
     int cpt;
-    return make_plan(g, 0, dl, P, cpt) && make_plan(g, 1, dl, P, cpt);
+    return make_plan(g, layer_mode(layer, 0), dl, P, cpt) &&
+           make_plan(g, layer_mode(layer, 1), dl, P, cpt);
 }
 
-bool resident_shape(const Geom& g, int dir, int sms, int smem_optin, ResidentShape& out) {
+bool resident_shape(const Geom& g, int layer, int dir, int sms, int smem_optin,
+                    ResidentShape& out) {
     DeviceLimits dl;
     dl.sms = sms;
     dl.smem_optin = smem_optin;
     ResPlan P, Q;
     int cpt, cpt_other;
-    if (!make_plan(g, dir, dl, P, cpt) || !make_plan(g, 1 - dir, dl, Q, cpt_other)) return false;
+    if (!make_plan(g, layer_mode(layer, dir), dl, P, cpt) ||
+        !make_plan(g, layer_mode(layer, 1 - dir), dl, Q, cpt_other))
+        return false;
     const bool nhwc = g.layout == kNHWC;
     out.grid = P.G;
     out.threads = kResThreads;
@@ -233,19 +262,21 @@ cudaError_t forward_resident(const Geom& g, const FwdArgs& f, const Workspace& w
     const DeviceLimits dl = device_limits();
     ResArgs a = base_args(g, w);
     int cpt;
-    if (!make_plan(g, 0, dl, a.P, cpt)) return cudaErrorNotSupported;
+    if (!make_plan(g, f.mode, dl, a.P, cpt)) return cudaErrorNotSupported;
     a.src0 = static_cast<const unsigned char*>(f.x);
     a.src1 = nullptr;
-    a.dst = static_cast<unsigned char*>(f.x);
+    a.dst = static_cast<unsigned char*>(f.dst);
+    a.dst2 = static_cast<unsigned char*>(f.dst2);
     a.gamma = f.gamma;
     a.beta = f.beta;
+    a.mean_in = nullptr;
     a.var_in = nullptr;
     a.out0 = f.save_mean;
     a.out1 = f.save_var;
     a.eps = f.eps;
     a.p = f.act_param;
     a.inv_p = f.act == kIdent ? 1.f : 1.f / f.act_param;
-    return launch(g, a, cpt, f.act, 0, dl.smem_optin, s);
+    return launch(g, a, cpt, f.act, f.mode, dl.smem_optin, s);
 }
 
 cudaError_t backward_resident(const Geom& g, const BwdArgs& b, const Workspace& w,
@@ -253,19 +284,21 @@ cudaError_t backward_resident(const Geom& g, const BwdArgs& b, const Workspace& 
     const DeviceLimits dl = device_limits();
     ResArgs a = base_args(g, w);
     int cpt;
-    if (!make_plan(g, 1, dl, a.P, cpt)) return cudaErrorNotSupported;
-    a.src0 = static_cast<const unsigned char*>(b.z);
+    if (!make_plan(g, b.mode, dl, a.P, cpt)) return cudaErrorNotSupported;
+    a.src0 = static_cast<const unsigned char*>(b.src);
     a.src1 = static_cast<const unsigned char*>(b.dz);
     a.dst = static_cast<unsigned char*>(b.dz);
+    a.dst2 = nullptr;
     a.gamma = b.gamma;
     a.beta = b.beta;
+    a.mean_in = b.save_mean;
     a.var_in = b.save_var;
     a.out0 = b.dgamma;
     a.out1 = b.dbeta;
     a.eps = b.eps;
     a.p = b.act_param;
     a.inv_p = b.act == kIdent ? 1.f : 1.f / b.act_param;
-    return launch(g, a, cpt, b.act, 1, dl.smem_optin, s);
+    return launch(g, a, cpt, b.act, b.mode, dl.smem_optin, s);
 }
 
 }  // namespace iabn

@@ -13,14 +13,17 @@
 // a CTA-wide barrier per tile.
 //
 //   phase A  tiles 0..n-1: per-thread partial statistics from shared memory.
-//            Forward: pivot-shifted sums of x (pivot = the tensor's first row,
-//            the same in every CTA) or, NCHW, exact per-plane two-pass mean and
-//            M2.  Backward: sum dy and sum dy*y (the "INPLACE-ABN II" form; for
+//            Forward NHWC: sums of x - K and (x - K)^2 in fp32 around the
+//            thread's own first value K of each channel, turned into (mean,
+//            M2) in fp64; NCHW: exact per-plane two-pass mean and M2.
+//            Backward: sum dy and sum dy*y (the "INPLACE-ABN II" form; for
 //            leaky-ReLU dy*y = dz*z).
 //            The last D tiles land in dedicated slots and stay resident; as
 //            soon as a streamed slot frees, the producer prefetches phase B.
-//   merge    NHWC: the threads of a column add their sums in row-phase
-//            order; one partial per (CTA, channel).  NCHW: one partial per plane.
+//   merge    NHWC: the threads of a column combine their summaries in
+//            row-phase order (forward: fp64 (mean, M2) around the first
+//            phase's mean); one partial per (CTA, channel).  NCHW: one partial
+//            per plane.
 //   barrier  grid-wide (bounded wait), a distributed fp64 finalize (one warp
 //            per channel, fixed order), a second grid barrier.
 //   phase B  tiles n-1..0: resident tiles first, then the streamed ones -- the
@@ -66,6 +69,9 @@ struct ResPlan {
     int VC, RP;          // NHWC: 16-byte columns per row; row phases (threads per column)
     int g, L;            // NCHW: planes per unit; lanes per plane
     int hints;           // 1: L2 eviction-priority hints on the bulk copies
+    int store_hint;      // 1: phase B's stores carry an L2 evict-first hint, so the
+                         // results cycle through few L2 lines instead of evicting the
+                         // tiles phase B still has to read back
     int stash_first;     // 1: the stash holds each thread's first rows, 0: its last
     int stash_cp;        // 1: the copy engine (tcgen05.cp) fills the stash from the
                          // landed slots (CPT 1, RP*VC = 256, first rows); 0: the
@@ -80,11 +86,14 @@ struct ResArgs {
     ResPlan P;
     int64_t N, C, HW;
     double M;
-    const unsigned char* src0;   // forward: x;            backward: z
+    const unsigned char* src0;   // forward: x;  backward: z, x or xhat (by mode)
     const unsigned char* src1;   // backward: dz
-    unsigned char* dst;          // forward: x (z over it); backward: dz (dx over it)
+    unsigned char* dst;          // forward: z (over x, or its own buffer), checkpointing
+                                 // forward: xhat (over x); backward: dx (over dz)
+    unsigned char* dst2;         // checkpointing forward: z
     const float* gamma;
     const float* beta;
+    const float* mean_in;        // standard backward: saved mean
     const float* var_in;         // backward: saved biased variance
     float* out0;                 // forward: save_mean;  backward: dgamma
     float* out1;                 // forward: save_var;   backward: dbeta
@@ -160,6 +169,11 @@ template <> struct Pairs<kF16> {
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
+// Up to two coefficient records of one channel (phase B, NCHW).
+struct Rec2 {
+    float4 a, b;
+};
+
 // 16 bytes <-> the 16/s consecutive elements they hold, as floats.
 template <int DT>
 __device__ __forceinline__ void unpack_all(const uint4& v, float* x) {
@@ -193,8 +207,15 @@ __device__ __forceinline__ float2 act_forward2(float2 y, float p, bool slope_le1
     return y;
 }
 
-template <int DT, int ACT, int LAYOUT, int CPT, int DIR>
+template <int DT, int ACT, int LAYOUT, int CPT, int MODE>
 __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
+    constexpr int DIR = MODE == kModeFwd || MODE == kModeFwdCkpt ? 0 : 1;
+    // checkpointing forward: a second output (z) besides xhat
+    constexpr bool CKPT = MODE == kModeFwdCkpt;
+    // backward from a stored x or xhat: y is recomputed by a scale and shift
+    constexpr bool SRCV = MODE == kModeBwdX || MODE == kModeBwdXhat;
+    // coefficient records per channel for phase B
+    constexpr int NREC = SRCV ? 2 : 1;
     constexpr int NT = DIR == 0 ? 1 : 2;       // tensors per tile
     constexpr int NP = Pairs<DT>::NP;          // channel pairs per 16-byte vector
     constexpr int NQ = CPT * NP;               // channel pairs per thread (NHWC)
@@ -206,10 +227,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     uint64_t* done = empty + kMaxSlots;
     uint64_t* cpdone = done + kMaxSlots;   // TMEM copies out of a slot have finished
     __shared__ int s_fail;
-    // gamma, beta (and, backward, the saved variance; forward NHWC, the pivot
-    // word) of the first channel each consumer half-warp finalizes, fetched
-    // while phase A streams
-    __shared__ float s_par[kConsumerWarps][2][3];
+    // gamma, beta (and, backward, the saved variance and, standard backward,
+    // the saved mean) of the first channel each consumer half-warp finalizes,
+    // fetched while phase A streams
+    __shared__ float s_par[kConsumerWarps][2][4];
 
     const ResPlan& P = a.P;
     unsigned char* scratch = smem + kBarBytes;
@@ -258,8 +279,11 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
     };
 
-    const int64_t u0 = (int64_t)b * P.units / G;
-    const int64_t u1 = (int64_t)(b + 1) * P.units / G;
+    // CTA b owns units [u0, u1): uq each, one more for the first ur CTAs
+    const int64_t uq = P.units / G;
+    const int ur = (int)(P.units - uq * G);
+    const int64_t u0 = (int64_t)b * uq + min(b, ur);
+    const int64_t u1 = u0 + uq + (b < ur ? 1 : 0);
     const int n = (int)((u1 - u0 + P.tile_units - 1) / P.tile_units);
     const int ring = P.ring;
     const int D = min(P.nslots - ring, n);
@@ -312,9 +336,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             cp_async4(&s_par[warp][h][0], a.gamma + c);
             cp_async4(&s_par[warp][h][1], a.beta + c);
             if (DIR == 1) cp_async4(&s_par[warp][h][2], a.var_in + c);
-            // forward NHWC: the aligned word holding the pivot x[0, c]
-            if (DIR == 0 && LAYOUT == kNHWC)
-                cp_async4(&s_par[warp][h][2], a.src0 + ((c * (int64_t)sizeof(typename Storage<DT>::T)) & ~int64_t(3)));
+            if (MODE == kModeBwdX) cp_async4(&s_par[warp][h][3], a.mean_in + c);
         }
     }
     if (stash && warp == 0) {
@@ -496,7 +518,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const float p = a.p, inv_p = a.inv_p;
     const bool le1 = p <= 1.f;
 
-    // NHWC accumulators: forward (sum d, sum d^2 with d = x - pivot); backward
+    // NHWC accumulators: forward (sum d, sum d^2 with d = x - K); backward
     // (sum dy, sum dy*y).
     float2 acc0[NQ], acc1[NQ], piv[NQ];
 #pragma unroll
@@ -505,17 +527,56 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         acc1[q] = f2(0.f, 0.f);
         piv[q] = f2(0.f, 0.f);
     }
-    if (DIR == 0 && LAYOUT == kNHWC && active) {
-        // pivot (negated): the tensor's first row, the same for every CTA, so
-        // the CTA partials are plain sums around it (no per-CTA counts)
+    // rows of the CTA's range this thread accumulates (NHWC): phase, phase +
+    // RP, ...
+    // (a CTA owns fewer than 2^31 units; the host plan checks it)
+    const int nrows32 = (int)nrows;
+    const int rq = nrows32 / RP, rr = nrows32 - rq * RP;   // rows per phase: rq or rq + 1
+    const int my_n = LAYOUT == kNHWC ? rq + (phase < rr ? 1 : 0) : 0;
+    if (DIR == 0 && LAYOUT == kNHWC && active && my_n > 0) {
+        // pivot K (kept negated): the thread's own first value of each of its
+        // channels, so its fp32 sums stay as small as the channel's spread
+        // allows whatever the data's offset (a pivot shared by the whole grid
+        // loses accuracy when that one value is far from the mean)
+        const uint4* row = reinterpret_cast<const uint4*>(a.src0 + (u0 + phase) * (int64_t)RBY);
 #pragma unroll
         for (int k = 0; k < CPT; ++k)
             if (colok[k]) {
                 float2 f[NP];
-                Pairs<DT>::unpack(__ldg(reinterpret_cast<const uint4*>(a.src0) + col[k]), f);
+                Pairs<DT>::unpack(__ldg(row + col[k]), f);
 #pragma unroll
                 for (int q = 0; q < NP; ++q) piv[k * NP + q] = f2(-f[q].x, -f[q].y);
             }
+    }
+
+    // standard / checkpointing backward (NHWC): the constants with which this
+    // thread recovers xhat and y from the stored values of its channels
+    float2 pxs[NQ], pxb[NQ], pys[NQ], pyb[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+        pxs[q] = f2(1.f, 1.f);
+        pxb[q] = pys[q] = pyb[q] = f2(0.f, 0.f);
+    }
+    if (SRCV && LAYOUT == kNHWC && active) {
+#pragma unroll
+        for (int k = 0; k < CPT; ++k)
+            if (colok[k])
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    const int j = k * NP + q;
+                    const int64_t ch = (int64_t)(col[k] * NP + q) * 2;
+                    float v[2][4];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        src_affine<MODE>(__ldg(a.gamma + ch + e), __ldg(a.beta + ch + e),
+                                         MODE == kModeBwdX ? __ldg(a.mean_in + ch + e) : 0.f,
+                                         MODE == kModeBwdX ? __ldg(a.var_in + ch + e) : 1.f,
+                                         a.eps, v[e][0], v[e][1], v[e][2], v[e][3]);
+                    pxs[j] = f2(v[0][0], v[1][0]);
+                    pxb[j] = f2(v[0][1], v[1][1]);
+                    pys[j] = f2(v[0][2], v[1][2]);
+                    pyb[j] = f2(v[0][3], v[1][3]);
+                }
     }
 
     if (copier && lane == 0 && scp) {
@@ -620,6 +681,25 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                                         const float2 d = __fadd2_rn(f[q], piv[j]);
                                         acc0[j] = __fadd2_rn(acc0[j], d);
                                         acc1[j] = __ffma2_rn(d, d, acc1[j]);
+                                    }
+                                } else if (SRCV) {
+                                    // standard / checkpointing: xhat and y from the
+                                    // stored value, dy from y
+                                    float2 fa[NP], fd[NP];
+                                    Pairs<DT>::unpack(vz[u][k], fa);
+                                    Pairs<DT>::unpack(vd[u][k], fd);
+#pragma unroll
+                                    for (int q = 0; q < NP; ++q) {
+                                        const int j = k * NP + q;
+                                        const float2 xh = MODE == kModeBwdX
+                                                              ? __ffma2_rn(fa[q], pxs[j], pxb[j])
+                                                              : fa[q];
+                                        const float2 y = __ffma2_rn(fa[q], pys[j], pyb[j]);
+                                        const float2 dy =
+                                            f2(act_dy_from_y<ACT, DT>(y.x, fd[q].x, p),
+                                               act_dy_from_y<ACT, DT>(y.y, fd[q].y, p));
+                                        acc0[j] = __fadd2_rn(acc0[j], dy);
+                                        acc1[j] = __ffma2_rn(dy, xh, acc1[j]);
                                     }
                                 } else {
                                     float2 fz[NP], fd[NP];
@@ -737,6 +817,44 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                                 make_double2((double)piv + d1 * (double)inv_hw_d,
                                              (double)s2 - d1 * d1 * (double)inv_hw_d);
                         }
+                    } else if (SRCV) {
+                        // standard / checkpointing: xhat and y from the stored
+                        // value with the plane's channel constants
+                        float s1a = 0.f, sya = 0.f, s1b = 0.f, syb = 0.f;
+                        if (valid) {
+                            const int64_t c = (plane0 + pp) % a.C;
+                            float xs, xb, ys, yb;
+                            src_affine<MODE>(__ldg(a.gamma + c), __ldg(a.beta + c),
+                                             MODE == kModeBwdX ? __ldg(a.mean_in + c) : 0.f,
+                                             MODE == kModeBwdX ? __ldg(a.var_in + c) : 1.f,
+                                             a.eps, xs, xb, ys, yb);
+                            auto add = [&](float av, float dv, float& s1, float& sy) {
+                                const float xh = MODE == kModeBwdX ? fmaf(av, xs, xb) : av;
+                                const float dy = act_dy_from_y<ACT, DT>(fmaf(av, ys, yb), dv, p);
+                                s1 += dy;
+                                sy = fmaf(dy, xh, sy);
+                            };
+                            const unsigned char* pd = pz + P.half_bytes;
+                            int i = glane;
+                            for (; i < lim(); i += PC * L) {
+                                float av[PC], dv[PC];
+#pragma unroll
+                                for (int k = 0; k < PC; ++k) {
+                                    av[k] = Elem<DT>::ld(pz, i + k * L);
+                                    dv[k] = Elem<DT>::ld(pd, i + k * L);
+                                }
+#pragma unroll
+                                for (int k = 0; k < PC; k += 2) {
+                                    add(av[k], dv[k], s1a, sya);
+                                    add(av[k + 1], dv[k + 1], s1b, syb);
+                                }
+                            }
+                            for (; i < HW; i += L)
+                                add(Elem<DT>::ld(pz, i), Elem<DT>::ld(pd, i), s1a, sya);
+                        }
+                        const float s1 = group_sum(s1a + s1b, L);
+                        const float sy = group_sum(sya + syb, L);
+                        if (valid && glane == 0) a.part[plane0 + pp] = make_double2(s1, sy);
                     } else {
                         float s1a = 0.f, sya = 0.f, s1b = 0.f, syb = 0.f;
                         if (valid) {
@@ -785,7 +903,81 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     stamp(1, tid == 0);
 
     // ------------------------------------------- per-CTA merge (NHWC)
-    if (!failed() && LAYOUT == kNHWC) {
+    if (!failed() && LAYOUT == kNHWC && DIR == 0) {
+        // Forward: each thread's sums around its pivot K become (mean, M2) in
+        // fp64: mean = K + S1/n, M2 = S2 - S1^2/n.  Row phases 1..RP-1 publish
+        // them ([phase-1][pair][mean | M2][column] double2s); phase 0 adds them
+        // around its own mean R in phase order:
+        //   s1 = sum n_p (mean_p - R),  s2 = sum M2_p + n_p (mean_p - R)^2,
+        // giving the CTA's (R + s1/n, s2 - s1^2/n) over its nrows rows.
+        const double inv_n = my_n > 0 ? 1.0 / (double)my_n : 0.0;
+        auto summary = [&](int i, double2& mean, double2& m2) {
+            const double s1x = acc0[i].x, s1y = acc0[i].y;
+            mean = make_double2(s1x * inv_n - (double)piv[i].x, s1y * inv_n - (double)piv[i].y);
+            m2 = make_double2((double)acc1[i].x - s1x * s1x * inv_n,
+                              (double)acc1[i].y - s1y * s1y * inv_n);
+        };
+        if (CPT == 1 && RP > 1) {
+            double2* scr = reinterpret_cast<double2*>(scratch);
+            if (colok[0] && phase > 0 && my_n > 0) {
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    double2 mean, m2;
+                    summary(q, mean, m2);
+                    scr[(((phase - 1) * NP + q) * 2) * VC + col[0]] = mean;
+                    scr[(((phase - 1) * NP + q) * 2 + 1) * VC + col[0]] = m2;
+                }
+            }
+            __syncthreads();
+            if (colok[0] && phase == 0) {
+                const double inv_rows = 1.0 / (double)nrows;
+                double2 R[NP], s1[NP], s2[NP];
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    summary(q, R[q], s2[q]);
+                    s1[q] = make_double2(0.0, 0.0);
+                }
+                for (int ph = 1; ph < RP && ph < nrows32; ++ph) {
+                    const double np = (double)(rq + (ph < rr ? 1 : 0));
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const double2 m = scr[(((ph - 1) * NP + q) * 2) * VC + col[0]];
+                        const double2 v = scr[(((ph - 1) * NP + q) * 2 + 1) * VC + col[0]];
+                        const double dx = m.x - R[q].x, dy = m.y - R[q].y;
+                        s1[q].x += np * dx;
+                        s1[q].y += np * dy;
+                        s2[q].x += v.x + np * dx * dx;
+                        s2[q].y += v.y + np * dy * dy;
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    const int64_t ch = (int64_t)(col[0] * NP + q) * 2;
+                    double2* dstp = a.part + (int64_t)b * a.C + ch;
+                    dstp[0] = make_double2(R[q].x + s1[q].x * inv_rows,
+                                           s2[q].x - s1[q].x * s1[q].x * inv_rows);
+                    dstp[1] = make_double2(R[q].y + s1[q].y * inv_rows,
+                                           s2[q].y - s1[q].y * s1[q].y * inv_rows);
+                }
+            }
+        } else if (active && phase == 0) {
+            // one thread per column: its summary is the CTA's
+#pragma unroll
+            for (int k = 0; k < CPT; ++k)
+                if (colok[k])
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        double2 mean, m2;
+                        summary(k * NP + q, mean, m2);
+                        const int64_t ch = (int64_t)(col[k] * NP + q) * 2;
+                        double2* dstp = a.part + (int64_t)b * a.C + ch;
+                        dstp[0] = make_double2(mean.x, m2.x);
+                        dstp[1] = make_double2(mean.y, m2.y);
+                    }
+        }
+        stamp(6, tid == 0);
+    }
+    if (!failed() && LAYOUT == kNHWC && DIR == 1) {
         if (CPT == 1 && RP > 1) {
             // Row phases 1..RP-1 publish their sums ([phase-1][pair][column]
             // float4s, so a warp's stores and loads are contiguous); phase 0
@@ -813,7 +1005,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
         stamp(6, tid == 0);
         if (active && phase == 0) {
-            // forward: (sum d, sum d^2) around the pivot; backward: (sum dy, sum dy*y)
+            // (sum dy, sum dy*y)
 #pragma unroll
             for (int k = 0; k < CPT; ++k)
                 if (colok[k])
@@ -838,6 +1030,23 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         atomicOr(&a.ctl->status, kStTimeout);
         set_failed();
     }
+    // Finalize (below): one consumer half-warp per channel pair, each lane
+    // caching up to KC partials k = lane%16 + 16 i.  The forward weighs them by
+    // the values behind them: NHWC, the rows of CTA k; NCHW, one plane.  Their
+    // counts are known before the partials are.
+    constexpr int KC = 10;   // partials cached per lane when K <= 160
+    const int64_t K = LAYOUT == kNHWC ? (int64_t)G : a.N;
+    const bool cached = K <= 16 * KC;
+    auto count_of = [&](int64_t k) -> double {
+        if (LAYOUT == kNCHW) return (double)a.HW;
+        return (double)(uq + (k < ur ? 1 : 0));
+    };
+    double wk[KC];
+#pragma unroll
+    for (int i = 0; i < KC; ++i) {
+        const int64_t k = (lane & 15) + 16 * i;
+        wk[i] = DIR == 0 && consumer && cached && k < K ? count_of(k) : 0.0;
+    }
     grid_barrier(a.ctl, bbase + (uint32_t)G, a.budget_ns, &s_fail);
     stamp(3, tid == 0);
     if (consumer && (lane & 15) == 0) cp_async_wait_all();   // s_par (issued at launch)
@@ -847,17 +1056,6 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         // warp-uniform; a half without a channel computes on a stand-in)
         const int hl = lane & 15, half = lane >> 4;
         const int64_t nw = (int64_t)G * kConsumerWarps;
-        const int64_t K = LAYOUT == kNHWC ? (int64_t)G : a.N;
-        constexpr int KC = 10;   // partials cached per lane when K <= 160
-        const bool cached = K <= 16 * KC;
-        const double hw = (double)a.HW;   // elements behind each NCHW partial
-        // the pivot x[0, c] from the aligned 32-bit word that holds it
-        auto pivot_of = [&](uint32_t w, int64_t c) -> float {
-            if (DT == kF32) return __uint_as_float(w);
-            const uint32_t h = (c & 1) ? (w >> 16) : (w & 0xffffu);
-            if (DT == kBF16) return __uint_as_float(h << 16);
-            return __half2float(__ushort_as_half((unsigned short)h));
-        };
         bool first = true;
         for (int64_t cpair = (int64_t)b * kConsumerWarps + warp; cpair * 2 < a.C;
              cpair += nw, first = false) {
@@ -871,58 +1069,45 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 pk[i] = cached && k < K ? a.part[k * a.C + c] : make_double2(0.0, 0.0);
             }
             // per-channel parameters (lane 0 of the half uses them)
-            float gmf = 0.f, btf = 0.f, vif = 0.f;
+            float gmf = 0.f, btf = 0.f, vif = 0.f, mnf = 0.f;
             if (hl == 0) {
                 if (first) {
                     gmf = s_par[warp][half][0];
                     btf = s_par[warp][half][1];
                     vif = s_par[warp][half][2];
+                    mnf = s_par[warp][half][3];
                 } else {
                     gmf = a.gamma[c];
                     btf = a.beta[c];
                     if (DIR == 1) vif = a.var_in[c];
-                    if (DIR == 0 && LAYOUT == kNHWC)
-                        vif = __uint_as_float(*reinterpret_cast<const uint32_t*>(
-                            a.src0 + ((c * (int64_t)sizeof(typename Storage<DT>::T)) & ~int64_t(3))));
+                    if (MODE == kModeBwdX) mnf = a.mean_in[c];
                 }
             }
             if (DIR == 0) {
-                // NHWC partials are sums around the pivot p (mean = p + s1/M,
-                // M2 = s2 - s1^2/M).  NCHW partials are per-plane (mean, M2): one
-                // pass around r, the first plane's mean:
-                //   s1 = sum n (mean_k - r),  s2 = sum M2_k + n (mean_k - r)^2.
-                double r = 0.0;
-                if (LAYOUT == kNCHW)
-                    r = __shfl_sync(0xffffffffu, cached ? pk[0].x : a.part[c].x, 0, 16);
+                // Partials are (mean_k, M2_k) over n_k values (NHWC: CTA k's
+                // rows; NCHW: plane k).  One pass around r, the first
+                // partial's mean:
+                //   s1 = sum n_k (mean_k - r),  s2 = sum M2_k + n_k (mean_k - r)^2,
+                //   mean = r + s1/M,  M2 = s2 - s1^2/M.
+                const double r = __shfl_sync(0xffffffffu, cached ? pk[0].x : a.part[c].x, 0, 16);
                 double s1 = 0.0, s2 = 0.0;
                 if (cached) {
 #pragma unroll
                     for (int i = 0; i < KC; ++i) {
-                        if (LAYOUT == kNHWC) {
-                            s1 += pk[i].x;
-                            s2 += pk[i].y;
-                        } else {
-                            const double w = (hl + 16 * i < K ? hw : 0.0) * (pk[i].x - r);
-                            s1 += w;
-                            s2 += pk[i].y + w * (pk[i].x - r);
-                        }
+                        const double w = wk[i] * (pk[i].x - r);
+                        s1 += w;
+                        s2 += pk[i].y + w * (pk[i].x - r);
                     }
                 } else {
                     for (int64_t k = hl; k < K; k += 16) {
                         const double2 v = a.part[k * a.C + c];
-                        if (LAYOUT == kNHWC) {
-                            s1 += v.x;
-                            s2 += v.y;
-                        } else {
-                            const double w = hw * (v.x - r);
-                            s1 += w;
-                            s2 += v.y + w * (v.x - r);
-                        }
+                        const double w = count_of(k) * (v.x - r);
+                        s1 += w;
+                        s2 += v.y + w * (v.x - r);
                     }
                 }
                 s1 = half_warp_sum(s1);
                 s2 = half_warp_sum(s2);
-                if (LAYOUT == kNHWC && hl == 0) r = (double)pivot_of(__float_as_uint(vif), c);
                 if (hl == 0 && cv) {
                     const double mean = r + s1 / a.M;
                     const double var = fmax((s2 - s1 * (s1 / a.M)) / a.M, 0.0);
@@ -930,9 +1115,16 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     a.out1[c] = (float)var;
                     const double rstd = 1.0 / sqrt(var + (double)a.eps);
                     const double sc = (double)gmf * rstd;
-                    // (mean, scale, beta, beta - mean*scale)
-                    a.coef[c] = make_float4((float)mean, (float)sc, btf,
-                                            (float)((double)btf - mean * sc));
+                    if (CKPT) {
+                        // xhat = (x - mean)*rstd (fp32 storage) or x*rstd - mean*rstd;
+                        // y = gamma*xhat + beta
+                        a.coef[c] = make_float4(DT == kF32 ? (float)-mean : (float)(-mean * rstd),
+                                                (float)rstd, gmf, btf);
+                    } else {
+                        // (mean, scale, beta, beta - mean*scale)
+                        a.coef[c] = make_float4((float)mean, (float)sc, btf,
+                                                (float)((double)btf - mean * sc));
+                    }
                 }
             } else {
                 double s1 = 0.0, sy = 0.0;
@@ -951,7 +1143,23 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 }
                 s1 = half_warp_sum(s1);
                 sy = half_warp_sum(sy);
-                if (hl == 0 && cv) {
+                if (SRCV && hl == 0 && cv) {
+                    // standard / checkpointing: dbeta = sum dy, dgamma = sum dy*xhat;
+                    // dx = A dy + B xhat + Cc with A = gamma rstd, B = -A dgamma/M,
+                    // Cc = -A dbeta/M, applied to the stored value a through
+                    // xhat = a*xs + xb:  dx = A dy + (B xs) a + (B xb + Cc)
+                    float xs, xb, ys, yb;
+                    src_affine<MODE>(gmf, btf, mnf, vif, a.eps, xs, xb, ys, yb);
+                    const double rstd = 1.0 / sqrt((double)vif + (double)a.eps);
+                    const double A = (double)gmf * rstd;
+                    const double B = -A * sy / a.M, Cc = -A * s1 / a.M;
+                    a.out0[c] = (float)sy;
+                    a.out1[c] = (float)s1;
+                    a.coef[c] = make_float4(ys, yb, (float)A, 0.f);
+                    a.coef[a.C + c] = make_float4((float)(B * (double)xs),
+                                                  (float)(B * (double)xb + Cc), 0.f, 0.f);
+                }
+                if (!SRCV && hl == 0 && cv) {
                     const double gm = gmf, bt = btf;
                     const double rstd = 1.0 / sqrt((double)vif + (double)a.eps);
                     if (!(fabs(gm) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN
@@ -985,7 +1193,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         if (consumer && !failed())
             for (int i = tid; i < P.ncoef; i += kConsumers) {
                 const int64_t c = ch0 + i;
-                scoef[i] = a.coef[c >= a.C ? c - a.C : c];
+                const int64_t cm = c >= a.C ? c - a.C : c;
+                scoef[i] = a.coef[cm];
+                if (NREC == 2) scoef[P.ncoef + i] = a.coef[a.C + cm];
             }
         __syncthreads();
     }
@@ -1011,6 +1221,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             stamp(7, true);
         }
     } else if (consumer && !failed()) {
+        // results go straight to global memory (16-byte stores)
+        const uint64_t pol_st = P.store_hint ? policy_evict_first() : policy_evict_normal();
+        auto put = [&](void* g, const uint4& v) { stg128_hint(g, v, pol_st); };
         // coefficients of this thread's channels (NHWC)
         // c3/c4 are kept per channel only when a thread owns one column;
         // otherwise the backward forms them on the fly (register budget).
@@ -1021,12 +1234,29 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
                 const int i = k * NP + q;
-                float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+                float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0, w0 = v0, w1 = v0;
                 if (colok[k]) {
                     v0 = a.coef[(col[k] * NP + q) * 2];
                     v1 = a.coef[(col[k] * NP + q) * 2 + 1];
+                    if (NREC == 2) {
+                        w0 = a.coef[a.C + (col[k] * NP + q) * 2];
+                        w1 = a.coef[a.C + (col[k] * NP + q) * 2 + 1];
+                    }
                 }
-                if (DIR == 0) {
+                if (CKPT) {
+                    // the checkpointing layer runs with one column per thread
+                    c0[i] = f2(v0.x, v1.x);                   // -mean or -mean*rstd
+                    c1[i] = f2(v0.y, v1.y);                   // rstd
+                    c2[i] = f2(v0.z, v1.z);                   // gamma
+                    c3[i < NQ34 ? i : 0] = f2(v0.w, v1.w);    // beta
+                } else if (SRCV) {
+                    // y = a*ys + yb; dx = A dy + B' a + C' (one column per thread)
+                    c0[i] = f2(v0.x, v1.x);                   // ys
+                    c1[i] = f2(v0.y, v1.y);                   // yb
+                    c2[i] = f2(v0.z, v1.z);                   // A
+                    c3[i < NQ34 ? i : 0] = f2(w0.x, w1.x);    // B'
+                    c4[i < NQ34 ? i : 0] = f2(w0.y, w1.y);    // C'
+                } else if (DIR == 0) {
                     c0[i] = f2(-v0.x, -v1.x);    // -mean
                     c1[i] = f2(v0.y, v1.y);      // scale
                     c2[i] = f2(v0.w, v1.w);      // beta - mean*scale (16-bit storage)
@@ -1044,11 +1274,40 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         // Rewrites the tile in slot s in place (forward: x -> z; backward: dz -> dx).
         // Rewrites one row's CPT vectors: forward x -> z in vz, backward
         // dz -> dx in vd (z in vz).
-        auto rewrite = [&](uint4* vz, uint4* vd) {
+        // (checkpointing forward: xhat into vz, z into vo.)
+        auto rewrite = [&](uint4* vz, uint4* vd, uint4* vo) {
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
                 if (CPT > 1 && !colok[k]) continue;
-                if (DIR == 0) {
+                if (CKPT) {
+                    float2 f[NP], o[NP];
+                    Pairs<DT>::unpack(vz[k], f);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const int j = k * NP + q;
+                        const float2 xh = DT == kF32 ? __fmul2_rn(__fadd2_rn(f[q], c0[j]), c1[j])
+                                                     : __ffma2_rn(f[q], c1[j], c0[j]);
+                        o[q] = act_forward2<ACT, DT>(__ffma2_rn(xh, c2[j], c3[j < NQ34 ? j : 0]),
+                                                     p, le1);
+                        f[q] = xh;
+                    }
+                    vz[k] = Pairs<DT>::pack(f);
+                    vo[k] = Pairs<DT>::pack(o);
+                } else if (SRCV) {
+                    float2 fa[NP], fd[NP];
+                    Pairs<DT>::unpack(vz[k], fa);
+                    Pairs<DT>::unpack(vd[k], fd);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const int j = k * NP + q;
+                        const int jj = j < NQ34 ? j : 0;
+                        const float2 y = __ffma2_rn(fa[q], c0[j], c1[j]);
+                        const float2 dy = f2(act_dy_from_y<ACT, DT>(y.x, fd[q].x, p),
+                                             act_dy_from_y<ACT, DT>(y.y, fd[q].y, p));
+                        fd[q] = __ffma2_rn(c2[j], dy, __ffma2_rn(c3[jj], fa[q], c4[jj]));
+                    }
+                    vd[k] = Pairs<DT>::pack(fd);
+                } else if (DIR == 0) {
                     float2 f[NP];
                     Pairs<DT>::unpack(vz[k], f);
 #pragma unroll
@@ -1104,9 +1363,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 const uint32_t sb = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
                 const uint32_t hb = DIR == 0 ? 0u : (uint32_t)P.half_bytes;
                 unsigned char* gtile = a.dst + t_u0(t) * P.unit_bytes;
+                unsigned char* gtile2 = CKPT ? a.dst2 + t_u0(t) * P.unit_bytes : nullptr;
                 // rows in batches of RB: loads, then math, then stores
                 for (int i0 = max(qlo, 0); i0 < m; i0 += RB) {
-                    uint4 vz[RB][CPT], vd[RB][CPT];
+                    uint4 vz[RB][CPT], vd[RB][CPT], vo[RB][CPT];
 #pragma unroll
                     for (int u = 0; u < RB; ++u)
 #pragma unroll
@@ -1118,15 +1378,16 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         }
 #pragma unroll
                     for (int u = 0; u < RB; ++u)
-                        if (i0 + u < m) rewrite(vz[u], vd[u]);
+                        if (i0 + u < m) rewrite(vz[u], vd[u], vo[u]);
                     // results go straight to their place in global memory
 #pragma unroll
                     for (int u = 0; u < RB; ++u)
 #pragma unroll
                         for (int k = 0; k < CPT; ++k) {
                             if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
-                            unsigned char* g = gtile + voff[k] + (size_t)(i0 + u) * vstep;
-                            stg128(g, DIR == 0 ? vz[u][k] : vd[u][k]);
+                            const size_t o = voff[k] + (size_t)(i0 + u) * vstep;
+                            put(gtile + o, DIR == 0 ? vz[u][k] : vd[u][k]);
+                            if (CKPT) put(gtile2 + o, vo[u][k]);
                         }
                 }
             } else {
@@ -1139,12 +1400,23 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 // window index of the tile's first plane (channel = ch0 + index mod C)
                 const uint32_t ibase = (uint32_t)(((t_u0(t) - u0) * P.g) % a.C);
                 const uint32_t sbv = slots_sa + (uint32_t)s * (uint32_t)P.slot_bytes;
-                auto coef_at = [&](uint32_t i) -> float4 {
-                    if (P.ncoef > 0) return scoef[i];
-                    const int64_t c = ch0 + i;
-                    return a.coef[c >= a.C ? c - a.C : c];
+                // coefficient record(s) of window index i (second record: the
+                // standard / checkpointing backward's B' and C')
+                auto coef_at = [&](uint32_t i) -> Rec2 {
+                    Rec2 r;
+                    if (P.ncoef > 0) {
+                        r.a = scoef[i];
+                        r.b = NREC == 2 ? scoef[P.ncoef + i] : r.a;
+                    } else {
+                        const int64_t c = ch0 + i;
+                        const int64_t cm = c >= a.C ? c - a.C : c;
+                        r.a = a.coef[cm];
+                        r.b = NREC == 2 ? a.coef[a.C + cm] : r.a;
+                    }
+                    return r;
                 };
                 unsigned char* gt = a.dst + t_u0(t) * P.unit_bytes;
+                unsigned char* gt2 = CKPT ? a.dst2 + t_u0(t) * P.unit_bytes : nullptr;
                 // This thread's vectors v = tid + kConsumers*j start ES elements
                 // apart: its plane offset `off` and window index `c` advance by
                 // fixed steps (dq planes + dr elements), no division per vector.
@@ -1166,14 +1438,24 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     const uint4 vz = lds128(sbv + (uint32_t)v * 16u);
                     uint4 vd = vz;
                     if (DIR == 1) vd = lds128(sbv + (uint32_t)P.half_bytes + (uint32_t)v * 16u);
-                    float xz[EPV], xd[EPV];
+                    float xz[EPV], xd[EPV], xo[EPV];
                     unpack_all<DT>(vz, xz);
                     if (DIR == 1) unpack_all<DT>(vd, xd);
                     // one element with coefficients q: forward (16-bit) y = x*scale +
                     // (beta - mean*scale), (fp32) y = (x - mean)*scale + beta;
-                    // backward dx = A dy + B y + Cc
-                    auto rewrite_elem = [&](int k, const float4& q) {
-                        if (DIR == 0) {
+                    // backward dx = A dy + B y + Cc; checkpointing forward xhat and
+                    // z = phi(gamma*xhat + beta); standard / checkpointing backward
+                    // y = a*ys + yb, dx = A dy + B' a + C'
+                    auto rewrite_elem = [&](int k, const Rec2& r) {
+                        const float4& q = r.a;
+                        if (CKPT) {
+                            const float xh = DT == kF32 ? (xz[k] + q.x) * q.y : fmaf(xz[k], q.y, q.x);
+                            xo[k] = act_forward<ACT, DT>(fmaf(xh, q.z, q.w), p);
+                            xz[k] = xh;
+                        } else if (SRCV) {
+                            const float dy = act_dy_from_y<ACT, DT>(fmaf(xz[k], q.x, q.y), xd[k], p);
+                            xz[k] = fmaf(q.z, dy, fmaf(r.b.x, xz[k], r.b.y));
+                        } else if (DIR == 0) {
                             const float y = DT == kF32 ? fmaf(xz[k] - q.x, q.y, q.z)
                                                        : fmaf(xz[k], q.y, q.w);
                             xz[k] = act_forward<ACT, DT>(y, p);
@@ -1186,16 +1468,14 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     if (hw >= (uint32_t)EPV) {
                         // planes at least a vector long: two coefficient sets at
                         // most, chosen per element without branches
-                        const float4 q0 = coef_at(cc), q1 = coef_at(cc + 1u == C32 ? 0u : cc + 1u);
+                        const Rec2 q0 = coef_at(cc), q1 = coef_at(cc + 1u == C32 ? 0u : cc + 1u);
 #pragma unroll
                         for (int k = 0; k < EPV; ++k) {
                             const bool first = (uint32_t)k < rem;
-                            const float4 q = make_float4(first ? q0.x : q1.x, first ? q0.y : q1.y,
-                                                         first ? q0.z : q1.z, first ? q0.w : q1.w);
-                            rewrite_elem(k, q);
+                            rewrite_elem(k, first ? q0 : q1);
                         }
                     } else {
-                        float4 q = coef_at(cc);
+                        Rec2 q = coef_at(cc);
 #pragma unroll
                         for (int k = 0; k < EPV; ++k) {
                             if (rem == 0u) {
@@ -1214,7 +1494,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         ++c;
                     }
                     if (c >= C32) c -= C32;
-                    stg128(gt + (size_t)v * 16, pack_all<DT>(xz));
+                    put(gt + (size_t)v * 16, pack_all<DT>(xz));
+                    if (CKPT) put(gt2 + (size_t)v * 16, pack_all<DT>(xo));
                 }
             }
         };
@@ -1224,10 +1505,11 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             // tensor): this thread's column k of group i is at TMEM column
             // 8*(NT*(i*CPT + k) + tensor) + 4*(warp/4)
             unsigned char* grow = a.dst + u0 * P.unit_bytes;
+            unsigned char* grow2 = CKPT ? a.dst2 + u0 * P.unit_bytes : nullptr;
             const uint32_t ta = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) +
                                 (uint32_t)(4 * ((warp >> 2) & 1));
             for (int i0 = 0; i0 < Jc; i0 += RB) {
-                uint4 bz[RB * CPT], bd[RB * CPT];
+                uint4 bz[RB * CPT], bd[RB * CPT], bo[RB * CPT];
                 const uint32_t f0 = (uint32_t)(i0 * CPT);
                 tmem_ld4x4(ta + 8u * NT * f0, 8u * NT, bz);
                 if (NT == 2) tmem_ld4x4(ta + 8u * NT * f0 + 8u, 8u * NT, bd);
@@ -1236,15 +1518,19 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     if (i0 + u >= Jc) continue;
                     uint4* vz = bz + u * CPT;
                     uint4* vd = NT == 2 ? bd + u * CPT : bz + u * CPT;
-                    rewrite(vz, vd);
+                    rewrite(vz, vd, bo + u * CPT);
 #pragma unroll
-                    for (int k = 0; k < CPT; ++k)
-                        stg128(grow + voff[k] + (size_t)(i0 + u) * vstep, DIR == 0 ? vz[k] : vd[k]);
+                    for (int k = 0; k < CPT; ++k) {
+                        const size_t o = voff[k] + (size_t)(i0 + u) * vstep;
+                        put(grow + o, DIR == 0 ? vz[k] : vd[k]);
+                        if (CKPT) put(grow2 + o, bo[u * CPT + k]);
+                    }
                 }
             }
         } else if (stash && active) {
             // the stashed rows first: no wait for any tile
             unsigned char* grow = a.dst + u0 * P.unit_bytes;
+            unsigned char* grow2 = CKPT ? a.dst2 + u0 * P.unit_bytes : nullptr;
             for (int i0 = 0; i0 < Jc; i0 += RB) {
                 uint4 buf[RB * VPR];   // RB*CPT = 4 vectors per tensor
                 if (NT == 1) tmem_ld16(tm_thread + (uint32_t)(i0 * VPR * 4), buf);
@@ -1252,18 +1538,19 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
 #pragma unroll
                 for (int u = 0; u < RB; ++u) {
                     if (i0 + u >= Jc) continue;
-                    uint4 vz[CPT], vd[CPT];
+                    uint4 vz[CPT], vd[CPT], vo[CPT];
 #pragma unroll
                     for (int k = 0; k < CPT; ++k) {
                         vz[k] = buf[(u * CPT + k) * NT];
                         vd[k] = buf[(u * CPT + k) * NT + (NT - 1)];
                     }
-                    rewrite(vz, vd);
+                    rewrite(vz, vd, vo);
                     const size_t j = (size_t)(js + i0 + u);
 #pragma unroll
                     for (int k = 0; k < CPT; ++k) {
                         if (CPT > 1 && !colok[k]) continue;
-                        stg128(grow + voff[k] + j * vstep, DIR == 0 ? vz[k] : vd[k]);
+                        put(grow + voff[k] + j * vstep, DIR == 0 ? vz[k] : vd[k]);
+                        if (CKPT) put(grow2 + voff[k] + j * vstep, vo[k]);
                     }
                 }
             }
@@ -1323,9 +1610,9 @@ namespace iabn {
 
 // Launches one instantiation cooperatively (all CTAs co-resident, which the
 // grid barrier relies on).
-template <int DT, int ACT, int LAYOUT, int CPT, int DIR>
+template <int DT, int ACT, int LAYOUT, int CPT, int MODE>
 cudaError_t launch_resident_one(const ResArgs& a, int smem_optin, cudaStream_t s) {
-    auto kern = k_resident<DT, ACT, LAYOUT, CPT, DIR>;
+    auto kern = k_resident<DT, ACT, LAYOUT, CPT, MODE>;
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1353,30 +1640,42 @@ cudaError_t launch_resident_one(const ResArgs& a, int smem_optin, cudaStream_t s
     return e;
 }
 
-template <int DT, int LAYOUT, int CPT, int DIR>
+template <int DT, int LAYOUT, int CPT, int MODE>
 cudaError_t launch_resident_act(const ResArgs& a, int act, int smem_optin, cudaStream_t s) {
     switch (act) {
-    case kLeaky: return launch_resident_one<DT, kLeaky, LAYOUT, CPT, DIR>(a, smem_optin, s);
-    case kElu: return launch_resident_one<DT, kElu, LAYOUT, CPT, DIR>(a, smem_optin, s);
-    default: return launch_resident_one<DT, kIdent, LAYOUT, CPT, DIR>(a, smem_optin, s);
+    case kLeaky: return launch_resident_one<DT, kLeaky, LAYOUT, CPT, MODE>(a, smem_optin, s);
+    case kElu: return launch_resident_one<DT, kElu, LAYOUT, CPT, MODE>(a, smem_optin, s);
+    default: return launch_resident_one<DT, kIdent, LAYOUT, CPT, MODE>(a, smem_optin, s);
     }
 }
 
-template <int DT, int DIR>
-cudaError_t launch_resident_dir(const ResArgs& a, int layout, int cpt, int act, int smem_optin,
-                                cudaStream_t s) {
-    if (layout == kNCHW) return launch_resident_act<DT, kNCHW, 1, DIR>(a, act, smem_optin, s);
-    if (cpt == 1) return launch_resident_act<DT, kNHWC, 1, DIR>(a, act, smem_optin, s);
-    if (cpt == 2) return launch_resident_act<DT, kNHWC, 2, DIR>(a, act, smem_optin, s);
-    return launch_resident_act<DT, kNHWC, 4, DIR>(a, act, smem_optin, s);
+// The in-place layer's modes take every resident shape; the standard
+// backward and the checkpointing modes only one 16-byte column per thread
+// (make_plan declines the rest).
+template <int DT, int MODE>
+cudaError_t launch_resident_mode(const ResArgs& a, int layout, int cpt, int act, int smem_optin,
+                                 cudaStream_t s) {
+    if (layout == kNCHW) return launch_resident_act<DT, kNCHW, 1, MODE>(a, act, smem_optin, s);
+    if (cpt == 1) return launch_resident_act<DT, kNHWC, 1, MODE>(a, act, smem_optin, s);
+    if constexpr (MODE == kModeFwd || MODE == kModeBwdZ) {
+        if (cpt == 2) return launch_resident_act<DT, kNHWC, 2, MODE>(a, act, smem_optin, s);
+        return launch_resident_act<DT, kNHWC, 4, MODE>(a, act, smem_optin, s);
+    } else {
+        return cudaErrorNotSupported;
+    }
 }
 
-// Defined in iabn_resident_{f32,bf16,f16}.cu.
-cudaError_t launch_resident_f32(const ResArgs& a, int layout, int cpt, int act, int dir,
-                                int smem_optin, cudaStream_t s);
-cudaError_t launch_resident_bf16(const ResArgs& a, int layout, int cpt, int act, int dir,
-                                 int smem_optin, cudaStream_t s);
-cudaError_t launch_resident_f16(const ResArgs& a, int layout, int cpt, int act, int dir,
-                                int smem_optin, cudaStream_t s);
+// Defined in iabn_resident_{f32,bf16,f16}_{fwd,bwd}.cu (forward modes /
+// backward modes).
+#define IABN_RESIDENT_DECL(NAME)                                                              \
+    cudaError_t NAME(const ResArgs& a, int layout, int cpt, int act, int mode, int smem_optin, \
+                     cudaStream_t s);
+IABN_RESIDENT_DECL(launch_resident_f32_fwd)
+IABN_RESIDENT_DECL(launch_resident_f32_bwd)
+IABN_RESIDENT_DECL(launch_resident_bf16_fwd)
+IABN_RESIDENT_DECL(launch_resident_bf16_bwd)
+IABN_RESIDENT_DECL(launch_resident_f16_fwd)
+IABN_RESIDENT_DECL(launch_resident_f16_bwd)
+#undef IABN_RESIDENT_DECL
 
 }  // namespace iabn

@@ -168,172 +168,63 @@ k_tp_finalize_fwd(const double2* __restrict__ part, int layout, int64_t C, int64
             save_mean[c] = (float)mean;
             save_var[c] = (float)var;
             const double rstd = 1.0 / sqrt(var + (double)eps);
-            coef[c] = make_float4((float)mean, (float)((double)gamma[c] * rstd), beta[c], 0.f);
+            const double sc = (double)gamma[c] * rstd;
+            // (mean, scale, beta, beta - mean*scale); second record: rstd (the
+            // checkpointing forward's xhat)
+            coef[c] = make_float4((float)mean, (float)sc, beta[c], (float)((double)beta[c] - mean * sc));
+            coef[C + c] = make_float4((float)rstd, 0.f, 0.f, 0.f);
         }
-    }
-}
-
-// Flat grid-stride apply; the channel of element i is tracked incrementally
-// (NHWC: i mod C; NCHW: (i div HW) mod C) so the loop has no division.
-template <int LAYOUT>
-struct ChannelWalker {
-    int64_t c, rem, sc, sr, sq, C, HW;
-    __device__ __forceinline__ void init(int64_t i, int64_t stride, int64_t C_, int64_t HW_) {
-        C = C_; HW = HW_;
-        if (LAYOUT == kNHWC) {
-            c = i % C; sc = stride % C;
-        } else {
-            rem = i % HW; c = (i / HW) % C; sr = stride % HW; sq = (stride / HW) % C;
-        }
-    }
-    __device__ __forceinline__ void advance() {
-        if (LAYOUT == kNHWC) {
-            c += sc;
-            if (c >= C) c -= C;
-        } else {
-            rem += sr;
-            int64_t carry = 0;
-            if (rem >= HW) { rem -= HW; carry = 1; }
-            c += sq + carry;
-            if (c >= C) c -= C;
-        }
-    }
-};
-
-template <int DT, int ACT, int LAYOUT>
-__global__ void __launch_bounds__(256)
-k_tp_apply_fwd(typename Storage<DT>::T* __restrict__ x, int64_t E, int64_t C, int64_t HW,
-               const float4* __restrict__ coef, float p) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= E) return;
-    ChannelWalker<LAYOUT> w;
-    w.init(i, stride, C, HW);
-    for (; i < E; i += stride) {
-        const float4 k = __ldg(coef + w.c);
-        const float v = Storage<DT>::load(x + i);
-        const float y = fmaf(v - k.x, k.y, k.z);
-        Storage<DT>::store(x + i, act_forward<ACT, DT>(y, p));
-        w.advance();
-    }
-}
-
-// Channel of a flat element index, moved without division: by one element
-// (step) or by the grid-stride loop's fixed stride (jump).  NHWC: c = i mod C;
-// NCHW: rem = i mod HW, c = (i div HW) mod C.
-struct ChannelPos {
-    int64_t c, rem;
-};
-
-template <int LAYOUT>
-struct ChannelStride {
-    int64_t C, HW, sc, sr, sq;
-    __device__ __forceinline__ void setup(int64_t stride, int64_t C_, int64_t HW_) {
-        C = C_;
-        HW = HW_;
-        sc = stride % C;
-        sr = stride % HW;
-        sq = (stride / HW) % C;
-    }
-    __device__ __forceinline__ ChannelPos at(int64_t i) const {
-        ChannelPos q;
-        if (LAYOUT == kNHWC) {
-            q.c = i % C;
-            q.rem = 0;
-        } else {
-            q.rem = i % HW;
-            q.c = (i / HW) % C;
-        }
-        return q;
-    }
-    __device__ __forceinline__ void jump(ChannelPos& q) const {
-        if (LAYOUT == kNHWC) {
-            q.c += sc;
-            if (q.c >= C) q.c -= C;
-        } else {
-            q.rem += sr;
-            int64_t carry = 0;
-            if (q.rem >= HW) {
-                q.rem -= HW;
-                carry = 1;
-            }
-            q.c += sq + carry;   // < 2C
-            if (q.c >= C) q.c -= C;
-        }
-    }
-    __device__ __forceinline__ void step(ChannelPos& q) const {
-        if (LAYOUT == kNHWC) {
-            if (++q.c == C) q.c = 0;
-        } else if (++q.rem == HW) {
-            q.rem = 0;
-            if (++q.c == C) q.c = 0;
-        }
-    }
-};
-
-// NCHW elementwise passes over 16-byte vectors (the tensors start on a
-// 16-byte boundary): thread t takes vectors t, t + nt, t + 2nt, ... two at a
-// time, both loaded before either is used; the last E mod VE elements go one
-// per thread to the first threads of the grid.  The eight (or four) values of
-// a vector lie in one or two planes, so the lanes of a warp read the
-// coefficients of a few neighbouring channels.  In NHWC they would read eight
-// channels each, 128 bytes apart across the lanes (one L1 wavefront per
-// element), so NHWC keeps the scalar pass above, whose lanes read
-// consecutive channels.
-template <int DT, int ACT, int LAYOUT>
-__global__ void __launch_bounds__(256)
-k_tp_apply_fwd_vec(typename Storage<DT>::T* __restrict__ x, int64_t E, int64_t C,
-                   int64_t HW, const float4* __restrict__ coef, float p) {
-    constexpr int VE = Vec<DT>::N;
-    const int64_t NV = E / VE;
-    const int64_t nt = (int64_t)gridDim.x * blockDim.x;
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    uint4* xv = reinterpret_cast<uint4*>(x);
-    ChannelStride<LAYOUT> cs;
-    cs.setup(2 * nt * VE, C, HW);
-    auto apply = [&](uint4& u, ChannelPos q) {
-        float f[VE];
-        Vec<DT>::unpack(u, f);
-#pragma unroll
-        for (int k = 0; k < VE; ++k) {
-            const float4 kk = __ldg(coef + q.c);
-            f[k] = act_forward<ACT, DT>(fmaf(f[k] - kk.x, kk.y, kk.z), p);
-            cs.step(q);
-        }
-        u = Vec<DT>::pack(f);
-    };
-    ChannelPos q0 = cs.at(t * VE), q1 = cs.at((t + nt) * VE);
-    for (int64_t v = t; v < NV; v += 2 * nt) {
-        const bool two = v + nt < NV;
-        uint4 a = xv[v];
-        uint4 b = two ? xv[v + nt] : make_uint4(0u, 0u, 0u, 0u);
-        apply(a, q0);
-        xv[v] = a;
-        if (two) {
-            apply(b, q1);
-            xv[v + nt] = b;
-        }
-        cs.jump(q0);
-        cs.jump(q1);
-    }
-    const int64_t i = NV * VE + t;
-    if (i < E) {
-        const float4 kk = __ldg(coef + cs.at(i).c);
-        const float xi = Storage<DT>::load(x + i);
-        Storage<DT>::store(x + i, act_forward<ACT, DT>(fmaf(xi - kk.x, kk.y, kk.z), p));
     }
 }
 
 // --------------------------------------------------------------- backward
 
-// Per-channel sums S1 = sum dy and S2 = sum dy*xhat, xhat = (y - beta)/gamma
-// recovered from z.  Same partition and merge order as the statistics.
-template <int DT, int ACT>
+// Per-channel inputs of the backward reductions.
+struct BwdIn {
+    const float* gamma;
+    const float* beta;
+    const float* mean;   // standard backward
+    const float* var;    // standard backward
+    float eps, p, inv_p;
+};
+
+// One channel's view of an element (a, dz) of the backward: dy and xhat.
+//   in-place (from z):       y = phi^-1(z), dy from z, xhat = (y - beta)/gamma
+//   standard / checkpointing: xhat = a*xs + xb, y = a*ys + yb, dy from y
+template <int MODE, int ACT, int DT>
+struct ElemBwd {
+    float ig, nb, xs, xb, ys, yb, p, inv_p;
+    __device__ __forceinline__ void setup(const BwdIn& in, int64_t c) {
+        p = in.p;
+        inv_p = in.inv_p;
+        if (MODE == kModeBwdZ) {
+            ig = 1.f / in.gamma[c];
+            nb = -in.beta[c] * ig;
+        } else {
+            src_affine<MODE>(in.gamma[c], in.beta[c], MODE == kModeBwdX ? in.mean[c] : 0.f,
+                             MODE == kModeBwdX ? in.var[c] : 1.f, in.eps, xs, xb, ys, yb);
+        }
+    }
+    __device__ __forceinline__ void eval(float a, float dz, float& xh, float& dy) const {
+        if (MODE == kModeBwdZ) {
+            float y;
+            act_backward<ACT, DT>(a, dz, p, inv_p, y, dy);
+            xh = fmaf(y, ig, nb);
+        } else {
+            xh = MODE == kModeBwdX ? fmaf(a, xs, xb) : a;
+            dy = act_dy_from_y<ACT, DT>(fmaf(a, ys, yb), dz, p);
+        }
+    }
+};
+
+// Per-channel sums S1 = sum dy and S2 = sum dy*xhat, with xhat recovered from
+// the stored value (ElemBwd).  Same partition and merge order as the
+// statistics.
+template <int DT, int ACT, int MODE>
 __global__ void __launch_bounds__(kTpRowThreads, 2)
 k_tp_reduce_nhwc(const typename Storage<DT>::T* __restrict__ z,
                  const typename Storage<DT>::T* __restrict__ dz, int64_t R, int64_t C, int RB,
-                 const float* __restrict__ gamma, const float* __restrict__ beta, float p,
-                 float inv_p, double2* __restrict__ part) {
+                 const BwdIn in, double2* __restrict__ part) {
     const int W = C < 256 ? (int)C : 256;
     const int RP = kTpRowThreads / W;
     const int t = threadIdx.x;
@@ -343,13 +234,13 @@ k_tp_reduce_nhwc(const typename Storage<DT>::T* __restrict__ z,
     const int64_t r0 = rb * R / RB, r1 = (rb + 1) * R / RB;
     float s1 = 0.f, s2 = 0.f;
     if (phase < RP && col < C) {
-        const float ig = 1.f / gamma[col];
-        const float nb = -beta[col] * ig;
+        ElemBwd<MODE, ACT, DT> eb;
+        eb.setup(in, col);
         auto add = [&](float zv, float dzv) {
-            float y, dy;
-            act_backward<ACT, DT>(zv, dzv, p, inv_p, y, dy);
+            float xh, dy;
+            eb.eval(zv, dzv, xh, dy);
             s1 += dy;
-            s2 = fmaf(dy, fmaf(y, ig, nb), s2);
+            s2 = fmaf(dy, xh, s2);
         };
         int64_t r = r0 + phase;
         for (; r + (kTpBatch - 1) * (int64_t)RP < r1; r += kTpBatch * (int64_t)RP) {
@@ -382,25 +273,23 @@ k_tp_reduce_nhwc(const typename Storage<DT>::T* __restrict__ z,
     if (phase == 0 && col < C) part[rb * C + col] = make_double2(a[t], b[t]);
 }
 
-template <int DT, int ACT>
+template <int DT, int ACT, int MODE>
 __global__ void __launch_bounds__(256)
 k_tp_reduce_nchw(const typename Storage<DT>::T* __restrict__ z,
                  const typename Storage<DT>::T* __restrict__ dz, int64_t planes, int64_t C,
-                 int64_t HW, const float* __restrict__ gamma, const float* __restrict__ beta,
-                 float p, float inv_p, double2* __restrict__ part) {
+                 int64_t HW, const BwdIn in, double2* __restrict__ part) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t pl = gw; pl < planes; pl += nw) {
-        const int64_t c = pl % C;
-        const float ig = 1.f / gamma[c];
-        const float nb = -beta[c] * ig;
+        ElemBwd<MODE, ACT, DT> eb;
+        eb.setup(in, pl % C);
         float s1 = 0.f, s2 = 0.f;
         auto add = [&](float zv, float dzv) {
-            float y, dy;
-            act_backward<ACT, DT>(zv, dzv, p, inv_p, y, dy);
+            float xh, dy;
+            eb.eval(zv, dzv, xh, dy);
             s1 += dy;
-            s2 = fmaf(dy, fmaf(y, ig, nb), s2);
+            s2 = fmaf(dy, xh, s2);
         };
         const typename Storage<DT>::T* zp = z + pl * HW;
         const typename Storage<DT>::T* dzp = dz + pl * HW;
@@ -432,16 +321,19 @@ k_tp_reduce_nchw(const typename Storage<DT>::T* __restrict__ z,
     }
 }
 
-// One warp per channel: S1, S2 summed in fp64; dbeta = S1, dgamma = S2; the
-// apply coefficients express dx in terms of y (the "INPLACE-ABN II" form):
-//   dx = A*dy + B*y + Cc,  A = gamma*rstd,  B = -rstd*S2/M,
-//   Cc = -gamma*rstd*S1/M - B*beta.
+// One warp per channel: S1 = sum dy and S2 = sum dy*xhat summed in fp64;
+// dbeta = S1, dgamma = S2.  The apply coefficients:
+//   in-place: dx in terms of y (the "INPLACE-ABN II" form), one record
+//     dx = A*dy + B*y + Cc,  A = gamma*rstd,  B = -rstd*S2/M,
+//     Cc = -gamma*rstd*S1/M - B*beta;
+//   standard / checkpointing: dx = A dy + B xhat + Cc (B = -A S2/M,
+//     Cc = -A S1/M) applied to the stored value a, xhat = a*xs + xb:
+//     record 0 (ys, yb, A), record 1 (B xs, B xb + Cc).
+template <int MODE>
 __global__ void __launch_bounds__(256)
 k_tp_finalize_bwd(const double2* __restrict__ part, int64_t C, int64_t K, double M,
-                  const float* __restrict__ gamma, const float* __restrict__ beta,
-                  const float* __restrict__ save_var, float eps, float* __restrict__ dgamma,
-                  float* __restrict__ dbeta, float4* __restrict__ coef,
-                  Control* __restrict__ ctl) {
+                  const BwdIn in, float* __restrict__ dgamma, float* __restrict__ dbeta,
+                  float4* __restrict__ coef, Control* __restrict__ ctl) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -454,27 +346,50 @@ k_tp_finalize_bwd(const double2* __restrict__ part, int64_t C, int64_t K, double
         }
         s1 = warp_sum(s1);
         s2 = warp_sum(s2);
-        if (lane == 0) {
-            const double g = gamma[c], b = beta[c];
-            const double rstd = 1.0 / sqrt((double)save_var[c] + (double)eps);
-            if (!(fabs(g) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN (or NaN)
-                atomicOr(&ctl->status, kStSingular);
-                dgamma[c] = __int_as_float(0x7fc00000);
-                dbeta[c] = __int_as_float(0x7fc00000);
-                coef[c] = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
-                                      __int_as_float(0x7fc00000), 0.f);
-            } else {
-                dbeta[c] = (float)s1;
-                dgamma[c] = (float)s2;
-                const double A = g * rstd, B = -rstd * s2 / M;
-                const double Cc = -g * rstd * s1 / M - B * b;
-                coef[c] = make_float4((float)A, (float)B, (float)Cc, 0.f);
-            }
+        if (lane != 0) continue;
+        const double g = in.gamma[c], b = in.beta[c];
+        const double rstd = 1.0 / sqrt((double)in.var[c] + (double)in.eps);
+        if (MODE != kModeBwdZ) {
+            float xs, xb, ys, yb;
+            src_affine<MODE>(in.gamma[c], in.beta[c], MODE == kModeBwdX ? in.mean[c] : 0.f,
+                             in.var[c], in.eps, xs, xb, ys, yb);
+            const double A = g * rstd, B = -A * s2 / M, Cc = -A * s1 / M;
+            dbeta[c] = (float)s1;
+            dgamma[c] = (float)s2;
+            coef[c] = make_float4(ys, yb, (float)A, 0.f);
+            coef[C + c] = make_float4((float)(B * (double)xs), (float)(B * (double)xb + Cc), 0.f, 0.f);
+        } else if (!(fabs(g) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN (or NaN)
+            atomicOr(&ctl->status, kStSingular);
+            dgamma[c] = __int_as_float(0x7fc00000);
+            dbeta[c] = __int_as_float(0x7fc00000);
+            coef[c] = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                  __int_as_float(0x7fc00000), 0.f);
+        } else {
+            dbeta[c] = (float)s1;
+            dgamma[c] = (float)s2;
+            const double A = g * rstd, B = -rstd * s2 / M;
+            const double Cc = -g * rstd * s1 / M - B * b;
+            coef[c] = make_float4((float)A, (float)B, (float)Cc, 0.f);
         }
     }
 }
 
-template <int DT, int ACT, int LAYOUT>
+// dx of one element (a, dz) of channel c from the finalize's record(s).
+template <int MODE, int ACT, int DT>
+__device__ __forceinline__ float bwd_apply_elem(float a, float dz, const float4* __restrict__ coef,
+                                                int64_t C, int64_t c, float p, float inv_p) {
+    const float4 k = __ldg(coef + c);
+    if (MODE == kModeBwdZ) {
+        float y, dy;
+        act_backward<ACT, DT>(a, dz, p, inv_p, y, dy);
+        return fmaf(k.x, dy, fmaf(k.y, y, k.z));
+    }
+    const float4 k2 = __ldg(coef + C + c);
+    const float dy = act_dy_from_y<ACT, DT>(fmaf(a, k.x, k.y), dz, p);
+    return fmaf(k.z, dy, fmaf(k2.x, a, k2.y));
+}
+
+template <int DT, int ACT, int LAYOUT, int MODE>
 __global__ void __launch_bounds__(256)
 k_tp_apply_bwd(const typename Storage<DT>::T* __restrict__ z, typename Storage<DT>::T* dz,
                int64_t E, int64_t C, int64_t HW, const float4* __restrict__ coef, float p,
@@ -485,16 +400,14 @@ k_tp_apply_bwd(const typename Storage<DT>::T* __restrict__ z, typename Storage<D
     ChannelWalker<LAYOUT> w;
     w.init(i, stride, C, HW);
     for (; i < E; i += stride) {
-        const float4 k = __ldg(coef + w.c);
-        float y, dy;
-        act_backward<ACT, DT>(Storage<DT>::load(z + i), Storage<DT>::load(dz + i), p, inv_p, y,
-                              dy);
-        Storage<DT>::store(dz + i, fmaf(k.x, dy, fmaf(k.y, y, k.z)));
+        Storage<DT>::store(dz + i, bwd_apply_elem<MODE, ACT, DT>(Storage<DT>::load(z + i),
+                                                                 Storage<DT>::load(dz + i), coef,
+                                                                 C, w.c, p, inv_p));
         w.advance();
     }
 }
 
-template <int DT, int ACT, int LAYOUT>
+template <int DT, int ACT, int LAYOUT, int MODE>
 __global__ void __launch_bounds__(256)
 k_tp_apply_bwd_vec(const typename Storage<DT>::T* __restrict__ z,
                    typename Storage<DT>::T* dz, int64_t E, int64_t C, int64_t HW,
@@ -513,10 +426,7 @@ k_tp_apply_bwd_vec(const typename Storage<DT>::T* __restrict__ z,
         Vec<DT>::unpack(ud, fd);
 #pragma unroll
         for (int k = 0; k < VE; ++k) {
-            const float4 kk = __ldg(coef + q.c);
-            float y, dy;
-            act_backward<ACT, DT>(fz[k], fd[k], p, inv_p, y, dy);
-            fd[k] = fmaf(kk.x, dy, fmaf(kk.y, y, kk.z));
+            fd[k] = bwd_apply_elem<MODE, ACT, DT>(fz[k], fd[k], coef, C, q.c, p, inv_p);
             cs.step(q);
         }
         ud = Vec<DT>::pack(fd);
@@ -539,29 +449,10 @@ k_tp_apply_bwd_vec(const typename Storage<DT>::T* __restrict__ z,
         cs.jump(q1);
     }
     const int64_t i = NV * VE + t;
-    if (i < E) {
-        const float4 kk = __ldg(coef + cs.at(i).c);
-        float y, dy;
-        act_backward<ACT, DT>(Storage<DT>::load(z + i), Storage<DT>::load(dz + i), p, inv_p, y,
-                              dy);
-        Storage<DT>::store(dz + i, fmaf(kk.x, dy, fmaf(kk.y, y, kk.z)));
-    }
-}
-
-// ------------------------------------------------------------ inference
-
-// Evaluation mode ([BN] Algorithm 2, the inference network): the running
-// averages stand in for the batch statistics.  The coefficients take the
-// training forward's form (mean, gamma*rstd, beta), so the forward's
-// elementwise pass applies them unchanged.
-__global__ void k_eval_coef(int64_t C, const float* __restrict__ gamma,
-                            const float* __restrict__ beta, const float* __restrict__ rmean,
-                            const float* __restrict__ rvar, float eps,
-                            float4* __restrict__ coef) {
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= C) return;
-    const double rstd = 1.0 / sqrt((double)rvar[c] + (double)eps);
-    coef[c] = make_float4(rmean[c], (float)((double)gamma[c] * rstd), beta[c], 0.f);
+    if (i < E)
+        Storage<DT>::store(dz + i, bwd_apply_elem<MODE, ACT, DT>(Storage<DT>::load(z + i),
+                                                                 Storage<DT>::load(dz + i), coef,
+                                                                 C, cs.at(i).c, p, inv_p));
 }
 
 // ------------------------------------------------------------ running stats
@@ -606,23 +497,6 @@ static int apply_grid(const Geom& g, int sms, int per_sm) {
     return grid_for(nv, 2 * 256, sms * per_sm);
 }
 
-template <int DT, int ACT, int LAYOUT>
-static cudaError_t fwd_apply(const Geom& g, void* x, const float4* coef, float p,
-                             cudaStream_t s, int sms) {
-    using T = typename Storage<DT>::T;
-    if (LAYOUT == kNHWC) {
-        k_tp_apply_fwd<DT, ACT, kNHWC><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
-            static_cast<T*>(x), g.E, g.C, g.HW, coef, p);
-    } else {
-        static std::atomic<int> occ{0};
-        auto kern = k_tp_apply_fwd_vec<DT, ACT, kNCHW>;
-        kern<<<apply_grid(g, sms, ctas_per_sm(kern, 256, occ)), 256, 0, s>>>(
-            static_cast<T*>(x), g.E, g.C, g.HW, coef, p);
-    }
-    count_launches(1);
-    return cudaGetLastError();
-}
-
 template <int DT>
 static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Workspace& w,
                                    cudaStream_t s, int sms) {
@@ -654,20 +528,8 @@ static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Worksp
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    void* xm = a.x;
-    const float p = a.act_param;
-    if (g.layout == kNHWC) {
-        switch (a.act) {
-        case kLeaky: return fwd_apply<DT, kLeaky, kNHWC>(g, xm, w.coef, p, s, sms);
-        case kElu: return fwd_apply<DT, kElu, kNHWC>(g, xm, w.coef, p, s, sms);
-        default: return fwd_apply<DT, kIdent, kNHWC>(g, xm, w.coef, p, s, sms);
-        }
-    }
-    switch (a.act) {
-    case kLeaky: return fwd_apply<DT, kLeaky, kNCHW>(g, xm, w.coef, p, s, sms);
-    case kElu: return fwd_apply<DT, kElu, kNCHW>(g, xm, w.coef, p, s, sms);
-    default: return fwd_apply<DT, kIdent, kNCHW>(g, xm, w.coef, p, s, sms);
-    }
+    // the elementwise pass with fixed channels per thread (iabn_elementwise.cu)
+    return forward_apply_pass(g, a, w.coef, s, sms);
 }
 
 cudaError_t forward_twophase(const Geom& g, const FwdArgs& a, const Workspace& w,
@@ -679,51 +541,61 @@ cudaError_t forward_twophase(const Geom& g, const FwdArgs& a, const Workspace& w
     }
 }
 
-template <int DT, int ACT>
-static cudaError_t bwd_twophase_act(const Geom& g, const BwdArgs& a, const Workspace& w,
-                                    cudaStream_t s, int sms) {
+template <int DT, int ACT, int MODE>
+static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Workspace& w,
+                                     cudaStream_t s, int sms) {
     using T = typename Storage<DT>::T;
-    const T* z = static_cast<const T*>(a.z);
+    const T* z = static_cast<const T*>(a.src);
     T* dz = static_cast<T*>(a.dz);
     const float p = a.act_param;
     const float inv_p = ACT == kIdent ? 1.f : 1.f / p;
+    const BwdIn in{a.gamma, a.beta, a.save_mean, a.save_var, a.eps, p, inv_p};
     int64_t K;
     if (g.layout == kNHWC) {
         const int RB = nhwc_row_blocks(g.R);
         const int W = g.C < 256 ? (int)g.C : 256;
         dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
-        k_tp_reduce_nhwc<DT, ACT><<<grid, kTpRowThreads, 0, s>>>(z, dz, g.R, g.C, RB, a.gamma,
-                                                                 a.beta, p, inv_p, w.part);
+        k_tp_reduce_nhwc<DT, ACT, MODE><<<grid, kTpRowThreads, 0, s>>>(z, dz, g.R, g.C, RB, in,
+                                                                       w.part);
         K = RB;
         count_launches(1);
     } else {
         const int64_t planes = g.N * g.C;
         static std::atomic<int> occ{0};
-        const int per_sm = ctas_per_sm(k_tp_reduce_nchw<DT, ACT>, 256, occ);
-        k_tp_reduce_nchw<DT, ACT><<<grid_for(planes, 8, sms * per_sm), 256, 0, s>>>(
-            z, dz, planes, g.C, g.HW, a.gamma, a.beta, p, inv_p, w.part);
+        const int per_sm = ctas_per_sm(k_tp_reduce_nchw<DT, ACT, MODE>, 256, occ);
+        k_tp_reduce_nchw<DT, ACT, MODE><<<grid_for(planes, 8, sms * per_sm), 256, 0, s>>>(
+            z, dz, planes, g.C, g.HW, in, w.part);
         K = g.N;
         count_launches(1);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_tp_finalize_bwd<<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
-        w.part, g.C, K, (double)g.M, a.gamma, a.beta, a.save_var, a.eps, a.dgamma, a.dbeta,
-        w.coef, w.ctl);
+    k_tp_finalize_bwd<MODE><<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
+        w.part, g.C, K, (double)g.M, in, a.dgamma, a.dbeta, w.coef, w.ctl);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (g.layout == kNHWC) {
-        k_tp_apply_bwd<DT, ACT, kNHWC><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
+        k_tp_apply_bwd<DT, ACT, kNHWC, MODE><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
             z, dz, g.E, g.C, g.HW, w.coef, p, inv_p);
     } else {
         static std::atomic<int> occ{0};
-        auto kern = k_tp_apply_bwd_vec<DT, ACT, kNCHW>;
+        auto kern = k_tp_apply_bwd_vec<DT, ACT, kNCHW, MODE>;
         kern<<<apply_grid(g, sms, ctas_per_sm(kern, 256, occ)), 256, 0, s>>>(
             z, dz, g.E, g.C, g.HW, w.coef, p, inv_p);
     }
     count_launches(1);
     return cudaGetLastError();
+}
+
+template <int DT, int ACT>
+static cudaError_t bwd_twophase_act(const Geom& g, const BwdArgs& a, const Workspace& w,
+                                    cudaStream_t s, int sms) {
+    switch (a.mode) {
+    case kModeBwdX: return bwd_twophase_mode<DT, ACT, kModeBwdX>(g, a, w, s, sms);
+    case kModeBwdXhat: return bwd_twophase_mode<DT, ACT, kModeBwdXhat>(g, a, w, s, sms);
+    default: return bwd_twophase_mode<DT, ACT, kModeBwdZ>(g, a, w, s, sms);
+    }
 }
 
 template <int DT>
@@ -742,39 +614,6 @@ cudaError_t backward_twophase(const Geom& g, const BwdArgs& a, const Workspace& 
     case kF32: return bwd_twophase_dt<kF32>(g, a, w, s, sms);
     case kBF16: return bwd_twophase_dt<kBF16>(g, a, w, s, sms);
     default: return bwd_twophase_dt<kF16>(g, a, w, s, sms);
-    }
-}
-
-template <int DT>
-static cudaError_t inference_dt(const Geom& g, const InfArgs& a, const float4* coef,
-                                cudaStream_t s, int sms) {
-    void* x = a.x;
-    const float p = a.act_param;
-    if (g.layout == kNHWC) {
-        switch (a.act) {
-        case kLeaky: return fwd_apply<DT, kLeaky, kNHWC>(g, x, coef, p, s, sms);
-        case kElu: return fwd_apply<DT, kElu, kNHWC>(g, x, coef, p, s, sms);
-        default: return fwd_apply<DT, kIdent, kNHWC>(g, x, coef, p, s, sms);
-        }
-    }
-    switch (a.act) {
-    case kLeaky: return fwd_apply<DT, kLeaky, kNCHW>(g, x, coef, p, s, sms);
-    case kElu: return fwd_apply<DT, kElu, kNCHW>(g, x, coef, p, s, sms);
-    default: return fwd_apply<DT, kIdent, kNCHW>(g, x, coef, p, s, sms);
-    }
-}
-
-cudaError_t inference_twophase(const Geom& g, const InfArgs& a, const Workspace& w,
-                               cudaStream_t s, int sms) {
-    k_eval_coef<<<(unsigned)((g.C + 255) / 256), 256, 0, s>>>(
-        g.C, a.gamma, a.beta, a.running_mean, a.running_var, a.eps, w.coef);
-    count_launches(1);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    switch (g.dtype) {
-    case kF32: return inference_dt<kF32>(g, a, w.coef, s, sms);
-    case kBF16: return inference_dt<kBF16>(g, a, w.coef, s, sms);
-    default: return inference_dt<kF16>(g, a, w.coef, s, sms);
     }
 }
 

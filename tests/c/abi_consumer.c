@@ -44,6 +44,13 @@ int main(void) {
     print_plan("trunk_bwd", &info);
     printf("describe_many_status %d\n", (int)iabn_describe_plan(&many, 0, 148, 232448, &info));
     print_plan("many_fwd", &info);
+    printf("describe_std_bwd_status %d\n",
+           (int)iabn_describe_plan(&trunk, IABN_CALL_BACKWARD_STANDARD, 148, 232448, &info));
+    print_plan("trunk_std_bwd", &info);
+    printf("describe_ckpt_fwd_status %d\n",
+           (int)iabn_describe_plan(&trunk, IABN_CALL_FORWARD_CHECKPOINT, 148, 232448, &info));
+    print_plan("trunk_ckpt_fwd", &info);
+    printf("describe_bad_call %d\n", (int)iabn_describe_plan(&trunk, 6, 148, 232448, &info));
     /* rejected on the host before any CUDA call */
     printf("forward_null_x %d\n",
            (int)iabn_forward(&trunk, NULL, dummy, dummy, 1e-5f, IABN_ACT_LEAKY_RELU, 0.01f,
@@ -54,6 +61,22 @@ int main(void) {
     printf("inference_bad_act %d\n",
            (int)iabn_inference(&trunk, dummy, dummy, dummy, dummy, dummy, 1e-5f, 9, 0.01f,
                                NULL, 0, NULL));
+    printf("forward_standard_null_z %d\n",
+           (int)iabn_forward_standard(&trunk, dummy, NULL, dummy, dummy, 1e-5f,
+                                      IABN_ACT_LEAKY_RELU, 0.01f, dummy, dummy, NULL, 0, NULL));
+    printf("backward_standard_null_mean %d\n",
+           (int)iabn_backward_standard(&trunk, dummy, dummy + 2, dummy, dummy, NULL, dummy, 1e-5f,
+                                       IABN_ACT_LEAKY_RELU, 0.01f, dummy, dummy, NULL, 0, NULL));
+    printf("forward_checkpoint_bad_eps %d\n",
+           (int)iabn_forward_checkpoint(&trunk, dummy, dummy, dummy, dummy, -1.f,
+                                        IABN_ACT_LEAKY_RELU, 0.01f, dummy, dummy, NULL, 0, NULL));
+    printf("backward_checkpoint_bad_desc %d\n",
+           (int)iabn_backward_checkpoint(&bad, dummy, dummy, dummy, dummy, dummy, 1e-5f,
+                                         IABN_ACT_LEAKY_RELU, 0.01f, dummy, dummy, NULL, 0,
+                                         NULL));
+    printf("recompute_null_xhat %d\n",
+           (int)iabn_checkpoint_recompute(&trunk, NULL, dummy, dummy, dummy,
+                                          IABN_ACT_LEAKY_RELU, 0.01f, NULL));
     printf("running_bad_count %d\n",
            (int)iabn_update_running_stats(256, 1, dummy, dummy, dummy, dummy, 0.1f, NULL));
     printf("status_null_ws %d\n", (int)iabn_get_device_status(NULL, NULL));

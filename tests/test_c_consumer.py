@@ -46,14 +46,24 @@ def test_c_consumer_matches_the_binding(tmp_path, compiler, flags, monkeypatch):
     for tag, shape, layout, dtype, direction in (
             ("trunk_fwd", (64, 256, 56, 56), iabn.IABN_NHWC, iabn.IABN_BF16, 0),
             ("trunk_bwd", (64, 256, 56, 56), iabn.IABN_NHWC, iabn.IABN_BF16, 1),
-            ("many_fwd", (128, 2048, 7, 7), iabn.IABN_NCHW, iabn.IABN_F16, 0)):
+            ("many_fwd", (128, 2048, 7, 7), iabn.IABN_NCHW, iabn.IABN_F16, 0),
+            ("trunk_std_bwd", (64, 256, 56, 56), iabn.IABN_NHWC, iabn.IABN_BF16,
+             iabn.IABN_CALL_BACKWARD_STANDARD),
+            ("trunk_ckpt_fwd", (64, 256, 56, 56), iabn.IABN_NHWC, iabn.IABN_BF16,
+             iabn.IABN_CALL_FORWARD_CHECKPOINT)):
         want = iabn.describe_plan(shape, layout, dtype, direction, sm_count=148,
                                   smem_optin=232448)
         want["plan"] = {"twophase": 0, "resident": 1}[want["plan"]]
         for k, v in want.items():
             assert int(got[f"{tag}.{k}"]) == v, (tag, k)
-    for k in ("describe_fwd_status", "describe_bwd_status", "describe_many_status"):
+    for k in ("describe_fwd_status", "describe_bwd_status", "describe_many_status",
+              "describe_std_bwd_status", "describe_ckpt_fwd_status"):
         assert int(got[k]) == iabn.IABN_OK
+    assert int(got["describe_bad_call"]) == iabn.IABN_ERR_INVALID_ARG
+    for k in ("forward_standard_null_z", "backward_standard_null_mean",
+              "forward_checkpoint_bad_eps", "backward_checkpoint_bad_desc",
+              "recompute_null_xhat"):
+        assert int(got[k]) == iabn.IABN_ERR_INVALID_ARG, k
     assert int(got["forward_null_x"]) == iabn.IABN_ERR_INVALID_ARG
     assert int(got["backward_bad_desc"]) == iabn.IABN_ERR_INVALID_ARG
     assert int(got["inference_bad_act"]) == iabn.IABN_ERR_INVALID_ARG

@@ -6,17 +6,22 @@ Forward: z (storage type), batch mean and biased variance.
 Backward (stage-separated): both sides start from the oracle's own rounded z
 and fp32 variance, so a one-ulp rounding flip in the forward is not blamed on
 the backward.  End to end: the GPU forward feeds the GPU backward; the
-oracle's chain feeds the oracle; same tolerance.
-Tolerances: fp32 rel 1e-5 / abs 1e-6; bf16, fp16 rel 2e-2 / abs 1e-2 (dx
-relative to the size of its terms, see gpu_util).
+oracle's chain feeds the oracle.
+Bound |got - want| <= abs + rel*|want|, fp32 rel 1e-5 / abs 1e-6; bf16, fp16
+rel 2e-2 / abs 1e-2, for the forward.  The stage-separated backward adds the
+fp32 rounding noise of the kernel's own summation order (gpu_util); the
+end-to-end outputs take the wider relative scale of gpu_util (one-ulp flips
+of z).  Every comparison's worst ratio under the plain bound is printed at
+the end of the session.
+Every device buffer is guarded against writes past its ends (gpu_util).
 """
 import numpy as np
 import pytest
 
 import oracle
 import workloads as wl
-from gpu_util import PLANS, TOL, GpuLayer, compare, forced_plan, oracle_expect, \
-    oracle_sweep_inputs
+from gpu_util import PLANS, TOL, GpuLayer, backward_noise, compare, forced_plan, \
+    oracle_expect, oracle_sweep_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -65,10 +70,11 @@ def check_layer(inp, exp, plan, *, running=False, e2e=True):
         var32 = torch.from_numpy(exp["var32"].astype(np.float32)).cuda()
         L.backward(z=z, var=var32)
         torch.cuda.synchronize()
-        compare(L.host(L.dz), exp["dx"], sp.dtype, f"{sp.name} dx", exp["dx_scale"])
+        nz = backward_noise(exp, sp)
+        compare(L.host(L.dz), exp["dx"], sp.dtype, f"{sp.name} dx", noise=nz["dx"])
         compare(L.dgamma.cpu().numpy(), exp["dgamma"], tol, f"{sp.name} dgamma",
-                exp["dgamma_scale"])
-        compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} dbeta", exp["dbeta_scale"])
+                noise=nz["dgamma"])
+        compare(L.dbeta.cpu().numpy(), exp["dbeta"], tol, f"{sp.name} dbeta", noise=nz["dbeta"])
         # z is read-only for the backward
         np.testing.assert_array_equal(L.host(L.x), exp["z"])
         assert L.status() == 0
@@ -87,6 +93,29 @@ def test_layer_sweep_parity(plan):
     chained input."""
     for inp, exp in oracle_sweep_inputs():
         check_layer(inp, exp, plan, e2e=False)
+
+
+# fp32 NHWC layers whose per-channel statistics stress the summation: the
+# resident plan's size (64x256x28x28, several tiles per CTA, ragged tile
+# ends) with heavy tails (Student-t, 3 degrees of freedom) or with the
+# first row of every channel 30 sigma away from the channel mean.
+STATS_STRESS = [
+    wl.LayerSpec("f32_nhwc_t3", 64, 256, 28, 28, wl.NHWC, wl.F32, wl.LEAKY_RELU, 0.01,
+                 seed=20180611, x_dist="student_t3"),
+    wl.LayerSpec("f32_nhwc_outlier_row0", 64, 256, 28, 28, wl.NHWC, wl.F32, wl.LEAKY_RELU,
+                 0.01, seed=20180612, first_row_outlier=30.0),
+    wl.LayerSpec("f32_nhwc_outlier_row0_neg", 16, 96, 23, 29, wl.NHWC, wl.F32, wl.ELU, 1.0,
+                 seed=20180613, first_row_outlier=-30.0),
+    wl.LayerSpec("f32_nchw_t3_outlier", 32, 64, 19, 21, wl.NCHW, wl.F32, wl.LEAKY_RELU, 0.01,
+                 seed=20180614, x_dist="student_t3", first_row_outlier=30.0),
+]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("sp", STATS_STRESS, ids=lambda s: s.name)
+def test_statistics_stress(sp, plan):
+    inp = wl.draw(sp)
+    check_layer(inp, oracle_expect(inp), plan, running=True)
 
 
 EDGE = [

@@ -502,3 +502,34 @@ def test_hand_derived_examples():
                                        case["momentum"], case["running_mean"], case["running_var"])
         _close(rm, e["running_mean"], rel=1e-14, abs_=1e-15)
         _close(rv, e["running_var"], rel=1e-14)
+
+
+def test_openmp_build_gives_identical_bits():
+    """The multi-core build of the oracle (same source with -fopenmp) splits
+    only the loops over channels; every result is bit for bit the plain
+    build's."""
+    rng = np.random.default_rng(90)
+    shape = (3, 9, 4, 5)
+    layers = {lay: _rand_layer(rng, shape, lay) for lay in (oracle.NCHW, oracle.NHWC)}
+    out = {}
+    for omp in (False, True):
+        oracle.openmp(omp)
+        try:
+            res = []
+            for layout, (xl, g, b, dzl) in layers.items():
+                x, dz = _flat(xl, layout), _flat(dzl, layout)
+                fw = oracle.forward(shape, layout, x, g, b, 1e-5, oracle.ELU, 1.0, want_xhat_y=True)
+                res += [fw["mean"], fw["var"], fw["z"], fw["xhat"]]
+                res += list(oracle.backward_inplace(shape, layout, fw["z"], dz, g, b, fw["var"],
+                                                    1e-5, oracle.ELU, 1.0).values())
+                res += list(oracle.backward_standard(shape, layout, x, dz, g, b, 1e-5,
+                                                     oracle.ELU, 1.0).values())
+                res += list(oracle.backward_checkpoint(shape, layout, fw["xhat"], dz, g, b,
+                                                       fw["var"], 1e-5, oracle.ELU, 1.0).values())
+                res.append(oracle.round_to(fw["z"], oracle.BF16))
+            out[omp] = res
+        finally:
+            oracle.openmp(False)
+    assert len(out[False]) == len(out[True]) > 0
+    for a, b in zip(out[False], out[True]):
+        np.testing.assert_array_equal(a, b)

@@ -1,7 +1,8 @@
 """The host-side launch planner, through iabn_describe_plan, without a GPU.
 
-The plan decides the launch shape of every call: grid, shared memory, tile
-sizes, the Tensor Memory stash.  A planning error would reach the device as
+The plan decides the launch shape of every call -- the in-place layer's
+forward and backward, the standard layer's and the checkpointing layer's:
+grid, shared memory, tile sizes, the Tensor Memory stash.  A planning error would reach the device as
 an oversized launch or an out-of-range slot, so its invariants are checked
 here on the CPU over a sweep of shapes, at the B200's limits (148 SMs,
 232448 bytes of opt-in shared memory per block) and at smaller ones.  The
@@ -34,23 +35,27 @@ def esize(dtype):
     return 4 if dtype == wl.F32 else 2
 
 
-def qualifies(shape, layout, dtype):
+CALLS = range(6)          # IABN_CALL_*: layer = call // 2, direction = call % 2
+
+
+def qualifies(shape, layout, dtype, call=0):
     """The resident plan's shape rule, restated: NHWC rows of C channels are a
-    multiple of 16 bytes and at most 16 KiB; NCHW units of g whole planes
-    (g = 16 / gcd(16, H*W*s)) start on 16-byte boundaries, N*C is a multiple
-    of g and a unit is at most 32 KiB."""
+    multiple of 16 bytes and at most 16 KiB (at most 4 KiB, one 16-byte
+    column per consumer thread, for the standard and the checkpointing
+    layers); NCHW units of g whole planes (g = 16 / gcd(16, H*W*s)) start on
+    16-byte boundaries, N*C is a multiple of g and a unit is at most 32 KiB."""
     n, c, h, w = shape
     s = esize(dtype)
     if layout == wl.NHWC:
-        return (c * s) % 16 == 0 and c * s <= 16384
+        return (c * s) % 16 == 0 and c * s <= (16384 if call < 2 else 4096)
     g = 16 // math.gcd(h * w * s, 16)
     return (n * c) % g == 0 and g * h * w * s <= 32768
 
 
-def check_resident(info, shape, layout, dtype, direction, sm_count, smem_optin):
+def check_resident(info, shape, layout, dtype, call, sm_count, smem_optin):
     n, c, h, w = shape
     s = esize(dtype)
-    nt = 1 if direction == 0 else 2          # tensors streamed: x; or z and dz
+    nt = 1 if call % 2 == 0 else 2           # tensors streamed: x; or z (x, xhat) and dz
     assert info["launches"] == 1 and info["threads"] == 320
     units = n * h * w if layout == wl.NHWC else n * c // info["planes_per_unit"]
     assert 1 <= info["grid"] <= min(sm_count, 256, units)
@@ -64,6 +69,7 @@ def check_resident(info, shape, layout, dtype, direction, sm_count, smem_optin):
         vc, cpt, rp = info["vectors_per_row"], info["cols_per_thread"], info["row_phases"]
         assert vc * 16 == c * s
         assert cpt in (1, 2, 4) and vc <= 256 * cpt and (cpt == 1 or vc > 256 * cpt // 2)
+        assert cpt == 1 or call < 2
         assert rp == (256 // vc if cpt == 1 else 1)
         assert tb % (c * s) == 0 and (tb // (c * s)) % rp == 0
         assert info["planes_per_unit"] == 0
@@ -107,33 +113,38 @@ def test_plan_invariants_over_shapes(limits, tiles, monkeypatch):
         monkeypatch.setenv("IABN_TILE_KB_BWD", str(tiles[1]))
     seen = {"resident": 0, "twophase": 0}
     for shape, layout, dtype in sweep():
-        for direction in (0, 1):
-            info = iabn.describe_plan(shape, layout, dtype, direction, **limits)
+        for call in CALLS:
+            info = iabn.describe_plan(shape, layout, dtype, call, **limits)
             seen[info["plan"]] += 1
             if info["plan"] == "resident":
-                assert qualifies(shape, layout, dtype), (shape, layout, dtype)
-                check_resident(info, shape, layout, dtype, direction, **limits)
+                assert qualifies(shape, layout, dtype, call), (shape, layout, dtype, call)
+                check_resident(info, shape, layout, dtype, call, **limits)
             else:
                 check_twophase(info)
                 if limits is B200:
                     # at the B200's limits every qualifying shape fits
-                    assert not qualifies(shape, layout, dtype), (shape, layout, dtype)
+                    assert not qualifies(shape, layout, dtype, call), (shape, layout, dtype, call)
     assert seen["resident"] > 0 and seen["twophase"] > 0
 
 
-def test_both_directions_agree_on_the_plan():
+def test_both_calls_of_a_layer_agree_on_the_plan():
     for shape, layout, dtype in sweep():
-        f = iabn.describe_plan(shape, layout, dtype, 0, **B200)
-        b = iabn.describe_plan(shape, layout, dtype, 1, **B200)
-        assert f["plan"] == b["plan"] and f["grid"] == b["grid"]
+        for layer in range(3):
+            f = iabn.describe_plan(shape, layout, dtype, 2 * layer, **B200)
+            b = iabn.describe_plan(shape, layout, dtype, 2 * layer + 1, **B200)
+            assert f["plan"] == b["plan"] and f["grid"] == b["grid"]
 
 
 def test_benchmark_workloads_take_the_resident_plan():
     specs = [wl.spec(i) for i in range(4)] + [wl.spec(4, l) for l in range(16)]
     for sp in specs:
-        for direction in (0, 1):
-            info = iabn.describe_plan(sp.shape, sp.layout, sp.dtype, direction, **B200)
-            assert info["plan"] == "resident", (sp.name, direction)
+        # every call of the in-place layer; the standard and the checkpointing
+        # layers wherever a row is at most 4 KiB (all but the two widest
+        # layers of the sweep)
+        calls = CALLS if sp.layout == wl.NCHW or sp.c * sp.itemsize <= 4096 else (0, 1)
+        for call in calls:
+            info = iabn.describe_plan(sp.shape, sp.layout, sp.dtype, call, **B200)
+            assert info["plan"] == "resident", (sp.name, call)
             if sp.n * sp.h * sp.w >= 148 * 8 or sp.layout == wl.NCHW and sp.n * sp.c >= 148 * 8:
                 assert info["grid"] == 148
     # the ResNet-trunk layer keeps rows in Tensor Memory, filled by the copy engine
@@ -169,7 +180,7 @@ def test_environment_knobs(monkeypatch):
 def test_describe_rejects_bad_arguments():
     d = iabn.make_desc((2, 8, 4, 4), wl.NHWC, wl.BF16)
     info = iabn.IabnPlanInfo()
-    assert iabn.iabn_describe_plan(d, 2, 148, 232448, info) == iabn.IABN_ERR_INVALID_ARG
+    assert iabn.iabn_describe_plan(d, 6, 148, 232448, info) == iabn.IABN_ERR_INVALID_ARG
     assert iabn.iabn_describe_plan(d, -1, 148, 232448, info) == iabn.IABN_ERR_INVALID_ARG
     assert iabn.iabn_describe_plan(d, 0, 148, 0, info) == iabn.IABN_ERR_INVALID_ARG
     assert iabn.iabn_describe_plan(d, 0, -1, 232448, info) == iabn.IABN_ERR_INVALID_ARG

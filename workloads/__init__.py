@@ -18,7 +18,9 @@ e ~ N(0, 1) (Student-t with 3 degrees of freedom for workload 2);
 gamma_c = s_c * U(0.5, 1.5) (U(0.05, 1.5) for workload 3) with s_c = +-1 at
 probability 1/2; beta_c ~ N(0, variance 0.1); dz ~ N(0, 1); eps = 1e-5;
 momentum = 0.1.  Generator: numpy PCG64 with seed 20180600 + workload id
-(+ 100 * layer for the layer sweep).  Values are drawn in fp64 in logical
+(+ 100 * layer for the layer sweep).  A spec may replace the first element
+of every channel, x[0, c, 0, 0], by mu_c + k*sigma_c (an outlier first row, used to
+stress the statistics' summation).  Values are drawn in fp64 in logical
 (n, c, h, w) order, arranged in the workload's layout and rounded to the
 storage type (round to nearest even).
 """
@@ -60,6 +62,7 @@ class LayerSpec:
     act_param: float
     seed: int
     x_dist: str = "normal"          # "normal" or "student_t3"
+    first_row_outlier: float = 0.0  # if nonzero: x[0, c, 0, 0] = mu_c + this * sigma_c
     gamma_lo: float = 0.5
     eps: float = EPS
     momentum: float = MOMENTUM
@@ -204,6 +207,8 @@ def draw(sp: LayerSpec, *, x_logical: np.ndarray | None = None) -> LayerInputs:
             raise ValueError(sp.x_dist)
         x_logical = mu[None, :, None, None] + sigma[None, :, None, None] * e
         del e
+        if sp.first_row_outlier:
+            x_logical[0, :, 0, 0] = mu + sp.first_row_outlier * sigma
     else:
         rng.standard_normal((n, c, h, w))   # keep the dz stream independent of x's source
     dz_logical = rng.standard_normal((n, c, h, w))
