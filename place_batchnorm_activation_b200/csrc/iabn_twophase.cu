@@ -321,6 +321,327 @@ k_tp_reduce_nchw(const typename Storage<DT>::T* __restrict__ z,
     }
 }
 
+// --------------------------------------------- NHWC rows of 16-byte vectors
+// When a row of C channels is a whole number of 16-byte vectors (VC of them),
+// the NHWC passes give every thread one fixed vector column: its VE = 16/s
+// channels' constants stay in registers, every load and store is 16 bytes,
+// and kRowBatch rows are loaded before any of them is used.  Block (rb, cb)
+// owns rows [rb*R/RB, (rb+1)*R/RB) -- the partition the finalize counts -- and
+// the columns [cb*W, cb*W + W); its RPB = threads/W row phases take rows
+// phase, phase + RPB, ...  The reductions run one block of kRowThreads per SM
+// (the partials are per block) with 16 loads in flight per thread; the
+// backward apply runs blocks of kApplyThreads, as many as fit, 8 loads in
+// flight per thread.
+
+constexpr int kRowThreads = 512;
+constexpr int kRowBatch = 8;
+constexpr int kStatsBatch = 16;
+constexpr int kApplyThreads = 256;
+
+template <int THREADS = kRowThreads>
+struct RowTile {
+    int W, RPB, phase;
+    int64_t col, r0, r1;
+    bool active;
+    __device__ __forceinline__ RowTile(int VC, int64_t R, int RB) {
+        W = VC < THREADS ? VC : THREADS;
+        RPB = THREADS / W;
+        phase = (int)threadIdx.x / W;
+        col = (int64_t)blockIdx.y * W + (int)threadIdx.x % W;
+        r0 = (int64_t)blockIdx.x * R / RB;
+        r1 = ((int64_t)blockIdx.x + 1) * R / RB;
+        active = phase < RPB && col < VC;
+    }
+    // rows of this thread in [r0, r1)
+    __device__ __forceinline__ int64_t count() const {
+        const int64_t n = r1 - r0;
+        return active && n > phase ? (n - 1 - phase) / RPB + 1 : 0;
+    }
+};
+
+// Forward statistics: each thread sums x - K and (x - K)^2 in fp32 around its
+// own first value K of each channel, turns them into (mean, M2) in fp64, and
+// the block's row phases combine around phase 0's mean in phase order; one
+// (mean, M2) partial per (row block, channel).
+template <int DT>
+__global__ void __launch_bounds__(kRowThreads)
+k_tp_stats_rows(const uint4* __restrict__ x, int64_t R, int VC, int RB, int64_t C,
+                double2* __restrict__ part) {
+    constexpr int VE = Vec<DT>::N;
+    const RowTile<> rt(VC, R, RB);
+    const int64_t n = rt.count();
+    float piv[VE], s1[VE], s2[VE];
+#pragma unroll
+    for (int e = 0; e < VE; ++e) piv[e] = s1[e] = s2[e] = 0.f;
+    if (n > 0) {
+        const uint4* src = x + rt.col;
+        Vec<DT>::unpack(src[(rt.r0 + rt.phase) * VC], piv);
+        const int64_t step = rt.RPB;
+        int64_t r = rt.r0 + rt.phase;
+        auto add = [&](const uint4& v) {
+            float f[VE];
+            Vec<DT>::unpack(v, f);
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+                const float d = f[e] - piv[e];
+                s1[e] += d;
+                s2[e] = fmaf(d, d, s2[e]);
+            }
+        };
+        for (; r + (kStatsBatch - 1) * step < rt.r1; r += kStatsBatch * step) {
+            uint4 v[kStatsBatch];
+#pragma unroll
+            for (int k = 0; k < kStatsBatch; ++k) v[k] = __ldcs(src + (r + k * step) * VC);
+#pragma unroll
+            for (int k = 0; k < kStatsBatch; ++k) add(v[k]);
+        }
+        for (; r < rt.r1; r += step) add(__ldcs(src + r * VC));
+    }
+    // combine the row phases of each column, one channel of the vector at a time
+    __shared__ double2 sm[kRowThreads];
+    const double inv_n = n > 0 ? 1.0 / (double)n : 0.0;
+    const int64_t nrows = rt.r1 - rt.r0;
+    for (int e = 0; e < VE; ++e) {
+        const double a1 = s1[e];
+        sm[threadIdx.x] = make_double2(n > 0 ? (double)piv[e] + a1 * inv_n : 0.0,
+                                       n > 0 ? (double)s2[e] - a1 * a1 * inv_n : 0.0);
+        __syncthreads();
+        if (rt.active && rt.phase == 0) {
+            const double R0 = sm[threadIdx.x].x;
+            double q1 = 0.0, q2 = sm[threadIdx.x].y;
+            for (int ph = 1; ph < rt.RPB && ph < nrows; ++ph) {
+                const double2 v = sm[threadIdx.x + ph * rt.W];
+                const double np = (double)((nrows - 1 - ph) / rt.RPB + 1);
+                const double d = v.x - R0;
+                q1 += np * d;
+                q2 += v.y + np * d * d;
+            }
+            const double inv_rows = 1.0 / (double)nrows;
+            part[(int64_t)blockIdx.x * C + rt.col * VE + e] =
+                make_double2(R0 + q1 * inv_rows, q2 - q1 * q1 * inv_rows);
+        }
+        __syncthreads();
+    }
+}
+
+// Backward sums S1 = sum dy and S2 = sum dy*xhat (ElemBwd), fp32 per thread,
+// the row phases added in phase order; one partial per (row block, channel).
+template <int DT, int ACT, int MODE>
+__global__ void __launch_bounds__(kRowThreads)
+k_tp_reduce_rows(const uint4* __restrict__ z, const uint4* __restrict__ dz, int64_t R, int VC,
+                 int RB, int64_t C, const BwdIn in, double2* __restrict__ part) {
+    constexpr int VE = Vec<DT>::N;
+    constexpr int B = kStatsBatch / 2;   // rows per batch (two tensors)
+    const RowTile<> rt(VC, R, RB);
+    float s1[VE], s2[VE];
+#pragma unroll
+    for (int e = 0; e < VE; ++e) s1[e] = s2[e] = 0.f;
+    if (rt.count() > 0) {
+        ElemBwd<MODE, ACT, DT> eb[VE];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) eb[e].setup(in, rt.col * VE + e);
+        const uint4* pz = z + rt.col;
+        const uint4* pd = dz + rt.col;
+        const int64_t step = rt.RPB;
+        auto add = [&](const uint4& vz, const uint4& vd) {
+            float fz[VE], fd[VE];
+            Vec<DT>::unpack(vz, fz);
+            Vec<DT>::unpack(vd, fd);
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+                float xh, dy;
+                eb[e].eval(fz[e], fd[e], xh, dy);
+                s1[e] += dy;
+                s2[e] = fmaf(dy, xh, s2[e]);
+            }
+        };
+        int64_t r = rt.r0 + rt.phase;
+        for (; r + (B - 1) * step < rt.r1; r += B * step) {
+            uint4 vz[B], vd[B];
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                vz[k] = pz[(r + k * step) * VC];
+                vd[k] = pd[(r + k * step) * VC];
+            }
+#pragma unroll
+            for (int k = 0; k < B; ++k) add(vz[k], vd[k]);
+        }
+        for (; r < rt.r1; r += step) add(pz[r * VC], pd[r * VC]);
+    }
+    __shared__ float2 sm[kRowThreads];
+    for (int e = 0; e < VE; ++e) {
+        sm[threadIdx.x] = make_float2(s1[e], s2[e]);
+        __syncthreads();
+        if (rt.active && rt.phase == 0) {
+            float a = 0.f, b = 0.f;
+            for (int ph = 0; ph < rt.RPB; ++ph) {
+                const float2 v = sm[threadIdx.x + ph * rt.W];
+                a += v.x;
+                b += v.y;
+            }
+            part[(int64_t)blockIdx.x * C + rt.col * VE + e] = make_double2(a, b);
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------ NCHW units of small planes
+// For planes of at most kUnitMaxBytes, g = 16/gcd(16, HW*s) whole planes form a
+// unit that starts on a 16-byte boundary (U = g*HW*s/16 vectors); each thread
+// takes one unit, loads its vectors kRowBatch at a time and accumulates the
+// planes one after the other, writing each plane's partial when it ends.
+constexpr int kUnitMaxBytes = 1024;
+
+template <int DT>
+__global__ void __launch_bounds__(256)
+k_tp_stats_units(const uint4* __restrict__ x, int64_t units, int U, int HW,
+                 double2* __restrict__ part) {
+    constexpr int VE = Vec<DT>::N;
+    const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= units) return;
+    const uint4* src = x + u * U;
+    const int64_t plane0 = u * (int64_t)U * VE / HW;
+    int64_t plane = plane0;
+    int rem = HW;
+    float piv = 0.f, s1 = 0.f, s2 = 0.f;
+    bool first = true;
+    const double inv_hw = 1.0 / (double)HW;
+    auto add = [&](const uint4& v) {
+        float f[VE];
+        Vec<DT>::unpack(v, f);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) {
+            if (first) {
+                piv = f[e];
+                first = false;
+            }
+            const float d = f[e] - piv;
+            s1 += d;
+            s2 = fmaf(d, d, s2);
+            if (--rem == 0) {
+                const double a = s1;
+                part[plane] = make_double2((double)piv + a * inv_hw, (double)s2 - a * a * inv_hw);
+                ++plane;
+                rem = HW;
+                s1 = s2 = 0.f;
+                first = true;
+            }
+        }
+    };
+    int v = 0;
+    for (; v + kRowBatch <= U; v += kRowBatch) {
+        uint4 b[kRowBatch];
+#pragma unroll
+        for (int k = 0; k < kRowBatch; ++k) b[k] = __ldcs(src + v + k);
+#pragma unroll
+        for (int k = 0; k < kRowBatch; ++k) add(b[k]);
+    }
+    for (; v < U; ++v) add(__ldcs(src + v));
+}
+
+template <int DT, int ACT, int MODE>
+__global__ void __launch_bounds__(256)
+k_tp_reduce_units(const uint4* __restrict__ z, const uint4* __restrict__ dz, int64_t units,
+                  int U, int HW, int64_t C, const BwdIn in, double2* __restrict__ part) {
+    constexpr int VE = Vec<DT>::N;
+    constexpr int B = kRowBatch / 2;
+    const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= units) return;
+    const uint4* pz = z + u * U;
+    const uint4* pd = dz + u * U;
+    int64_t plane = u * (int64_t)U * VE / HW;
+    int rem = HW;
+    float s1 = 0.f, s2 = 0.f;
+    ElemBwd<MODE, ACT, DT> eb;
+    eb.setup(in, plane % C);
+    auto add = [&](const uint4& vz, const uint4& vd) {
+        float fz[VE], fd[VE];
+        Vec<DT>::unpack(vz, fz);
+        Vec<DT>::unpack(vd, fd);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) {
+            float xh, dy;
+            eb.eval(fz[e], fd[e], xh, dy);
+            s1 += dy;
+            s2 = fmaf(dy, xh, s2);
+            if (--rem == 0) {
+                part[plane] = make_double2(s1, s2);
+                ++plane;
+                rem = HW;
+                s1 = s2 = 0.f;
+                eb.setup(in, plane % C);
+            }
+        }
+    };
+    int v = 0;
+    for (; v + B <= U; v += B) {
+        uint4 bz[B], bd[B];
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            bz[k] = pz[v + k];
+            bd[k] = pd[v + k];
+        }
+#pragma unroll
+        for (int k = 0; k < B; ++k) add(bz[k], bd[k]);
+    }
+    for (; v < U; ++v) add(pz[v], pd[v]);
+}
+
+// Backward apply: block b of RB walks the rows [b*R/RB, (b+1)*R/RB) from the
+// end (the reduction's blocks read their ranges' ends last, so those are the
+// likeliest still in L2), the coefficients of the thread's channels in
+// registers; dx written over dz.
+template <int DT, int ACT, int MODE>
+__global__ void __launch_bounds__(kApplyThreads)
+k_tp_apply_bwd_rows(const uint4* __restrict__ z, uint4* dz, int64_t R, int VC, int RB, int64_t C,
+                    const float4* __restrict__ coef, float p, float inv_p) {
+    constexpr int VE = Vec<DT>::N;
+    constexpr int B = kRowBatch / 2;
+    const RowTile<kApplyThreads> rt(VC, R, RB);
+    const int64_t n = rt.count();
+    if (n == 0) return;
+    float4 k0[VE], k1[VE];
+#pragma unroll
+    for (int e = 0; e < VE; ++e) {
+        const int64_t c = rt.col * VE + e;
+        k0[e] = __ldg(coef + c);
+        k1[e] = MODE == kModeBwdZ ? k0[e] : __ldg(coef + C + c);
+    }
+    auto dx_of = [&](const uint4& vz, const uint4& vd) -> uint4 {
+        float fz[VE], fd[VE];
+        Vec<DT>::unpack(vz, fz);
+        Vec<DT>::unpack(vd, fd);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) {
+            if (MODE == kModeBwdZ) {
+                float y, dy;
+                act_backward<ACT, DT>(fz[e], fd[e], p, inv_p, y, dy);
+                fd[e] = fmaf(k0[e].x, dy, fmaf(k0[e].y, y, k0[e].z));
+            } else {
+                const float dy = act_dy_from_y<ACT, DT>(fmaf(fz[e], k0[e].x, k0[e].y), fd[e], p);
+                fd[e] = fmaf(k0[e].z, dy, fmaf(k1[e].x, fz[e], k1[e].y));
+            }
+        }
+        return Vec<DT>::pack(fd);
+    };
+    const uint4* pz = z + rt.col;
+    uint4* pd = dz + rt.col;
+    const int64_t step = rt.RPB;
+    // this thread's rows, last first: r = rlast, rlast - step, ...
+    int64_t r = rt.r0 + rt.phase + (n - 1) * step;
+    for (; r - (B - 1) * step >= rt.r0; r -= B * step) {
+        uint4 vz[B], vd[B];
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            vz[k] = __ldcs(pz + (r - k * step) * VC);
+            vd[k] = __ldcs(pd + (r - k * step) * VC);
+        }
+#pragma unroll
+        for (int k = 0; k < B; ++k) __stcs(pd + (r - k * step) * VC, dx_of(vz[k], vd[k]));
+    }
+    for (; r >= rt.r0; r -= step) __stcs(pd + r * VC, dx_of(__ldcs(pz + r * VC), __ldcs(pd + r * VC)));
+}
+
 // One warp per channel: S1 = sum dy and S2 = sum dy*xhat summed in fp64;
 // dbeta = S1, dgamma = S2.  The apply coefficients:
 //   in-place: dx in terms of y (the "INPLACE-ABN II" form), one record
@@ -497,6 +818,65 @@ static int apply_grid(const Geom& g, int sms, int per_sm) {
     return grid_for(nv, 2 * 256, sms * per_sm);
 }
 
+// NHWC rows that are a whole number of 16-byte vectors take the vector-column
+// kernels.
+static bool rows_vectorised(const Geom& g) {
+    const int64_t rby = g.C * g.esize;
+    return g.layout == kNHWC && rby % 16 == 0 && rby / 16 <= (int64_t)kRowThreads * 65535;
+}
+
+struct RowGrid {
+    int RB, GY, VC;
+};
+
+// NCHW small planes: g whole planes per 16-byte aligned unit (0: not used).
+static int unit_planes(const Geom& g) {
+    if (g.layout != kNCHW) return 0;
+    const int64_t pb = g.HW * g.esize;
+    int64_t a = pb, b = 16;
+    while (b) {
+        const int64_t t = a % b;
+        a = b;
+        b = t;
+    }
+    const int64_t gq = 16 / a;
+    if ((g.N * g.C) % gq != 0 || gq * pb > kUnitMaxBytes) return 0;
+    return (int)gq;
+}
+
+// Row blocks: a multiple of the SM count (an uneven second block on some SMs
+// would run alone), at most the workspace's partial slots and the rows.
+static RowGrid row_grid(const Geom& g, int sms) {
+    RowGrid rg;
+    rg.VC = (int)(g.C * g.esize / 16);
+    const int W = rg.VC < kRowThreads ? rg.VC : kRowThreads;
+    rg.GY = (rg.VC + W - 1) / W;
+    const int RPB = kRowThreads / W;
+    int64_t rb = sms > 0 ? (int64_t)(kMaxPartialBlocks / sms) * sms : kMaxPartialBlocks;
+    if (rb < 1) rb = kMaxPartialBlocks;
+    // a row block of fewer rows than row phases leaves threads idle
+    const int64_t most = (g.R + RPB - 1) / RPB;
+    if (rb > most) rb = most < 1 ? 1 : most;
+    rg.RB = (int)rb;
+    return rg;
+}
+
+// Row blocks of the backward apply: about `blocks` blocks in all (one wave),
+// none with fewer rows than row phases.
+static RowGrid apply_row_grid(const Geom& g, int blocks) {
+    RowGrid rg;
+    rg.VC = (int)(g.C * g.esize / 16);
+    const int W = rg.VC < kApplyThreads ? rg.VC : kApplyThreads;
+    rg.GY = (rg.VC + W - 1) / W;
+    const int RPB = kApplyThreads / W;
+    int64_t rb = blocks / rg.GY;
+    const int64_t most = (g.R + RPB - 1) / RPB;
+    if (rb > most) rb = most;
+    if (rb > 65535) rb = 65535;
+    rg.RB = (int)(rb < 1 ? 1 : rb);
+    return rg;
+}
+
 template <int DT>
 static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Workspace& w,
                                    cudaStream_t s, int sms) {
@@ -504,12 +884,26 @@ static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Worksp
     const T* x = static_cast<const T*>(a.x);
     int64_t K;
     int RB = 1;
-    if (g.layout == kNHWC) {
+    if (rows_vectorised(g)) {
+        const RowGrid rg = row_grid(g, sms);
+        RB = rg.RB;
+        k_tp_stats_rows<DT><<<dim3(rg.RB, rg.GY), kRowThreads, 0, s>>>(
+            static_cast<const uint4*>(a.x), g.R, rg.VC, rg.RB, g.C, w.part);
+        K = RB;
+        count_launches(1);
+    } else if (g.layout == kNHWC) {
         RB = nhwc_row_blocks(g.R);
         const int W = g.C < 256 ? (int)g.C : 256;
         dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
         k_tp_stats_nhwc<DT><<<grid, kTpRowThreads, 0, s>>>(x, g.R, g.C, RB, w.part);
         K = RB;
+        count_launches(1);
+    } else if (const int gq = unit_planes(g)) {
+        const int64_t units = g.N * g.C / gq;
+        k_tp_stats_units<DT><<<(unsigned)((units + 255) / 256), 256, 0, s>>>(
+            static_cast<const uint4*>(a.x), units, (int)(gq * g.HW * g.esize / 16), (int)g.HW,
+            w.part);
+        K = g.N;
         count_launches(1);
     } else {
         const int64_t planes = g.N * g.C;
@@ -551,13 +945,28 @@ static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Work
     const float inv_p = ACT == kIdent ? 1.f : 1.f / p;
     const BwdIn in{a.gamma, a.beta, a.save_mean, a.save_var, a.eps, p, inv_p};
     int64_t K;
-    if (g.layout == kNHWC) {
+    const bool rows = rows_vectorised(g);
+    const RowGrid rg = rows ? row_grid(g, sms) : RowGrid{};
+    if (rows) {
+        k_tp_reduce_rows<DT, ACT, MODE><<<dim3(rg.RB, rg.GY), kRowThreads, 0, s>>>(
+            static_cast<const uint4*>(a.src), static_cast<const uint4*>(a.dz), g.R, rg.VC, rg.RB,
+            g.C, in, w.part);
+        K = rg.RB;
+        count_launches(1);
+    } else if (g.layout == kNHWC) {
         const int RB = nhwc_row_blocks(g.R);
         const int W = g.C < 256 ? (int)g.C : 256;
         dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
         k_tp_reduce_nhwc<DT, ACT, MODE><<<grid, kTpRowThreads, 0, s>>>(z, dz, g.R, g.C, RB, in,
                                                                        w.part);
         K = RB;
+        count_launches(1);
+    } else if (const int gq = unit_planes(g)) {
+        const int64_t units = g.N * g.C / gq;
+        k_tp_reduce_units<DT, ACT, MODE><<<(unsigned)((units + 255) / 256), 256, 0, s>>>(
+            static_cast<const uint4*>(a.src), static_cast<const uint4*>(a.dz), units,
+            (int)(gq * g.HW * g.esize / 16), (int)g.HW, g.C, in, w.part);
+        K = g.N;
         count_launches(1);
     } else {
         const int64_t planes = g.N * g.C;
@@ -575,7 +984,14 @@ static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Work
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (g.layout == kNHWC) {
+    if (rows) {
+        auto kern = k_tp_apply_bwd_rows<DT, ACT, MODE>;
+        static std::atomic<int> occ{0};
+        const RowGrid ag = apply_row_grid(g, sms * ctas_per_sm(kern, kApplyThreads, occ));
+        kern<<<dim3(ag.RB, ag.GY), kApplyThreads, 0, s>>>(
+            static_cast<const uint4*>(a.src), static_cast<uint4*>(a.dz), g.R, ag.VC, ag.RB, g.C,
+            w.coef, p, inv_p);
+    } else if (g.layout == kNHWC) {
         k_tp_apply_bwd<DT, ACT, kNHWC, MODE><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
             z, dz, g.E, g.C, g.HW, w.coef, p, inv_p);
     } else {

@@ -155,8 +155,11 @@ def fp32_chain_length(sp: wl.LayerSpec, call: int = 1) -> int:
     backward passes through before it is widened to fp64, as the plan the
     backward call takes partitions the work (its launch shape comes from
     iabn_describe_plan; the two-phase partition is the one its kernels
-    document: NHWC blocks of 512 threads over 256 columns and at most 256
-    row blocks, merged in a tree; NCHW one warp per plane)."""
+    document: NHWC rows of whole 16-byte vectors in blocks of 512 threads
+    with fixed vector columns; other NHWC rows in blocks of 512 threads over
+    256 columns and at most 256 row blocks, merged in a tree; NCHW planes of
+    up to 1 KiB per 16-byte aligned group one thread per plane, larger ones
+    one warp per plane)."""
     import math
     import place_batchnorm_activation_b200 as iabn
     n, c, h, w = sp.shape
@@ -171,10 +174,23 @@ def fp32_chain_length(sp: wl.LayerSpec, call: int = 1) -> int:
             while lanes < 32 and lanes * 8 < hw:
                 lanes *= 2
         return -(-hw // lanes) + int(math.log2(lanes))
+    if sp.layout == wl.NHWC and (c * sp.itemsize) % 16 == 0:
+        # 16-byte vector columns: 512 threads, W = min(VC, 512) columns, row
+        # blocks a multiple of the SM count (at most 256) and at most the rows
+        # over the row phases; the phases are added in fp32 one by one
+        import torch
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        vc = c * sp.itemsize // 16
+        rp = 512 // min(vc, 512)
+        rb = min((256 // sms) * sms or 256, -(-rows // rp))
+        return -(-(-(-rows // rb)) // rp) + rp
     if sp.layout == wl.NHWC:
         rb = min(rows, 256)
         rp = 512 // min(c, 256)
         return -(-(-(-rows // rb)) // rp) + int(math.ceil(math.log2(rp)))
+    g = 16 // math.gcd(16, hw * sp.itemsize)
+    if (n * c) % g == 0 and g * hw * sp.itemsize <= 1024:
+        return hw + 1       # small planes: one thread sums a whole plane
     return -(-hw // 32) + 5
 
 
