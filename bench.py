@@ -249,7 +249,7 @@ class L2Flush:
         l2 = torch.cuda.get_device_properties(device).L2_cache_size
         n = 2 * max(l2, 64 << 20)
         self.w = torch.empty(n, dtype=torch.uint8, device=device)
-        self.r = torch.ones(n // 4, dtype=torch.int32, device=device)
+        self.r = torch.ones(n // 4, dtype=torch.float32, device=device)
         self.write_only = write_only
 
     def zero_(self):
@@ -597,7 +597,7 @@ def bench_inference(flush, steps, warmup, hbm_peak, device):
     return {"us": round(t * 1e3, 2), "gbs": round(gbs, 1),
             "frac_measured_hbm": round(gbs / hbm_peak, 4), "bytes_per_call": nbytes,
             "launches_per_call": launches,
-            "plan": "two launches: per-channel coefficients, then the elementwise pass"}
+            "plan": "one launch: coefficients formed in the elementwise pass"}
 
 
 def bench_twophase(flush, steps, warmup, hbm_peak, device):

@@ -42,13 +42,16 @@ struct Control {
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
-// Largest number of CTAs whose per-channel partials a workspace holds.
-constexpr int kMaxPartialBlocks = 256;
+// Largest number of blocks whose per-channel partials a workspace holds (NHWC).
+constexpr int kMaxPartialBlocks = 512;
+
+// Largest grid of the resident plan (one CTA per SM).
+constexpr int kMaxResidentCtas = 256;
 
 // Optional phase trace (IABN_TRACE=1): %globaltimer stamps, kTraceSlots per
-// CTA, in the workspace right after the control block.
+// resident CTA, in the workspace right after the control block.
 constexpr int kTraceSlots = 16;
-constexpr size_t kTraceBytes = (size_t)kMaxPartialBlocks * kTraceSlots * 8;
+constexpr size_t kTraceBytes = (size_t)kMaxResidentCtas * kTraceSlots * 8;
 
 // Default time budget of one bounded wait (grid barrier, mbarrier): 1 s.
 constexpr unsigned long long kWaitBudgetNs = 1000000000ull;
@@ -168,6 +171,17 @@ __device__ __forceinline__ void src_affine(float g, float b, float mean, float v
 }
 
 // ------------------------------------------------------------ small helpers
+
+// 16-byte global load, streaming (evict-first) cache hint.  asm volatile keeps
+// a batch of these in program order, so a batch is in flight before its values
+// are used.
+__device__ __forceinline__ uint4 ldg_cs(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
 
 __device__ __forceinline__ unsigned long long global_ns() {
     unsigned long long t;

@@ -179,7 +179,7 @@ bool make_plan(const Geom& g, int mode, const DeviceLimits& dl, ResPlan& P, int&
     P.ring = ring;
     P.smem_bytes = kBarBytes + P.scratch_bytes + nslots * P.slot_bytes;
     P.G = (int)(P.units < dl.sms ? P.units : dl.sms);
-    if (P.G > kMaxPartialBlocks) P.G = kMaxPartialBlocks;
+    if (P.G > kMaxResidentCtas) P.G = kMaxResidentCtas;
     // the kernel counts a CTA's units in 32 bits
     if ((P.units + P.G - 1) / P.G >= ((int64_t)1 << 31)) return false;
     P.hints = env_long("IABN_L2_HINTS", 1) != 0 ? 1 : 0;

@@ -28,9 +28,10 @@ constexpr int kTpRowThreads = 512;
 // values are used (the accumulation order stays row by row).
 constexpr int kTpBatch = 8;
 
-// Partial-summary slots per channel of the NHWC split statistics.
+// Row blocks of the NHWC reductions over single channels (rows that are not
+// whole 16-byte vectors).
 static inline int nhwc_row_blocks(int64_t R) {
-    return (int)(R < kMaxPartialBlocks ? R : kMaxPartialBlocks);
+    return (int)(R < 256 ? R : 256);
 }
 
 // ---------------------------------------------------------------- forward
@@ -140,8 +141,9 @@ __device__ __forceinline__ double partial_count(int layout, int64_t k, int64_t R
 }
 
 // One warp per channel: combine the K partial summaries (count_k, mean_k,
-// M2_k) in fp64 with the parallel-axis identity
-//   mean = sum count_k mean_k / M,  M2 = sum (M2_k + count_k (mean_k - mean)^2),
+// M2_k) in fp64 in one pass around r, the first partial's mean:
+//   s1 = sum count_k (mean_k - r),  s2 = sum M2_k + count_k (mean_k - r)^2,
+//   mean = r + s1/M,  M2 = s2 - s1^2/M,
 // then write the batch statistics and the apply coefficients.
 __global__ void __launch_bounds__(256)
 k_tp_finalize_fwd(const double2* __restrict__ part, int layout, int64_t C, int64_t K,
@@ -153,17 +155,20 @@ k_tp_finalize_fwd(const double2* __restrict__ part, int layout, int64_t C, int64
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t c = gw; c < C; c += nw) {
-        double s = 0.0;
-        for (int64_t k = lane; k < K; k += 32)
-            s += partial_count(layout, k, R, RB, HW) * part[k * C + c].x;
-        const double mean = warp_sum(s) / M;
-        double q = 0.0;
+        const double r = part[c].x;
+        double s1 = 0.0, s2 = 0.0;
+#pragma unroll 4
         for (int64_t k = lane; k < K; k += 32) {
             const double2 pk = part[k * C + c];
-            const double d = pk.x - mean;
-            q += pk.y + partial_count(layout, k, R, RB, HW) * d * d;
+            const double d = pk.x - r;
+            const double w = partial_count(layout, k, R, RB, HW) * d;
+            s1 += w;
+            s2 += pk.y + w * d;
         }
-        const double var = warp_sum(q) / M;
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        const double mean = r + s1 / M;
+        const double var = fmax((s2 - s1 * (s1 / M)) / M, 0.0);
         if (lane == 0) {
             save_mean[c] = (float)mean;
             save_var[c] = (float)var;
@@ -329,7 +334,8 @@ k_tp_reduce_nchw(const typename Storage<DT>::T* __restrict__ z,
 // owns rows [rb*R/RB, (rb+1)*R/RB) -- the partition the finalize counts -- and
 // the columns [cb*W, cb*W + W); its RPB = threads/W row phases take rows
 // phase, phase + RPB, ...  The reductions run one block of kRowThreads per SM
-// (the partials are per block) with 16 loads in flight per thread; the
+// (the partials are per block) with 16 loads in flight per thread (128 KiB
+// per SM); the
 // backward apply runs blocks of kApplyThreads, as many as fit, 8 loads in
 // flight per thread.
 
@@ -364,7 +370,7 @@ struct RowTile {
 // the block's row phases combine around phase 0's mean in phase order; one
 // (mean, M2) partial per (row block, channel).
 template <int DT>
-__global__ void __launch_bounds__(kRowThreads)
+__global__ void __launch_bounds__(kRowThreads, 1)
 k_tp_stats_rows(const uint4* __restrict__ x, int64_t R, int VC, int RB, int64_t C,
                 double2* __restrict__ part) {
     constexpr int VE = Vec<DT>::N;
@@ -391,16 +397,19 @@ k_tp_stats_rows(const uint4* __restrict__ x, int64_t R, int VC, int RB, int64_t 
         for (; r + (kStatsBatch - 1) * step < rt.r1; r += kStatsBatch * step) {
             uint4 v[kStatsBatch];
 #pragma unroll
-            for (int k = 0; k < kStatsBatch; ++k) v[k] = __ldcs(src + (r + k * step) * VC);
+            for (int k = 0; k < kStatsBatch; ++k) v[k] = ldg_cs(src + (r + k * step) * VC);
 #pragma unroll
             for (int k = 0; k < kStatsBatch; ++k) add(v[k]);
         }
-        for (; r < rt.r1; r += step) add(__ldcs(src + r * VC));
+        for (; r < rt.r1; r += step) add(ldg_cs(src + r * VC));
     }
-    // combine the row phases of each column, one channel of the vector at a time
+    // combine the row phases of each column, one channel of the vector at a
+    // time (unrolled: the per-channel registers must not be indexed at run time)
     __shared__ double2 sm[kRowThreads];
     const double inv_n = n > 0 ? 1.0 / (double)n : 0.0;
-    const int64_t nrows = rt.r1 - rt.r0;
+    const int nrows = (int)(rt.r1 - rt.r0);   // a row block's rows fit in 32 bits
+    const int pq = nrows / rt.RPB, pr = nrows - pq * rt.RPB;   // phase p has pq + (p < pr) rows
+#pragma unroll
     for (int e = 0; e < VE; ++e) {
         const double a1 = s1[e];
         sm[threadIdx.x] = make_double2(n > 0 ? (double)piv[e] + a1 * inv_n : 0.0,
@@ -411,7 +420,7 @@ k_tp_stats_rows(const uint4* __restrict__ x, int64_t R, int VC, int RB, int64_t 
             double q1 = 0.0, q2 = sm[threadIdx.x].y;
             for (int ph = 1; ph < rt.RPB && ph < nrows; ++ph) {
                 const double2 v = sm[threadIdx.x + ph * rt.W];
-                const double np = (double)((nrows - 1 - ph) / rt.RPB + 1);
+                const double np = (double)(pq + (ph < pr ? 1 : 0));
                 const double d = v.x - R0;
                 q1 += np * d;
                 q2 += v.y + np * d * d;
@@ -427,7 +436,7 @@ k_tp_stats_rows(const uint4* __restrict__ x, int64_t R, int VC, int RB, int64_t 
 // Backward sums S1 = sum dy and S2 = sum dy*xhat (ElemBwd), fp32 per thread,
 // the row phases added in phase order; one partial per (row block, channel).
 template <int DT, int ACT, int MODE>
-__global__ void __launch_bounds__(kRowThreads)
+__global__ void __launch_bounds__(kRowThreads, 1)
 k_tp_reduce_rows(const uint4* __restrict__ z, const uint4* __restrict__ dz, int64_t R, int VC,
                  int RB, int64_t C, const BwdIn in, double2* __restrict__ part) {
     constexpr int VE = Vec<DT>::N;
@@ -460,15 +469,16 @@ k_tp_reduce_rows(const uint4* __restrict__ z, const uint4* __restrict__ dz, int6
             uint4 vz[B], vd[B];
 #pragma unroll
             for (int k = 0; k < B; ++k) {
-                vz[k] = pz[(r + k * step) * VC];
-                vd[k] = pd[(r + k * step) * VC];
+                vz[k] = ldg_cs(pz + (r + k * step) * VC);
+                vd[k] = ldg_cs(pd + (r + k * step) * VC);
             }
 #pragma unroll
             for (int k = 0; k < B; ++k) add(vz[k], vd[k]);
         }
-        for (; r < rt.r1; r += step) add(pz[r * VC], pd[r * VC]);
+        for (; r < rt.r1; r += step) add(ldg_cs(pz + r * VC), ldg_cs(pd + r * VC));
     }
     __shared__ float2 sm[kRowThreads];
+#pragma unroll
     for (int e = 0; e < VE; ++e) {
         sm[threadIdx.x] = make_float2(s1[e], s2[e]);
         __syncthreads();
@@ -852,8 +862,9 @@ static RowGrid row_grid(const Geom& g, int sms) {
     const int W = rg.VC < kRowThreads ? rg.VC : kRowThreads;
     rg.GY = (rg.VC + W - 1) / W;
     const int RPB = kRowThreads / W;
-    int64_t rb = sms > 0 ? (int64_t)(kMaxPartialBlocks / sms) * sms : kMaxPartialBlocks;
-    if (rb < 1) rb = kMaxPartialBlocks;
+    // one block per SM, 16 loads in flight per thread
+    int64_t rb = sms > 0 ? (int64_t)sms : 256;
+    if (rb > kMaxPartialBlocks) rb = kMaxPartialBlocks;
     // a row block of fewer rows than row phases leaves threads idle
     const int64_t most = (g.R + RPB - 1) / RPB;
     if (rb > most) rb = most < 1 ? 1 : most;
