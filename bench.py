@@ -86,7 +86,9 @@ def parse_args():
                     help="skip the other workloads and the CPU baseline")
     ap.add_argument("--profile", type=int, default=0, metavar="WORKLOAD",
                     help="profiling run: only `warmup` + `steps` fwd/bwd/running steps of "
-                         "workload 1, 2 or 3 (no e2e, extras or JSON line)")
+                         "workload 1, 2, 3 or 4 (no e2e, extras or JSON line)")
+    ap.add_argument("--layer", type=int, default=0,
+                    help="with --profile 4: the layer of the sweep")
     return ap.parse_args()
 
 
@@ -746,7 +748,7 @@ def run_profile(args):
     import workloads as wl
     device = torch.device("cuda", 0)
     flush = L2Flush(device, write_only=os.environ.get("IABN_BENCH_WRITE_FLUSH") == "1")
-    sp = wl.spec(args.profile)
+    sp = wl.spec(args.profile, args.layer if args.profile == 4 else 0)
     layer = Layer(sp, sp.seed, device)
     f, b, u, launches, _ = timed_layer_steps(layer, flush, args.steps, args.warmup)
     print(f"profile {sp.name}: fwd_us={statistics.mean(f) * 1e3:.2f} "
