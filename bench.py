@@ -34,15 +34,18 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elements/s"
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
-# resident kernels on the ResNet-trunk layer, from one ncu capture of
-# `python bench.py --profile 1 --steps 1 --warmup 1` (see
-# profiles/k_resident_resnet_trunk.md).  Reported only while the CUDA sources
-# hash to the value they were captured on; otherwise "traffic" is null.
+# DRAM bytes per launch (dram__bytes_read.sum, dram__bytes_write.sum) of the
+# resident kernels on the ResNet-trunk layer, from one ncu capture:
+#   python bench.py --profile 1 --steps 1 --warmup 1
+#   ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum \
+#       --clock-control none -k regex:k_resident -s 2 -c 2 --csv \
+#       python bench.py --profile 1 --steps 1 --warmup 1
+# Reported only while the CUDA sources hash to the value they were captured
+# on; otherwise "traffic" and "dram_bytes" are null.
 NCU_TRAFFIC = {
-    "sources_sha256": "3f329c8647407bf0f144fbd15a039b5083c86d7822a943c50809dc7cfbefd2eb",
-    "backward": 287329536 + 34717440,
-    "forward": 109736192 + 23128064,
+    "sources_sha256": "12dc261b5b714a43a82074d78278cdff307fea806943802f38b1400834dc3ec7",
+    "backward": {"read": 287629824, "write": 37336064},
+    "forward": {"read": 110013440, "write": 22978560},
 }
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -70,10 +73,18 @@ def kernel_sources_sha256() -> str:
 
 
 def ncu_traffic(direction: str):
-    """Captured DRAM bytes per launch, or None if the kernels changed since."""
+    """Captured DRAM bytes (read + write) per launch, or None if the kernels
+    changed since."""
     if kernel_sources_sha256() != NCU_TRAFFIC["sources_sha256"]:
         return None
-    return NCU_TRAFFIC[direction]
+    return NCU_TRAFFIC[direction]["read"] + NCU_TRAFFIC[direction]["write"]
+
+
+def ncu_dram(direction: str):
+    """The captured DRAM read and write bytes per launch (None if stale)."""
+    if kernel_sources_sha256() != NCU_TRAFFIC["sources_sha256"]:
+        return None
+    return dict(NCU_TRAFFIC[direction])
 
 
 def parse_args():
@@ -89,6 +100,9 @@ def parse_args():
                          "workload 1, 2, 3 or 4 (no e2e, extras or JSON line)")
     ap.add_argument("--layer", type=int, default=0,
                     help="with --profile 4: the layer of the sweep")
+    ap.add_argument("--layer-kind", choices=["inplace", "standard", "checkpoint", "inference"],
+                    default="inplace",
+                    help="with --profile: which layer's calls to run (default: in-place)")
     return ap.parse_args()
 
 
@@ -749,6 +763,34 @@ def run_profile(args):
     device = torch.device("cuda", 0)
     flush = L2Flush(device, write_only=os.environ.get("IABN_BENCH_WRITE_FLUSH") == "1")
     sp = wl.spec(args.profile, args.layer if args.profile == 4 else 0)
+    if args.layer_kind != "inplace":
+        # per-call times of the other layers' calls, same protocol
+        L = LayerVariants(sp, sp.seed, device)
+        if args.layer_kind == "inference":
+            for _ in range(3):
+                L.restore()
+                L.fwd()
+                L.run()
+            calls = [("inference", lambda: L.iabn.inference(
+                L.x, L.gamma, L.beta, L.rmean, L.rvar, L.ws, **L.kw()))]
+        else:
+            calls = L.calls(args.layer_kind)
+        times = {name: [] for name, _ in calls}
+        for i in range(args.warmup + args.steps):
+            L.restore()
+            for name, fn in calls:
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                if i >= args.warmup:
+                    times[name].append((a, b))
+        torch.cuda.synchronize()
+        print(f"profile {sp.name} {args.layer_kind}: " + " ".join(
+            f"{k}_us={statistics.mean(x.elapsed_time(y) for x, y in v) * 1e3:.2f}"
+            for k, v in times.items()), flush=True)
+        return 0
     layer = Layer(sp, sp.seed, device)
     f, b, u, launches, _ = timed_layer_steps(layer, flush, args.steps, args.warmup)
     print(f"profile {sp.name}: fwd_us={statistics.mean(f) * 1e3:.2f} "
@@ -893,12 +935,14 @@ def main():
                          "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(achieved / hbm_peak, 4),
                          "traffic": ncu_traffic("backward"),
+                         "dram_bytes": ncu_dram("backward"),
                          "peak_source": f"{peak_kind} hbm_gbs",
                          "algorithmic_bytes_per_launch": bwd_bytes},
             "roofline_fwd": {"bound": "hbm", "achieved": round(fwd_achieved, 1),
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(fwd_achieved / hbm_peak, 4),
                              "traffic": ncu_traffic("forward"),
+                             "dram_bytes": ncu_dram("forward"),
                              "algorithmic_bytes_per_launch": 2 * sp.numel * sp.itemsize},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e_max, 3)},

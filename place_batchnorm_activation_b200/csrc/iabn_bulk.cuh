@@ -101,13 +101,6 @@ __device__ __forceinline__ void stg128(void* p, const uint4& v) {
                  : "memory");
 }
 
-// The same with an L2 eviction-priority policy (createpolicy) for the line.
-__device__ __forceinline__ void stg128_hint(void* p, const uint4& v, uint64_t policy) {
-    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p),
-                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy)
-                 : "memory");
-}
-
 // 16-byte shared-memory load / store at a 32-bit shared address.
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;

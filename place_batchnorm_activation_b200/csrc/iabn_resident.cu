@@ -13,7 +13,6 @@
 // Tuning knobs read from the environment (defaults in brackets):
 //   IABN_L2_HINTS [1]       L2 evict-last on tiles phase B reloads, evict-first
 //                           on the rest; 0 = no hints.
-//   IABN_STORE_HINT [1]     phase B's stores evict-first in L2 (needs IABN_L2_HINTS).
 //   IABN_TILE_KB_FWD, IABN_TILE_KB_BWD [48, 24] KiB per tensor per tile.
 //   IABN_RING_FWD, IABN_RING_BWD       [4, 4]   slots cycled by the stream.
 //   IABN_BARRIER_BUDGET_NS  [1e9] time budget of each bounded wait.
@@ -183,7 +182,6 @@ bool make_plan(const Geom& g, int mode, const DeviceLimits& dl, ResPlan& P, int&
     // the kernel counts a CTA's units in 32 bits
     if ((P.units + P.G - 1) / P.G >= ((int64_t)1 << 31)) return false;
     P.hints = env_long("IABN_L2_HINTS", 1) != 0 ? 1 : 0;
-    P.store_hint = P.hints && env_long("IABN_STORE_HINT", 1) != 0 ? 1 : 0;
     return true;
 }
 

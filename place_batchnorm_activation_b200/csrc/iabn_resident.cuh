@@ -69,9 +69,6 @@ struct ResPlan {
     int VC, RP;          // NHWC: 16-byte columns per row; row phases (threads per column)
     int g, L;            // NCHW: planes per unit; lanes per plane
     int hints;           // 1: L2 eviction-priority hints on the bulk copies
-    int store_hint;      // 1: phase B's stores carry an L2 evict-first hint, so the
-                         // results cycle through few L2 lines instead of evicting the
-                         // tiles phase B still has to read back
     int stash_first;     // 1: the stash holds each thread's first rows, 0: its last
     int stash_cp;        // 1: the copy engine (tcgen05.cp) fills the stash from the
                          // landed slots (CPT 1, RP*VC = 256, first rows); 0: the
@@ -1223,8 +1220,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         }
     } else if (consumer && !failed()) {
         // results go straight to global memory (16-byte stores)
-        const uint64_t pol_st = P.store_hint ? policy_evict_first() : policy_evict_normal();
-        auto put = [&](void* g, const uint4& v) { stg128_hint(g, v, pol_st); };
+        auto put = [&](void* g, const uint4& v) { stg128(g, v); };
         // coefficients of this thread's channels (NHWC)
         // c3/c4 are kept per channel only when a thread owns one column;
         // otherwise the backward forms them on the fly (register budget).
