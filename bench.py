@@ -22,6 +22,7 @@ oracle (test infrastructure) on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -47,6 +48,10 @@ NCU_TRAFFIC = {
     "backward": {"read": 287629824, "write": 37336064},
     "forward": {"read": 110013440, "write": 22978560},
 }
+# the resident kernels' phase trace in the workspace (IABN_TRACE=1): up to 256
+# CTAs x 16 slots of 8 bytes, right after the 256-byte control block
+TRACE_SLOTS = 16
+TRACE_BYTES = 256 * TRACE_SLOTS * 8
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
@@ -103,6 +108,9 @@ def parse_args():
     ap.add_argument("--layer-kind", choices=["inplace", "standard", "checkpoint", "inference"],
                     default="inplace",
                     help="with --profile: which layer's calls to run (default: in-place)")
+    ap.add_argument("--probe", action="store_true",
+                    help="run the measurement probes of include/iabn_probe.h (launch floor, "
+                         "L2 retention and read rates, cluster occupancy) and print them")
     return ap.parse_args()
 
 
@@ -519,7 +527,7 @@ def bench_other_workloads(flush, steps, warmup, hbm_peak, device):
         tf, tb = statistics.median(f), statistics.median(b)
         gbs = L.bytes / ((tf + tb) * 1e-3) / 1e9
         out[sp.name] = {"fwd_us": round(tf * 1e3, 2), "bwd_us": round(tb * 1e3, 2),
-                        "gbs": round(gbs, 1), "frac_measured_hbm": round(gbs / hbm_peak, 4),
+                        "gbs": round(gbs, 1), "frac_hbm_peak": round(gbs / hbm_peak, 4),
                         "frac_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
                         "elements_per_s": sp.numel / ((tf + tb) * 1e-3)}
         del L
@@ -567,7 +575,7 @@ def bench_other_workloads(flush, steps, warmup, hbm_peak, device):
     total_bytes = sum(L.bytes for L in layers)
     gbs = total_bytes / (t * 1e-3) / 1e9
     out["layer_sweep"] = {"sum_of_32_calls_us": round(t * 1e3, 2), "gbs": round(gbs, 1),
-                          "frac_measured_hbm": round(gbs / hbm_peak, 4),
+                          "frac_hbm_peak": round(gbs / hbm_peak, 4),
                           "frac_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
                           "elements_per_s": sum(L.sp.numel for L in layers) / (t * 1e-3),
                           "dz": "fresh N(0,1) per layer"}
@@ -611,7 +619,7 @@ def bench_inference(flush, steps, warmup, hbm_peak, device):
     del L
     torch.cuda.empty_cache()
     return {"us": round(t * 1e3, 2), "gbs": round(gbs, 1),
-            "frac_measured_hbm": round(gbs / hbm_peak, 4), "bytes_per_call": nbytes,
+            "frac_hbm_peak": round(gbs / hbm_peak, 4), "bytes_per_call": nbytes,
             "launches_per_call": launches,
             "plan": "one launch: coefficients formed in the elementwise pass"}
 
@@ -637,7 +645,7 @@ def bench_twophase(flush, steps, warmup, hbm_peak, device):
     del L
     torch.cuda.empty_cache()
     return {"fwd_us": round(tf * 1e3, 2), "bwd_us": round(tb * 1e3, 2), "gbs": round(gbs, 1),
-            "frac_measured_hbm": round(gbs / hbm_peak, 4),
+            "frac_hbm_peak": round(gbs / hbm_peak, 4),
             "launches_per_step": launches / max(1, steps),
             "plan": "IABN_FORCE_PLAN=twophase"}
 
@@ -806,12 +814,12 @@ def run_profile(args):
             if what == "bwd":
                 layer.fwd()
                 flush.zero_()
-                layer.ws[256:256 + 32768].zero_()
+                layer.ws[256:256 + TRACE_BYTES].zero_()
             else:
-                layer.ws[256:256 + 32768].zero_()
+                layer.ws[256:256 + TRACE_BYTES].zero_()
             call()
             torch.cuda.synchronize()
-            tr = layer.ws[256:256 + 32768].view(torch.int64).view(256, 16).cpu()
+            tr = layer.ws[256:256 + TRACE_BYTES].view(torch.int64).view(256, TRACE_SLOTS).cpu()
             rows = [r for r in tr.tolist() if r[0] != 0]
             if not rows:
                 print(f"trace {sp.name} {what}: no resident-kernel stamps (two-phase plan)",
@@ -830,10 +838,119 @@ def run_profile(args):
     return 0
 
 
+def run_probe(args):
+    """The measurement probes of include/iabn_probe.h on GPU 0.
+
+    * launch floor: CUDA events around nothing, around one empty kernel of the
+      resident kernel's shape (148 x 320; without and with the cooperative
+      attribute and the resident kernel's dynamic shared memory) and around
+      two; the bench's L2 flush before every window; median of 40.
+    * L2: for a buffer of S MB, a read after the flush (cold), a second read
+      of the same bytes in the same order (what L2 kept), then an in-place
+      read + write; mean of 3 after one discarded round.  Marginal rates come
+      from the difference between two sizes, which cancels the launch cost.
+    * cluster occupancy: co-resident clusters of 1..16 blocks of 320 threads
+      with the resident kernel's dynamic shared memory (a host query).
+    """
+    import torch
+    import place_batchnorm_activation_b200 as iabn
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    props = torch.cuda.get_device_properties(device)
+    sms = props.multi_processor_count
+    optin = int(getattr(props, "shared_memory_per_block_optin", 232448))
+    smem = optin - 1024
+    flush = L2Flush(device)
+    st = torch.cuda.current_stream(device)
+    sh = ctypes.c_void_p(st.cuda_stream)
+
+    def ok(rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what}: status {rc}")
+
+    def timed(fn, reps, discard=0):
+        ts = []
+        for r in range(reps + discard):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            b.synchronize()
+            if r >= discard:
+                ts.append(a.elapsed_time(b) * 1e3)
+        return ts
+
+    floor = {}
+    cases = [("events only", []),
+             ("empty 148x320, no shared memory, plain", [(0, 0)]),
+             ("the same, cooperative", [(0, 1)]),
+             (f"the same with {smem // 1024} KB dynamic shared memory, plain", [(smem, 0)]),
+             ("the same, cooperative", [(smem, 1)]),
+             (f"two {smem // 1024} KB cooperative empty kernels", [(smem, 1), (smem, 1)])]
+    for i, (name, launches) in enumerate(cases):
+        def fn(launches=launches):
+            for sm_bytes, coop in launches:
+                ok(iabn.iabn_probe_empty(sms, 320, sm_bytes, coop, sh), "iabn_probe_empty")
+        floor[f"{i}: {name}"] = round(statistics.median(timed(fn, 40, 3)), 2)
+
+    MB = 1 << 20
+    sizes = [24, 40, 56, 72, 88, 104, 120, 160]
+    buf = torch.zeros(max(sizes) * MB, dtype=torch.uint8, device=device)
+    l2 = {}
+    for S in sizes:
+        nb = S * MB
+        cold, warm, rw = [], [], []
+        for r in range(4):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(st)
+            ok(iabn.iabn_probe_read(buf.data_ptr(), nb, sms, sh), "iabn_probe_read")
+            ev[1].record(st)
+            ok(iabn.iabn_probe_read(buf.data_ptr(), nb, sms, sh), "iabn_probe_read")
+            ev[2].record(st)
+            ok(iabn.iabn_probe_read_write(buf.data_ptr(), nb, sms, sh), "iabn_probe_read_write")
+            ev[3].record(st)
+            ev[3].synchronize()
+            if r > 0:
+                cold.append(ev[0].elapsed_time(ev[1]) * 1e3)
+                warm.append(ev[1].elapsed_time(ev[2]) * 1e3)
+                rw.append(ev[2].elapsed_time(ev[3]) * 1e3)
+        l2[S] = {"cold_read_us": round(statistics.mean(cold), 2),
+                 "re_read_us": round(statistics.mean(warm), 2),
+                 "read_write_us": round(statistics.mean(rw), 2)}
+    lo, hi = 24, 72
+
+    def marginal(key, factor=1):
+        dt = l2[hi][key] - l2[lo][key]
+        return round(factor * (hi - lo) * MB / (dt * 1e3), 1) if dt > 0 else None
+
+    rates = {"dram_read_gbs": marginal("cold_read_us"),
+             "l2_hit_read_gbs": marginal("re_read_us"),
+             "l2_read_plus_write_gbs": marginal("read_write_us", 2),
+             "sizes_mb": [lo, hi]}
+    clusters = {k: iabn.iabn_probe_cluster_occupancy(k, 320, smem) for k in (1, 2, 4, 8, 16)}
+    for name, us in floor.items():
+        print(f"floor  {name}: {us} us", flush=True)
+    for S, v in l2.items():
+        print(f"l2     {S:4d} MB: cold {v['cold_read_us']:.2f} us  re-read {v['re_read_us']:.2f} us"
+              f"  read+write {v['read_write_us']:.2f} us", flush=True)
+    print(f"rates  {rates}", flush=True)
+    for k, n in clusters.items():
+        print(f"clusters of {k:2d}: {n} resident ({n * k} blocks of {sms} SMs)", flush=True)
+    print(json.dumps({"probe": {"sms": sms, "launch_floor_us": floor, "l2_mb": l2,
+                                "marginal_rates": rates,
+                                "clusters": {str(k): v for k, v in clusters.items()},
+                                "smem_bytes": smem}}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.probe:
+        return run_probe(args)
     if args.profile:
         return run_profile(args)
     import torch
@@ -930,7 +1047,11 @@ def main():
             "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
             "running_update_us": round(statistics.mean(u) * 1e3, 2),
             "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
-            "frac_of_measured_hbm": round(value / world / hbm_peak, 4),
+            "frac_of_hbm_peak": round(value / world / hbm_peak, 4),
+            "hbm_peak": {"gbs": hbm_peak,
+                         "source": ("measured copy bandwidth (MEASURED_PEAKS.json)"
+                                    if peak_kind == "measured" else
+                                    "fallback: no MEASURED_PEAKS.json beside bench.py")},
             "roofline": {"bound": "hbm", "kernel": "backward (iabn_backward)",
                          "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(achieved / hbm_peak, 4),

@@ -50,6 +50,9 @@ EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_backward",
            "iabn_forward_static_ws", "iabn_describe_plan", "iabn_inference",
            "iabn_forward_standard", "iabn_backward_standard", "iabn_forward_checkpoint",
            "iabn_backward_checkpoint", "iabn_checkpoint_recompute")
+# Symbols include/iabn_probe.h declares: measurement probes, not the method.
+PROBE_EXPORTS = ("iabn_probe_empty", "iabn_probe_read", "iabn_probe_read_write",
+                 "iabn_probe_cluster_occupancy")
 
 # iabn_call values (iabn_describe_plan)
 (IABN_CALL_FORWARD, IABN_CALL_BACKWARD, IABN_CALL_FORWARD_STANDARD, IABN_CALL_BACKWARD_STANDARD,
@@ -127,6 +130,14 @@ def lib() -> ctypes.CDLL:
             L.iabn_forward_static_ws.restype = i32
             L.iabn_describe_plan.argtypes = [pd, i32, i32, i32, ctypes.POINTER(IabnPlanInfo)]
             L.iabn_describe_plan.restype = i32
+            L.iabn_probe_empty.argtypes = [i32, i32, i32, i32, vp]
+            L.iabn_probe_empty.restype = i32
+            L.iabn_probe_read.argtypes = [vp, ctypes.c_size_t, i32, vp]
+            L.iabn_probe_read.restype = i32
+            L.iabn_probe_read_write.argtypes = [vp, ctypes.c_size_t, i32, vp]
+            L.iabn_probe_read_write.restype = i32
+            L.iabn_probe_cluster_occupancy.argtypes = [i32, i32, i32, ctypes.POINTER(i32)]
+            L.iabn_probe_cluster_occupancy.restype = i32
             _lib = L
     return _lib
 
@@ -220,6 +231,27 @@ def iabn_forward_static_ws(desc, x_inout, gamma, beta, eps, act, act_param, save
 def iabn_describe_plan(desc, call, sm_count, smem_optin, info) -> int:
     return int(lib().iabn_describe_plan(ctypes.byref(desc), call, sm_count, smem_optin,
                                         ctypes.byref(info)))
+
+
+def iabn_probe_empty(blocks, threads, smem_bytes, cooperative, stream) -> int:
+    return int(lib().iabn_probe_empty(blocks, threads, smem_bytes, cooperative, stream))
+
+
+def iabn_probe_read(src, nbytes, blocks, stream) -> int:
+    return int(lib().iabn_probe_read(src, nbytes, blocks, stream))
+
+
+def iabn_probe_read_write(buf, nbytes, blocks, stream) -> int:
+    return int(lib().iabn_probe_read_write(buf, nbytes, blocks, stream))
+
+
+def iabn_probe_cluster_occupancy(cluster_size, threads, smem_bytes) -> int:
+    """The number of co-resident clusters (raises on an error status)."""
+    n = ctypes.c_int32(0)
+    _ok(int(lib().iabn_probe_cluster_occupancy(cluster_size, threads, smem_bytes,
+                                               ctypes.byref(n))),
+        "iabn_probe_cluster_occupancy")
+    return int(n.value)
 
 
 # ---------------------------------------------------------- tensor helpers

@@ -18,29 +18,32 @@ import place_batchnorm_activation_b200 as iabn
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "iabn.h")
+PROBE_HEADER = os.path.join(ROOT, "include", "iabn_probe.h")
 
 no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
                                  reason="fake device addresses are only passed without a GPU")
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(iabn_[a-z_]+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_exports():
     assert declared_functions() == sorted(iabn.EXPORTS)
+    assert declared_functions(PROBE_HEADER) == sorted(iabn.PROBE_EXPORTS)
 
 
 def test_library_exports_every_declared_symbol():
     lib = iabn.lib()
-    for name in declared_functions():
+    declared = declared_functions() + declared_functions(PROBE_HEADER)
+    for name in declared:
         assert hasattr(lib, name), name
     out = subprocess.run(["nm", "-D", "--defined-only", iabn.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = set(re.findall(r"\bT (iabn_\w+)", out))
-    assert set(declared_functions()) <= exported
+    assert set(declared) <= exported
 
 
 def test_workspace_size():
@@ -173,3 +176,15 @@ def test_tensor_helpers_refuse_cpu_tensors():
     with pytest.raises(iabn.IabnError):
         iabn.forward(x, g, g, g, g, torch.zeros(1 << 16, dtype=torch.uint8),
                      shape=(2, 4, 3, 3), layout=0, eps=1e-5, act=0, act_param=0.01)
+
+
+@no_gpu_only
+def test_probes_reject_bad_arguments_on_the_host():
+    assert iabn.iabn_probe_empty(0, 320, 0, 0, None) == iabn.IABN_ERR_INVALID_ARG
+    assert iabn.iabn_probe_empty(148, 2048, 0, 0, None) == iabn.IABN_ERR_INVALID_ARG
+    assert iabn.iabn_probe_read(None, 1 << 20, 148, None) == iabn.IABN_ERR_INVALID_ARG
+    assert iabn.iabn_probe_read(FAKE, 17, 148, None) == iabn.IABN_ERR_INVALID_ARG
+    assert iabn.iabn_probe_read_write(FAKE + 8, 1 << 20, 148, None) == iabn.IABN_ERR_INVALID_ARG
+    assert iabn.iabn_probe_read_write(FAKE, 1 << 20, 0, None) == iabn.IABN_ERR_INVALID_ARG
+    with pytest.raises(RuntimeError):
+        iabn.iabn_probe_cluster_occupancy(0, 320, 0)

@@ -80,6 +80,9 @@ def test_ncu_traffic_only_for_captured_sources(monkeypatch):
     import bench
     traffic = dict(bench.NCU_TRAFFIC)
     monkeypatch.setattr(bench, "NCU_TRAFFIC", dict(traffic, sources_sha256=bench.kernel_sources_sha256()))
-    assert bench.ncu_traffic("backward") == traffic["backward"]
+    bwd = traffic["backward"]
+    assert bench.ncu_traffic("backward") == bwd["read"] + bwd["write"]
+    assert bench.ncu_dram("backward") == bwd
     monkeypatch.setattr(bench, "NCU_TRAFFIC", dict(traffic, sources_sha256="0" * 64))
     assert bench.ncu_traffic("backward") is None
+    assert bench.ncu_dram("backward") is None
