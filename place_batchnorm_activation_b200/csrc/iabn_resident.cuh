@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const uint32_t bbase = tid == 0 ? bar_base(a.ctl) : 0u;
     if (consumer && (lane & 15) == 0) {
         const int h = lane >> 4;
-        const int64_t c = ((int64_t)b * kConsumerWarps + warp) * 2 + h;
+        const int64_t c = ((int64_t)warp * G + b) * 2 + h;
         if (c < a.C) {
             cp_async4(&s_par[warp][h][0], a.gamma + c);
             cp_async4(&s_par[warp][h][1], a.beta + c);
@@ -951,10 +951,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
 #pragma unroll
                 for (int q = 0; q < NP; ++q) {
                     const int64_t ch = (int64_t)(col[0] * NP + q) * 2;
-                    double2* dstp = a.part + (int64_t)b * a.C + ch;
+                    double2* dstp = a.part + ch * G + b;   // channel-major
                     dstp[0] = make_double2(R[q].x + s1[q].x * inv_rows,
                                            s2[q].x - s1[q].x * s1[q].x * inv_rows);
-                    dstp[1] = make_double2(R[q].y + s1[q].y * inv_rows,
+                    dstp[G] = make_double2(R[q].y + s1[q].y * inv_rows,
                                            s2[q].y - s1[q].y * s1[q].y * inv_rows);
                 }
             }
@@ -968,9 +968,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         double2 mean, m2;
                         summary(k * NP + q, mean, m2);
                         const int64_t ch = (int64_t)(col[k] * NP + q) * 2;
-                        double2* dstp = a.part + (int64_t)b * a.C + ch;
+                        double2* dstp = a.part + ch * G + b;   // channel-major
                         dstp[0] = make_double2(mean.x, m2.x);
-                        dstp[1] = make_double2(mean.y, m2.y);
+                        dstp[G] = make_double2(mean.y, m2.y);
                     }
         }
         stamp(6, tid == 0);
@@ -1011,9 +1011,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     for (int q = 0; q < NP; ++q) {
                         const int64_t ch = (int64_t)(col[k] * NP + q) * 2;
                         const int i = k * NP + q;
-                        double2* dstp = a.part + (int64_t)b * a.C + ch;
+                        double2* dstp = a.part + ch * G + b;   // channel-major
                         dstp[0] = make_double2(acc0[i].x, acc1[i].x);
-                        dstp[1] = make_double2(acc0[i].y, acc1[i].y);
+                        dstp[G] = make_double2(acc0[i].y, acc1[i].y);
                     }
         }
     }
@@ -1034,6 +1034,11 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     // counts are known before the partials are.
     constexpr int KC = 10;   // partials cached per lane when K <= 160
     const int64_t K = LAYOUT == kNHWC ? (int64_t)G : a.N;
+    // partial k of channel c: NHWC channel-major (a half-warp's loads of one
+    // channel are contiguous), NCHW per plane (n, c) in plane order
+    auto part_at = [&](int64_t k, int64_t c) -> double2 {
+        return LAYOUT == kNHWC ? a.part[c * K + k] : a.part[k * a.C + c];
+    };
     const bool cached = K <= 16 * KC;
     auto count_of = [&](int64_t k) -> double {
         if (LAYOUT == kNCHW) return (double)a.HW;
@@ -1051,11 +1056,13 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     if (!failed() && consumer) {
         // one consumer half-warp per channel over the whole grid, fp64, fixed
         // order; a warp takes the channels 2cp and 2cp+1 (the loop is
-        // warp-uniform; a half without a channel computes on a stand-in)
+        // warp-uniform; a half without a channel computes on a stand-in).
+        // Channel pairs go to warp 0 of every CTA first, then warp 1, ...: the
+        // scattered partial loads spread over as many SMs as there are pairs.
         const int hl = lane & 15, half = lane >> 4;
         const int64_t nw = (int64_t)G * kConsumerWarps;
         bool first = true;
-        for (int64_t cpair = (int64_t)b * kConsumerWarps + warp; cpair * 2 < a.C;
+        for (int64_t cpair = (int64_t)warp * G + b; cpair * 2 < a.C;
              cpair += nw, first = false) {
             const int64_t cw = cpair * 2 + half;
             const bool cv = cw < a.C;
@@ -1064,7 +1071,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
 #pragma unroll
             for (int i = 0; i < KC; ++i) {
                 const int64_t k = hl + 16 * i;
-                pk[i] = cached && k < K ? a.part[k * a.C + c] : make_double2(0.0, 0.0);
+                pk[i] = cached && k < K ? part_at(k, c) : make_double2(0.0, 0.0);
             }
             // per-channel parameters (lane 0 of the half uses them)
             float gmf = 0.f, btf = 0.f, vif = 0.f, mnf = 0.f;
@@ -1087,7 +1094,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 // partial's mean:
                 //   s1 = sum n_k (mean_k - r),  s2 = sum M2_k + n_k (mean_k - r)^2,
                 //   mean = r + s1/M,  M2 = s2 - s1^2/M.
-                const double r = __shfl_sync(0xffffffffu, cached ? pk[0].x : a.part[c].x, 0, 16);
+                const double r = __shfl_sync(0xffffffffu, cached ? pk[0].x : part_at(0, c).x, 0, 16);
                 double s1 = 0.0, s2 = 0.0;
                 if (cached) {
 #pragma unroll
@@ -1098,7 +1105,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     }
                 } else {
                     for (int64_t k = hl; k < K; k += 16) {
-                        const double2 v = a.part[k * a.C + c];
+                        const double2 v = part_at(k, c);
                         const double w = count_of(k) * (v.x - r);
                         s1 += w;
                         s2 += v.y + w * (v.x - r);
@@ -1134,7 +1141,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     }
                 } else {
                     for (int64_t k = hl; k < K; k += 16) {
-                        const double2 v = a.part[k * a.C + c];
+                        const double2 v = part_at(k, c);
                         s1 += v.x;
                         sy += v.y;
                     }
