@@ -2,9 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one pass of the whole layer over one batch: iabn_forward (x -> z in
-place), iabn_backward (dz -> dx in place, dgamma, dbeta) and
-iabn_update_running_stats, on the ResNet-trunk workload: NHWC bf16 storage,
+One step = one pass of the whole layer over one batch:
+iabn_forward_with_running_stats (x -> z in place, the batch statistics, and
+the running-statistics update in the forward's finalize) and iabn_backward
+(dz -> dx in place, dgamma, dbeta), on the ResNet-trunk workload: NHWC bf16 storage,
 N=64 C=256 H=W=56, leaky-ReLU 0.01.  Inputs are synthetic (seeded, same value
 recipe as the tests) and restored before every step (the layer is in place);
 the L2 cache is flushed (a 2x-L2 write) before every forward and every
@@ -12,7 +13,7 @@ backward call, outside the timed events.
 
 Metric: GB/s of compulsory traffic, 5*E*s bytes per step (the forward reads x
 and writes z; the backward reads z and dz and writes dx), divided by the
-device time of the three calls (CUDA events on the launching stream).  Under
+device time of the two calls (CUDA events on the launching stream).  Under
 torchrun (N > 1) every rank runs its own replica (no cross-GPU statistics):
 value = N * bytes / max-over-ranks time ("weak" scaling).
 
@@ -260,6 +261,15 @@ class Layer:
         self.iabn.update_running_stats(self.mean, self.var, self.rmean, self.rvar,
                                        count=self.sp.per_channel, momentum=self.sp.momentum)
 
+    def fwd_train(self):
+        """The training step's forward: z over x, the batch statistics and the
+        running-statistics update, in one call."""
+        sp = self.sp
+        self.iabn.forward_with_running_stats(self.x, self.gamma, self.beta, self.mean, self.var,
+                                             self.rmean, self.rvar, self.ws, shape=sp.shape,
+                                             layout=sp.layout, eps=sp.eps, act=sp.act,
+                                             act_param=sp.act_param, momentum=sp.momentum)
+
 
 class L2Flush:
     """Evicts the L2 before a timed call: writes a buffer of twice the L2 size,
@@ -289,17 +299,18 @@ class L2Flush:
 
 def timed_layer_steps(layer, flush, steps, warmup, dist_barrier=None, sampler=None):
     """Warm-up, then `steps` timed steps; returns per-step event times (ms) of
-    fwd, bwd and the running-stat update, and the launch count in between."""
+    the forward (with the running-statistics update in its finalize) and the
+    backward, a list of zeros for a separate running update (there is none),
+    and the launch count in between."""
     import torch
     ev = lambda: torch.cuda.Event(enable_timing=True)
     for _ in range(warmup):
         layer.restore()
         flush.zero_()
-        layer.fwd()
+        layer.fwd_train()
         flush.zero_()
         layer.bwd()
-        layer.run()
-    records = [(ev(), ev(), ev(), ev(), ev(), ev()) for _ in range(steps)]
+    records = [(ev(), ev(), ev(), ev()) for _ in range(steps)]
     if dist_barrier:
         dist_barrier()
     torch.cuda.synchronize()
@@ -311,15 +322,12 @@ def timed_layer_steps(layer, flush, steps, warmup, dist_barrier=None, sampler=No
             layer.restore()
             flush.zero_()
             r[0].record()
-            layer.fwd()
+            layer.fwd_train()
             r[1].record()
             flush.zero_()
             r[2].record()
             layer.bwd()
             r[3].record()
-            r[4].record()
-            layer.run()
-            r[5].record()
         if dist_barrier:
             dist_barrier()
         torch.cuda.synchronize()
@@ -327,7 +335,7 @@ def timed_layer_steps(layer, flush, steps, warmup, dist_barrier=None, sampler=No
     launches = layer.iabn.iabn_kernel_launches() - l0
     f = [r[0].elapsed_time(r[1]) for r in records]
     b = [r[2].elapsed_time(r[3]) for r in records]
-    u = [r[4].elapsed_time(r[5]) for r in records]
+    u = [0.0 for _ in records]
     return f, b, u, launches, wall
 
 
@@ -354,9 +362,8 @@ def e2e_steps(layer, steps, warmup):
     def step():
         layer.x.copy_(hx, non_blocking=True)
         layer.dz.copy_(hdz, non_blocking=True)
-        layer.fwd()
+        layer.fwd_train()
         layer.bwd()
-        layer.run()
         hz.copy_(layer.x, non_blocking=True)
         hdx.copy_(layer.dz, non_blocking=True)
         hg.copy_(layer.dgamma, non_blocking=True)
@@ -397,7 +404,7 @@ def drained_steps(layer, flush, steps, warmup):
         r[1].record()
         flush.zero_()
         r[2].record()
-        layer.fwd()
+        layer.fwd_train()
         flush.read_()
         r[3].record()
         flush.zero_()
@@ -405,7 +412,6 @@ def drained_steps(layer, flush, steps, warmup):
         layer.bwd()
         flush.read_()
         r[5].record()
-        layer.run()
         if i >= warmup:
             recs.append(r)
     torch.cuda.synchronize()
@@ -1045,7 +1051,7 @@ def main():
                                "other data (which writes back what the call left dirty), "
                                "minus that read's time on an L2 holding only clean lines"},
             "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
-            "running_update_us": round(statistics.mean(u) * 1e3, 2),
+            "running_update": "in the forward's finalize (iabn_forward_with_running_stats)",
             "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
             "frac_of_hbm_peak": round(value / world / hbm_peak, 4),
             "hbm_peak": {"gbs": hbm_peak,

@@ -112,6 +112,20 @@ iabn_status iabn_forward(const iabn_desc* d, void* x_inout,
                          float* save_mean, float* save_var,
                          void* workspace, size_t ws_bytes, void* stream);
 
+/* iabn_forward and iabn_update_running_stats(C, M, ...) in one call: the
+ * running statistics are updated by the forward's own finalize (the same
+ * fp32 arithmetic, so the same bits as the two calls), which saves the
+ * update's kernel launch.
+ * running_mean, running_var [C] float32, updated in place; momentum in
+ * [0, 1].  Other arguments, errors and the workspace as for iabn_forward. */
+iabn_status iabn_forward_with_running_stats(const iabn_desc* d, void* x_inout,
+                                            const float* gamma, const float* beta, float eps,
+                                            int32_t act, float act_param,
+                                            float* save_mean, float* save_var,
+                                            float* running_mean, float* running_var,
+                                            float momentum,
+                                            void* workspace, size_t ws_bytes, void* stream);
+
 /* Backward from the stored output only ([ABN] section 3, "INPLACE-ABN" and
  * "INPLACE-ABN II"; appendix "Derivation of Gradient dL").
  *   y = phi^-1(z); dy = dz * phi'(y) (phi' read from z);
@@ -209,6 +223,67 @@ iabn_status iabn_checkpoint_recompute(const iabn_desc* d, const void* xhat, void
  * dz_inout  [N,C,H,W]: dL/dz on entry, dL/dx on return; must not overlap xhat.
  * gamma may be zero.  Other arguments and errors as for iabn_backward. */
 iabn_status iabn_backward_checkpoint(const iabn_desc* d, const void* xhat, void* dz_inout,
+                                     const float* gamma, const float* beta,
+                                     const float* save_var, float eps,
+                                     int32_t act, float act_param,
+                                     float* dgamma, float* dbeta,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * INPLACE-ABNsync ([ABN] section 4, "Semantic segmentation": the
+ * segmentation results use synchronised statistics across GPUs).  The batch
+ * is split along N over `world` GPUs; each GPU holds its shard, and the
+ * statistics are those of the whole batch.  Each direction is two calls with
+ * the exchange between them, which the caller does (e.g. one all-gather of
+ * the per-GPU records with NCCL):
+ *   forward:  iabn_sync_forward_stats -> gather the records of all GPUs ->
+ *             iabn_sync_forward_apply;
+ *   backward: iabn_sync_backward_stats -> gather -> iabn_sync_backward_apply.
+ * A record is 3 float64 per channel, record[c*3 + i]:
+ *   forward  (n, mean, M2) of this GPU's values of channel c, M2 = sum (x - mean)^2;
+ *   backward (n, sum dy, sum dy*xhat) over this GPU's values.
+ * `gathered` is [world][C][3] float64 (device memory), the records of GPUs
+ * 0 .. world-1 in rank order; every GPU must pass the same array so that all
+ * of them compute the same statistics (they are combined in rank order in
+ * float64, so they agree bitwise).  With world = 1 the layer is the plain
+ * in-place layer (same arithmetic up to the summation order).
+ * The descriptor of each call is this GPU's shard; shards may differ in N.
+ * ------------------------------------------------------------------------ */
+
+/* This GPU's forward record of x (n = N*H*W of the shard).
+ * x [N,C,H,W]: not modified.  stats [C*3] float64, written. */
+iabn_status iabn_sync_forward_stats(const iabn_desc* d, const void* x, double* stats,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* Combines the gathered forward records into the whole batch's
+ *   mean_c = sum_r n_r mean_r / Mt,  var_c = M2_c / Mt  (Mt = sum_r n_r; biased),
+ * writes save_mean, save_var (the whole batch's) and overwrites x with
+ *   z = phi(gamma_c*(x - mean_c)/sqrt(var_c + eps) + beta_c)
+ * as iabn_forward does.  world >= 1; the records' n must sum to >= 2.
+ * Other arguments as for iabn_forward. */
+iabn_status iabn_sync_forward_apply(const iabn_desc* d, void* x_inout, const double* gathered,
+                                    int32_t world, const float* gamma, const float* beta,
+                                    float eps, int32_t act, float act_param,
+                                    float* save_mean, float* save_var,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* This GPU's backward record from z and dz (y and xhat recovered from z as
+ * iabn_backward does; dy = dz*phi'(y)).  z, dz not modified.  stats [C*3]
+ * float64, written.  gamma, beta, act, act_param as passed to the forward. */
+iabn_status iabn_sync_backward_stats(const iabn_desc* d, const void* z, const void* dz,
+                                     const float* gamma, const float* beta,
+                                     int32_t act, float act_param, double* stats,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Combines the gathered backward records (sums in rank order) into the whole
+ * batch's dbeta_c = sum dy and dgamma_c = sum dy*xhat, writes them, and
+ * overwrites dz with
+ *   dx = gamma_c*rstd*(dy - dbeta_c/Mt - xhat*dgamma_c/Mt),  Mt = sum_r n_r,
+ * rstd = 1/sqrt(save_var_c + eps) (save_var: the whole batch's, from
+ * iabn_sync_forward_apply).  |gamma_c| < FLT_MIN: as for iabn_backward.
+ * Other arguments as for iabn_backward. */
+iabn_status iabn_sync_backward_apply(const iabn_desc* d, const void* z, void* dz_inout,
+                                     const double* gathered, int32_t world,
                                      const float* gamma, const float* beta,
                                      const float* save_var, float eps,
                                      int32_t act, float act_param,

@@ -17,6 +17,11 @@ Two levels:
     ``inference``, ``update_running_stats``, ``workspace_size``,
     ``get_device_status``: the same calls taking torch tensors;
     ``describe_plan``: the launch plan of a call on a descriptor, as a dict.
+  * INPLACE-ABNsync (statistics over a batch split across GPUs):
+    ``sync_forward_stats`` / ``sync_forward_apply``,
+    ``sync_backward_stats`` / ``sync_backward_apply`` (the C calls), and
+    ``forward_sync`` / ``backward_sync``, which put ``gather_records`` (an
+    all-gather over a torch.distributed group) between them.
 """
 from __future__ import annotations
 
@@ -45,11 +50,14 @@ IABN_F32, IABN_BF16, IABN_F16 = 0, 1, 2
 IABN_ACT_LEAKY_RELU, IABN_ACT_ELU, IABN_ACT_IDENTITY = 0, 1, 2
 
 # Symbols include/iabn.h declares (checked by the tests).
-EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_backward",
+EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_forward_with_running_stats",
+           "iabn_backward",
            "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches",
            "iabn_forward_static_ws", "iabn_describe_plan", "iabn_inference",
            "iabn_forward_standard", "iabn_backward_standard", "iabn_forward_checkpoint",
-           "iabn_backward_checkpoint", "iabn_checkpoint_recompute")
+           "iabn_backward_checkpoint", "iabn_checkpoint_recompute",
+           "iabn_sync_forward_stats", "iabn_sync_forward_apply", "iabn_sync_backward_stats",
+           "iabn_sync_backward_apply")
 # Symbols include/iabn_probe.h declares: measurement probes, not the method.
 PROBE_EXPORTS = ("iabn_probe_empty", "iabn_probe_read", "iabn_probe_read_write",
                  "iabn_probe_cluster_occupancy")
@@ -100,6 +108,9 @@ def lib() -> ctypes.CDLL:
             L.iabn_forward.argtypes = [pd, vp, vp, vp, f32, i32, f32, vp, vp, vp,
                                        ctypes.c_size_t, vp]
             L.iabn_forward.restype = i32
+            L.iabn_forward_with_running_stats.argtypes = [pd, vp, vp, vp, f32, i32, f32, vp, vp,
+                                                          vp, vp, f32, vp, ctypes.c_size_t, vp]
+            L.iabn_forward_with_running_stats.restype = i32
             L.iabn_backward.argtypes = [pd, vp, vp, vp, vp, vp, f32, i32, f32, vp, vp, vp,
                                         ctypes.c_size_t, vp]
             L.iabn_backward.restype = i32
@@ -130,6 +141,17 @@ def lib() -> ctypes.CDLL:
             L.iabn_forward_static_ws.restype = i32
             L.iabn_describe_plan.argtypes = [pd, i32, i32, i32, ctypes.POINTER(IabnPlanInfo)]
             L.iabn_describe_plan.restype = i32
+            L.iabn_sync_forward_stats.argtypes = [pd, vp, vp, vp, ctypes.c_size_t, vp]
+            L.iabn_sync_forward_stats.restype = i32
+            L.iabn_sync_forward_apply.argtypes = [pd, vp, vp, i32, vp, vp, f32, i32, f32, vp, vp,
+                                                  vp, ctypes.c_size_t, vp]
+            L.iabn_sync_forward_apply.restype = i32
+            L.iabn_sync_backward_stats.argtypes = [pd, vp, vp, vp, vp, i32, f32, vp, vp,
+                                                   ctypes.c_size_t, vp]
+            L.iabn_sync_backward_stats.restype = i32
+            L.iabn_sync_backward_apply.argtypes = [pd, vp, vp, vp, i32, vp, vp, vp, f32, i32, f32,
+                                                   vp, vp, vp, ctypes.c_size_t, vp]
+            L.iabn_sync_backward_apply.restype = i32
             L.iabn_probe_empty.argtypes = [i32, i32, i32, i32, vp]
             L.iabn_probe_empty.restype = i32
             L.iabn_probe_read.argtypes = [vp, ctypes.c_size_t, i32, vp]
@@ -157,6 +179,15 @@ def iabn_forward(desc, x_inout, gamma, beta, eps, act, act_param, save_mean, sav
                  workspace, ws_bytes, stream) -> int:
     return int(lib().iabn_forward(ctypes.byref(desc), x_inout, gamma, beta, eps, act,
                                   act_param, save_mean, save_var, workspace, ws_bytes, stream))
+
+
+def iabn_forward_with_running_stats(desc, x_inout, gamma, beta, eps, act, act_param, save_mean,
+                                    save_var, running_mean, running_var, momentum, workspace,
+                                    ws_bytes, stream) -> int:
+    return int(lib().iabn_forward_with_running_stats(ctypes.byref(desc), x_inout, gamma, beta,
+                                                     eps, act, act_param, save_mean, save_var,
+                                                     running_mean, running_var, momentum,
+                                                     workspace, ws_bytes, stream))
 
 
 def iabn_backward(desc, z, dz_inout, gamma, beta, save_var, eps, act, act_param, dgamma,
@@ -231,6 +262,31 @@ def iabn_forward_static_ws(desc, x_inout, gamma, beta, eps, act, act_param, save
 def iabn_describe_plan(desc, call, sm_count, smem_optin, info) -> int:
     return int(lib().iabn_describe_plan(ctypes.byref(desc), call, sm_count, smem_optin,
                                         ctypes.byref(info)))
+
+
+def iabn_sync_forward_stats(desc, x, stats, workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_sync_forward_stats(ctypes.byref(desc), x, stats, workspace, ws_bytes,
+                                             stream))
+
+
+def iabn_sync_forward_apply(desc, x_inout, gathered, world, gamma, beta, eps, act, act_param,
+                            save_mean, save_var, workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_sync_forward_apply(ctypes.byref(desc), x_inout, gathered, world, gamma,
+                                             beta, eps, act, act_param, save_mean, save_var,
+                                             workspace, ws_bytes, stream))
+
+
+def iabn_sync_backward_stats(desc, z, dz, gamma, beta, act, act_param, stats, workspace,
+                             ws_bytes, stream) -> int:
+    return int(lib().iabn_sync_backward_stats(ctypes.byref(desc), z, dz, gamma, beta, act,
+                                              act_param, stats, workspace, ws_bytes, stream))
+
+
+def iabn_sync_backward_apply(desc, z, dz_inout, gathered, world, gamma, beta, save_var, eps, act,
+                             act_param, dgamma, dbeta, workspace, ws_bytes, stream) -> int:
+    return int(lib().iabn_sync_backward_apply(ctypes.byref(desc), z, dz_inout, gathered, world,
+                                              gamma, beta, save_var, eps, act, act_param, dgamma,
+                                              dbeta, workspace, ws_bytes, stream))
 
 
 def iabn_probe_empty(blocks, threads, smem_bytes, cooperative, stream) -> int:
@@ -318,6 +374,20 @@ def forward(x, gamma, beta, save_mean, save_var, workspace, *, shape, layout: in
         "iabn_forward")
 
 
+def forward_with_running_stats(x, gamma, beta, save_mean, save_var, running_mean, running_var,
+                               workspace, *, shape, layout: int, eps: float, act: int,
+                               act_param: float, momentum: float, stream=None) -> None:
+    """``forward`` plus the running-statistics update, in the forward's own
+    launch."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    _ok(iabn_forward_with_running_stats(desc, _ptr(x), _ptr(gamma), _ptr(beta), float(eps),
+                                        int(act), float(act_param), _ptr(save_mean),
+                                        _ptr(save_var), _ptr(running_mean), _ptr(running_var),
+                                        float(momentum), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream_ptr(stream)), "iabn_forward_with_running_stats")
+
+
 def backward(z, dz, gamma, beta, save_var, dgamma, dbeta, workspace, *, shape, layout: int,
              eps: float, act: int, act_param: float, stream=None) -> None:
     """dz is overwritten with dx; dgamma and dbeta are written."""
@@ -399,6 +469,98 @@ def update_running_stats(save_mean, save_var, running_mean, running_var, *, coun
                                   _ptr(save_var), _ptr(running_mean), _ptr(running_var),
                                   float(momentum), _stream_ptr(stream)),
         "iabn_update_running_stats")
+
+
+# ------------------------------------------------------------ INPLACE-ABNsync
+# The batch split along N over the ranks of a process group, one GPU each;
+# the statistics are the whole batch's.  Records are float64 tensors of C*3
+# values (see include/iabn.h); `gathered` holds all ranks' records in rank
+# order, shape [world, C*3].
+
+def sync_forward_stats(x, stats, workspace, *, shape, layout: int, stream=None) -> None:
+    """This rank's forward record of its shard x into ``stats`` (float64, C*3)."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    _ok(iabn_sync_forward_stats(desc, _ptr(x), _ptr(stats), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(),
+                                _stream_ptr(stream)), "iabn_sync_forward_stats")
+
+
+def sync_forward_apply(x, gathered, gamma, beta, save_mean, save_var, workspace, *, shape,
+                       layout: int, eps: float, act: int, act_param: float, stream=None) -> None:
+    """x (this rank's shard) is overwritten with z under the whole batch's
+    statistics, which are written to save_mean / save_var."""
+    desc = make_desc(shape, layout, _dtype_code(x))
+    world = gathered.numel() // (3 * int(shape[1]))
+    _ok(iabn_sync_forward_apply(desc, _ptr(x), _ptr(gathered), world, _ptr(gamma), _ptr(beta),
+                                float(eps), int(act), float(act_param), _ptr(save_mean),
+                                _ptr(save_var), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(),
+                                _stream_ptr(stream)), "iabn_sync_forward_apply")
+
+
+def sync_backward_stats(z, dz, gamma, beta, stats, workspace, *, shape, layout: int, act: int,
+                        act_param: float, stream=None) -> None:
+    """This rank's backward record (n, sum dy, sum dy*xhat) into ``stats``."""
+    desc = make_desc(shape, layout, _dtype_code(z))
+    _ok(iabn_sync_backward_stats(desc, _ptr(z), _ptr(dz), _ptr(gamma), _ptr(beta), int(act),
+                                 float(act_param), _ptr(stats), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(),
+                                 _stream_ptr(stream)), "iabn_sync_backward_stats")
+
+
+def sync_backward_apply(z, dz, gathered, gamma, beta, save_var, dgamma, dbeta, workspace, *,
+                        shape, layout: int, eps: float, act: int, act_param: float,
+                        stream=None) -> None:
+    """dz (this rank's shard) is overwritten with dx; dgamma and dbeta (the
+    whole batch's) are written."""
+    desc = make_desc(shape, layout, _dtype_code(z))
+    world = gathered.numel() // (3 * int(shape[1]))
+    _ok(iabn_sync_backward_apply(desc, _ptr(z), _ptr(dz), _ptr(gathered), world, _ptr(gamma),
+                                 _ptr(beta), _ptr(save_var), float(eps), int(act),
+                                 float(act_param), _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(),
+                                 _stream_ptr(stream)), "iabn_sync_backward_apply")
+
+
+def gather_records(stats, group=None):
+    """All ranks' records in rank order, shape [world, numel]: an all-gather
+    over ``group`` (NCCL for CUDA tensors); without an initialised process
+    group, this rank's record alone."""
+    import torch
+    import torch.distributed as dist
+    flat = stats.reshape(-1).contiguous()
+    if not (dist.is_available() and dist.is_initialized()):
+        return flat.reshape(1, -1)
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(flat) for _ in range(world)]
+    dist.all_gather(parts, flat, group=group)
+    return torch.stack(parts)
+
+
+def forward_sync(x, gamma, beta, save_mean, save_var, stats, workspace, *, shape, layout: int,
+                 eps: float, act: int, act_param: float, group=None, stream=None):
+    """INPLACE-ABNsync forward of this rank's shard: record, all-gather,
+    apply.  Returns the gathered records (their n column sums to the whole
+    batch's values per channel, the count for the running statistics)."""
+    sync_forward_stats(x, stats, workspace, shape=shape, layout=layout, stream=stream)
+    gathered = gather_records(stats, group)
+    sync_forward_apply(x, gathered, gamma, beta, save_mean, save_var, workspace, shape=shape,
+                       layout=layout, eps=eps, act=act, act_param=act_param, stream=stream)
+    return gathered
+
+
+def backward_sync(z, dz, gamma, beta, save_var, dgamma, dbeta, stats, workspace, *, shape,
+                  layout: int, eps: float, act: int, act_param: float, group=None,
+                  stream=None):
+    """INPLACE-ABNsync backward of this rank's shard: record, all-gather,
+    apply.  Returns the gathered records."""
+    sync_backward_stats(z, dz, gamma, beta, stats, workspace, shape=shape, layout=layout,
+                        act=act, act_param=act_param, stream=stream)
+    gathered = gather_records(stats, group)
+    sync_backward_apply(z, dz, gathered, gamma, beta, save_var, dgamma, dbeta, workspace,
+                        shape=shape, layout=layout, eps=eps, act=act, act_param=act_param,
+                        stream=stream)
+    return gathered
 
 
 def get_device_status(workspace, stream=None) -> int:

@@ -158,8 +158,8 @@ static iabn_status check_forward(const iabn_desc* d, Geom& g, const void* x, con
                                  bool separate_out, const float* gamma, const float* beta,
                                  float eps, int32_t act, float act_param,
                                  const float* save_mean, const float* save_var,
-                                 const void* workspace, size_t ws_bytes) {
-    iabn_status st = make_geom(d, g);
+                                 const void* workspace, size_t ws_bytes, int64_t min_m = 2) {
+    iabn_status st = make_geom(d, g, min_m);
     if (st != IABN_OK) return st;
     if (!x || !gamma || !beta || !save_mean || !save_var) return IABN_ERR_INVALID_ARG;
     if (separate_out && (!z_out || overlap(g, x, z_out))) return IABN_ERR_INVALID_ARG;
@@ -176,8 +176,9 @@ static iabn_status check_backward(const iabn_desc* d, Geom& g, const void* src, 
                                   const float* gamma, const float* beta, const float* save_var,
                                   float eps, int32_t act, float act_param, const float* dgamma,
                                   const float* dbeta, const void* workspace, size_t ws_bytes,
-                                  bool need_mean = false, const float* save_mean = nullptr) {
-    iabn_status st = make_geom(d, g);
+                                  bool need_mean = false, const float* save_mean = nullptr,
+                                  int64_t min_m = 2) {
+    iabn_status st = make_geom(d, g, min_m);
     if (st != IABN_OK) return st;
     if (!src || !dz || !gamma || !beta || !save_var || !dgamma || !dbeta)
         return IABN_ERR_INVALID_ARG;
@@ -231,6 +232,24 @@ extern "C" iabn_status iabn_forward(const iabn_desc* d, void* x_inout, const flo
     if (st != IABN_OK) return st;
     const FwdArgs a{x_inout, x_inout, nullptr, kModeFwd, kLayerInPlace, gamma, beta, eps,
                     (int)act, act_param, save_mean, save_var};
+    return run_forward(g, a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" iabn_status iabn_forward_with_running_stats(
+    const iabn_desc* d, void* x_inout, const float* gamma, const float* beta, float eps,
+    int32_t act, float act_param, float* save_mean, float* save_var, float* running_mean,
+    float* running_var, float momentum, void* workspace, size_t ws_bytes, void* stream) {
+    if (!running_mean || !running_var) return IABN_ERR_INVALID_ARG;
+    if (!(momentum >= 0.f && momentum <= 1.f)) return IABN_ERR_INVALID_ARG;
+    Geom g;
+    const iabn_status st = check_forward(d, g, x_inout, nullptr, false, gamma, beta, eps, act,
+                                         act_param, save_mean, save_var, workspace, ws_bytes);
+    if (st != IABN_OK) return st;
+    FwdArgs a{x_inout, x_inout, nullptr, kModeFwd, kLayerInPlace, gamma, beta, eps, (int)act,
+              act_param, save_mean, save_var};
+    a.running_mean = running_mean;
+    a.running_var = running_var;
+    a.momentum = momentum;
     return run_forward(g, a, workspace, static_cast<cudaStream_t>(stream));
 }
 
@@ -305,6 +324,88 @@ extern "C" iabn_status iabn_backward_checkpoint(const iabn_desc* d, const void* 
     const BwdArgs a{xhat, dz_inout, kModeBwdXhat, kLayerCkpt, gamma, beta, nullptr, save_var,
                     eps, (int)act, act_param, dgamma, dbeta};
     return run_backward(g, a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------ INPLACE-ABNsync
+// (the shard of one call may hold a single value per channel: M >= 1)
+
+static bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+extern "C" iabn_status iabn_sync_forward_stats(const iabn_desc* d, const void* x, double* stats,
+                                               void* workspace, size_t ws_bytes,
+                                               void* stream) {
+    Geom g;
+    const iabn_status st = make_geom(d, g, 1);
+    if (st != IABN_OK) return st;
+    if (!x || !stats || !aligned8(stats)) return IABN_ERR_INVALID_ARG;
+    if (!aligned16(x)) return IABN_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < workspace_bytes(g) || !aligned16(workspace))
+        return IABN_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
+    return from_cuda(sync_forward_stats(g, x, stats, carve(workspace, g),
+                                        static_cast<cudaStream_t>(stream), device_sms(dev)));
+}
+
+extern "C" iabn_status iabn_sync_forward_apply(const iabn_desc* d, void* x_inout,
+                                               const double* gathered, int32_t world,
+                                               const float* gamma, const float* beta, float eps,
+                                               int32_t act, float act_param, float* save_mean,
+                                               float* save_var, void* workspace,
+                                               size_t ws_bytes, void* stream) {
+    if (!gathered || !aligned8(gathered) || world < 1) return IABN_ERR_INVALID_ARG;
+    Geom g;
+    const iabn_status st = check_forward(d, g, x_inout, nullptr, false, gamma, beta, eps, act,
+                                         act_param, save_mean, save_var, workspace, ws_bytes, 1);
+    if (st != IABN_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
+    const FwdArgs a{x_inout, x_inout, nullptr, kModeFwd, kLayerInPlace, gamma, beta, eps,
+                    (int)act, act_param, save_mean, save_var};
+    return from_cuda(sync_forward_apply(g, a, gathered, (int)world, carve(workspace, g),
+                                        static_cast<cudaStream_t>(stream), device_sms(dev)));
+}
+
+extern "C" iabn_status iabn_sync_backward_stats(const iabn_desc* d, const void* z, const void* dz,
+                                                const float* gamma, const float* beta,
+                                                int32_t act, float act_param, double* stats,
+                                                void* workspace, size_t ws_bytes,
+                                                void* stream) {
+    Geom g;
+    iabn_status st = make_geom(d, g, 1);
+    if (st != IABN_OK) return st;
+    if (!z || !dz || !gamma || !beta || !stats || !aligned8(stats)) return IABN_ERR_INVALID_ARG;
+    if ((st = check_act(act, act_param)) != IABN_OK) return st;
+    if (!aligned16(z) || !aligned16(dz)) return IABN_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < workspace_bytes(g) || !aligned16(workspace))
+        return IABN_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
+    const BwdArgs a{z, const_cast<void*>(dz), kModeBwdZ, kLayerInPlace, gamma, beta, nullptr,
+                    nullptr, 0.f, (int)act, act_param, nullptr, nullptr};
+    return from_cuda(sync_backward_stats(g, a, stats, carve(workspace, g),
+                                         static_cast<cudaStream_t>(stream), device_sms(dev)));
+}
+
+extern "C" iabn_status iabn_sync_backward_apply(const iabn_desc* d, const void* z, void* dz_inout,
+                                                const double* gathered, int32_t world,
+                                                const float* gamma, const float* beta,
+                                                const float* save_var, float eps, int32_t act,
+                                                float act_param, float* dgamma, float* dbeta,
+                                                void* workspace, size_t ws_bytes,
+                                                void* stream) {
+    if (!gathered || !aligned8(gathered) || world < 1) return IABN_ERR_INVALID_ARG;
+    Geom g;
+    const iabn_status st = check_backward(d, g, z, dz_inout, gamma, beta, save_var, eps, act,
+                                          act_param, dgamma, dbeta, workspace, ws_bytes, false,
+                                          nullptr, 1);
+    if (st != IABN_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaErrorNoDevice);
+    const BwdArgs a{z, dz_inout, kModeBwdZ, kLayerInPlace, gamma, beta, nullptr, save_var, eps,
+                    (int)act, act_param, dgamma, dbeta};
+    return from_cuda(sync_backward_apply(g, a, gathered, (int)world, carve(workspace, g),
+                                         static_cast<cudaStream_t>(stream), device_sms(dev)));
 }
 
 extern "C" iabn_status iabn_checkpoint_recompute(const iabn_desc* d, const void* xhat,

@@ -253,6 +253,17 @@ __device__ __forceinline__ void bar_pad(Control* ctl, uint32_t G, uint32_t nbar)
     atomicAdd(&ctl->bar_count, 2u * kBarStride - nbar * G);
 }
 
+// One channel's running statistics step (momentum m, unbias = M/(M-1)):
+//   running_mean <- (1 - m)*running_mean + m*mean,
+//   running_var  <- (1 - m)*running_var + m*var*unbias,
+// in fp32 from the fp32 batch statistics; the standalone update kernel and
+// the forwards that fuse the update share it, so both give the same bits.
+__device__ __forceinline__ void running_step(float* rmean, float* rvar, float mean, float var,
+                                             float m, float unbias) {
+    *rmean = fmaf(m, mean, (1.f - m) * *rmean);
+    *rvar = fmaf(m, var * unbias, (1.f - m) * *rvar);
+}
+
 // ------------------------------------------------ channel of a flat index
 
 // The channel of element i of a flat grid-stride loop, tracked incrementally

@@ -49,6 +49,11 @@ struct FwdArgs {
     float act_param;
     float* save_mean;
     float* save_var;
+    // optional: the running statistics, updated in the finalize with the
+    // arithmetic of running_update (count M); null: not updated
+    float* running_mean = nullptr;
+    float* running_var = nullptr;
+    float momentum = 0.f;
 };
 
 struct BwdArgs {
@@ -97,6 +102,17 @@ cudaError_t recompute_pass(const Geom& g, const void* xhat, void* z, const float
                            int sms);
 cudaError_t forward_apply_pass(const Geom& g, const FwdArgs& f, const float4* coef,
                                cudaStream_t s, int sms);
+// INPLACE-ABNsync (iabn_twophase.cu): this GPU's per-channel record (3
+// doubles per channel), and the apply from the records of all GPUs
+// ([world][C][3], rank order).
+cudaError_t sync_forward_stats(const Geom& g, const void* x, double* rec, const Workspace& w,
+                               cudaStream_t s, int sms);
+cudaError_t sync_forward_apply(const Geom& g, const FwdArgs& a, const double* gathered,
+                               int world, const Workspace& w, cudaStream_t s, int sms);
+cudaError_t sync_backward_stats(const Geom& g, const BwdArgs& a, double* rec,
+                                const Workspace& w, cudaStream_t s, int sms);
+cudaError_t sync_backward_apply(const Geom& g, const BwdArgs& a, const double* gathered,
+                                int world, const Workspace& w, cudaStream_t s, int sms);
 cudaError_t running_update(int64_t C, int64_t count, const float* mean, const float* var,
                            float* rmean, float* rvar, float momentum, cudaStream_t s);
 

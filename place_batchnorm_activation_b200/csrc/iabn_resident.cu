@@ -271,6 +271,10 @@ cudaError_t forward_resident(const Geom& g, const FwdArgs& f, const Workspace& w
     a.var_in = nullptr;
     a.out0 = f.save_mean;
     a.out1 = f.save_var;
+    a.rmean = f.running_mean;
+    a.rvar = f.running_var;
+    a.momentum = f.momentum;
+    a.unbias = (float)(g.M / (double)(g.M - 1));
     a.eps = f.eps;
     a.p = f.act_param;
     a.inv_p = f.act == kIdent ? 1.f : 1.f / f.act_param;
@@ -293,6 +297,8 @@ cudaError_t backward_resident(const Geom& g, const BwdArgs& b, const Workspace& 
     a.var_in = b.save_var;
     a.out0 = b.dgamma;
     a.out1 = b.dbeta;
+    a.rmean = a.rvar = nullptr;
+    a.momentum = a.unbias = 0.f;
     a.eps = b.eps;
     a.p = b.act_param;
     a.inv_p = b.act == kIdent ? 1.f : 1.f / b.act_param;

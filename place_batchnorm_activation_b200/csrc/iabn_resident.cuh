@@ -94,6 +94,9 @@ struct ResArgs {
     const float* var_in;         // backward: saved biased variance
     float* out0;                 // forward: save_mean;  backward: dgamma
     float* out1;                 // forward: save_var;   backward: dbeta
+    float* rmean;                // forward: running statistics to update, or null
+    float* rvar;
+    float momentum, unbias;      // running update: momentum, M/(M-1)
     float eps, p, inv_p;
     Control* ctl;
     double2* part;
@@ -1118,6 +1121,9 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                     const double var = fmax((s2 - s1 * (s1 / a.M)) / a.M, 0.0);
                     a.out0[c] = (float)mean;
                     a.out1[c] = (float)var;
+                    if (a.rmean != nullptr)
+                        running_step(a.rmean + c, a.rvar + c, (float)mean, (float)var,
+                                     a.momentum, a.unbias);
                     const double rstd = 1.0 / sqrt(var + (double)a.eps);
                     const double sc = (double)gmf * rstd;
                     if (CKPT) {

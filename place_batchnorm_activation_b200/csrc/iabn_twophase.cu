@@ -140,6 +140,32 @@ __device__ __forceinline__ double partial_count(int layout, int64_t k, int64_t R
     return (double)HW;
 }
 
+// The batch statistics of channel c and the forward's apply coefficients:
+// record 0 (mean, scale, beta, beta - mean*scale), record 1 (rstd, for the
+// checkpointing forward's xhat).
+// Optionally (rmean != null) the running statistics' step.
+struct RunUpd {
+    float* rmean;
+    float* rvar;
+    float momentum, unbias;
+};
+
+__device__ __forceinline__ void fwd_coef_write(int64_t c, int64_t C, double mean, double var,
+                                               const float* __restrict__ gamma,
+                                               const float* __restrict__ beta, float eps,
+                                               float* __restrict__ save_mean,
+                                               float* __restrict__ save_var,
+                                               float4* __restrict__ coef, const RunUpd& ru) {
+    save_mean[c] = (float)mean;
+    save_var[c] = (float)var;
+    if (ru.rmean != nullptr)
+        running_step(ru.rmean + c, ru.rvar + c, (float)mean, (float)var, ru.momentum, ru.unbias);
+    const double rstd = 1.0 / sqrt(var + (double)eps);
+    const double sc = (double)gamma[c] * rstd;
+    coef[c] = make_float4((float)mean, (float)sc, beta[c], (float)((double)beta[c] - mean * sc));
+    coef[C + c] = make_float4((float)rstd, 0.f, 0.f, 0.f);
+}
+
 // One warp per channel: combine the K partial summaries (count_k, mean_k,
 // M2_k) in fp64 in one pass around r, the first partial's mean:
 //   s1 = sum count_k (mean_k - r),  s2 = sum M2_k + count_k (mean_k - r)^2,
@@ -150,7 +176,7 @@ k_tp_finalize_fwd(const double2* __restrict__ part, int layout, int64_t C, int64
                   int64_t R, int RB, int64_t HW, double M,
                   const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                   float* __restrict__ save_mean, float* __restrict__ save_var,
-                  float4* __restrict__ coef) {
+                  float4* __restrict__ coef, const RunUpd ru) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -169,16 +195,8 @@ k_tp_finalize_fwd(const double2* __restrict__ part, int layout, int64_t C, int64
         s2 = warp_sum(s2);
         const double mean = r + s1 / M;
         const double var = fmax((s2 - s1 * (s1 / M)) / M, 0.0);
-        if (lane == 0) {
-            save_mean[c] = (float)mean;
-            save_var[c] = (float)var;
-            const double rstd = 1.0 / sqrt(var + (double)eps);
-            const double sc = (double)gamma[c] * rstd;
-            // (mean, scale, beta, beta - mean*scale); second record: rstd (the
-            // checkpointing forward's xhat)
-            coef[c] = make_float4((float)mean, (float)sc, beta[c], (float)((double)beta[c] - mean * sc));
-            coef[C + c] = make_float4((float)rstd, 0.f, 0.f, 0.f);
-        }
+        if (lane == 0)
+            fwd_coef_write(c, C, mean, var, gamma, beta, eps, save_mean, save_var, coef, ru);
     }
 }
 
@@ -652,6 +670,42 @@ k_tp_apply_bwd_rows(const uint4* __restrict__ z, uint4* dz, int64_t R, int VC, i
     for (; r >= rt.r0; r -= step) __stcs(pd + r * VC, dx_of(__ldcs(pz + r * VC), __ldcs(pd + r * VC)));
 }
 
+// Channel c's parameter gradients (dbeta = S1, dgamma = S2) and the
+// backward's apply coefficients from the sums over the whole batch of M
+// values (see k_tp_finalize_bwd).
+template <int MODE>
+__device__ __forceinline__ void bwd_coef_write(int64_t c, int64_t C, double s1, double s2,
+                                               double M, const BwdIn& in,
+                                               float* __restrict__ dgamma,
+                                               float* __restrict__ dbeta,
+                                               float4* __restrict__ coef,
+                                               Control* __restrict__ ctl) {
+    const double g = in.gamma[c], b = in.beta[c];
+    const double rstd = 1.0 / sqrt((double)in.var[c] + (double)in.eps);
+    if (MODE != kModeBwdZ) {
+        float xs, xb, ys, yb;
+        src_affine<MODE>(in.gamma[c], in.beta[c], MODE == kModeBwdX ? in.mean[c] : 0.f,
+                         in.var[c], in.eps, xs, xb, ys, yb);
+        const double A = g * rstd, B = -A * s2 / M, Cc = -A * s1 / M;
+        dbeta[c] = (float)s1;
+        dgamma[c] = (float)s2;
+        coef[c] = make_float4(ys, yb, (float)A, 0.f);
+        coef[C + c] = make_float4((float)(B * (double)xs), (float)(B * (double)xb + Cc), 0.f, 0.f);
+    } else if (!(fabs(g) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN (or NaN)
+        atomicOr(&ctl->status, kStSingular);
+        dgamma[c] = __int_as_float(0x7fc00000);
+        dbeta[c] = __int_as_float(0x7fc00000);
+        coef[c] = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                              __int_as_float(0x7fc00000), 0.f);
+    } else {
+        dbeta[c] = (float)s1;
+        dgamma[c] = (float)s2;
+        const double A = g * rstd, B = -rstd * s2 / M;
+        const double Cc = -g * rstd * s1 / M - B * b;
+        coef[c] = make_float4((float)A, (float)B, (float)Cc, 0.f);
+    }
+}
+
 // One warp per channel: S1 = sum dy and S2 = sum dy*xhat summed in fp64;
 // dbeta = S1, dgamma = S2.  The apply coefficients:
 //   in-place: dx in terms of y (the "INPLACE-ABN II" form), one record
@@ -677,31 +731,7 @@ k_tp_finalize_bwd(const double2* __restrict__ part, int64_t C, int64_t K, double
         }
         s1 = warp_sum(s1);
         s2 = warp_sum(s2);
-        if (lane != 0) continue;
-        const double g = in.gamma[c], b = in.beta[c];
-        const double rstd = 1.0 / sqrt((double)in.var[c] + (double)in.eps);
-        if (MODE != kModeBwdZ) {
-            float xs, xb, ys, yb;
-            src_affine<MODE>(in.gamma[c], in.beta[c], MODE == kModeBwdX ? in.mean[c] : 0.f,
-                             in.var[c], in.eps, xs, xb, ys, yb);
-            const double A = g * rstd, B = -A * s2 / M, Cc = -A * s1 / M;
-            dbeta[c] = (float)s1;
-            dgamma[c] = (float)s2;
-            coef[c] = make_float4(ys, yb, (float)A, 0.f);
-            coef[C + c] = make_float4((float)(B * (double)xs), (float)(B * (double)xb + Cc), 0.f, 0.f);
-        } else if (!(fabs(g) >= 1.17549435082228750797e-38)) {   // |gamma| < FLT_MIN (or NaN)
-            atomicOr(&ctl->status, kStSingular);
-            dgamma[c] = __int_as_float(0x7fc00000);
-            dbeta[c] = __int_as_float(0x7fc00000);
-            coef[c] = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
-                                  __int_as_float(0x7fc00000), 0.f);
-        } else {
-            dbeta[c] = (float)s1;
-            dgamma[c] = (float)s2;
-            const double A = g * rstd, B = -rstd * s2 / M;
-            const double Cc = -g * rstd * s1 / M - B * b;
-            coef[c] = make_float4((float)A, (float)B, (float)Cc, 0.f);
-        }
+        if (lane == 0) bwd_coef_write<MODE>(c, C, s1, s2, M, in, dgamma, dbeta, coef, ctl);
     }
 }
 
@@ -793,8 +823,7 @@ __global__ void k_running_update(int64_t C, float unbias, const float* __restric
                                  float* __restrict__ rvar, float m) {
     const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= C) return;
-    rmean[c] = fmaf(m, mean[c], (1.f - m) * rmean[c]);
-    rvar[c] = fmaf(m, var[c] * unbias, (1.f - m) * rvar[c]);
+    running_step(rmean + c, rvar + c, mean[c], var[c], m, unbias);
 }
 
 // ------------------------------------------------------------ host launch
@@ -888,34 +917,32 @@ static RowGrid apply_row_grid(const Geom& g, int blocks) {
     return rg;
 }
 
+// The statistics pass of x: per-block (mean, M2) partials in w.part, K per
+// channel (block partition RB for the row kernels).
 template <int DT>
-static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Workspace& w,
-                                   cudaStream_t s, int sms) {
+static cudaError_t fwd_stats_launch(const Geom& g, const void* xv, const Workspace& w,
+                                    cudaStream_t s, int sms, int64_t& K, int& RB) {
     using T = typename Storage<DT>::T;
-    const T* x = static_cast<const T*>(a.x);
-    int64_t K;
-    int RB = 1;
+    const T* x = static_cast<const T*>(xv);
+    RB = 1;
     if (rows_vectorised(g)) {
         const RowGrid rg = row_grid(g, sms);
         RB = rg.RB;
         k_tp_stats_rows<DT><<<dim3(rg.RB, rg.GY), kRowThreads, 0, s>>>(
-            static_cast<const uint4*>(a.x), g.R, rg.VC, rg.RB, g.C, w.part);
+            static_cast<const uint4*>(xv), g.R, rg.VC, rg.RB, g.C, w.part);
         K = RB;
-        count_launches(1);
     } else if (g.layout == kNHWC) {
         RB = nhwc_row_blocks(g.R);
         const int W = g.C < 256 ? (int)g.C : 256;
         dim3 grid(RB, (unsigned)((g.C + W - 1) / W));
         k_tp_stats_nhwc<DT><<<grid, kTpRowThreads, 0, s>>>(x, g.R, g.C, RB, w.part);
         K = RB;
-        count_launches(1);
     } else if (const int gq = unit_planes(g)) {
         const int64_t units = g.N * g.C / gq;
         k_tp_stats_units<DT><<<(unsigned)((units + 255) / 256), 256, 0, s>>>(
-            static_cast<const uint4*>(a.x), units, (int)(gq * g.HW * g.esize / 16), (int)g.HW,
+            static_cast<const uint4*>(xv), units, (int)(gq * g.HW * g.esize / 16), (int)g.HW,
             w.part);
         K = g.N;
-        count_launches(1);
     } else {
         const int64_t planes = g.N * g.C;
         static std::atomic<int> occ{0};
@@ -923,13 +950,23 @@ static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Worksp
         k_tp_stats_nchw<DT><<<grid_for(planes, 8, sms * per_sm), 256, 0, s>>>(x, planes, g.HW,
                                                                               w.part);
         K = g.N;
-        count_launches(1);
     }
-    cudaError_t e = cudaGetLastError();
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <int DT>
+static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Workspace& w,
+                                   cudaStream_t s, int sms) {
+    int64_t K = 0;
+    int RB = 1;
+    cudaError_t e = fwd_stats_launch<DT>(g, a.x, w, s, sms, K, RB);
     if (e != cudaSuccess) return e;
     k_tp_finalize_fwd<<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
         w.part, g.layout, g.C, K, g.R, RB, g.HW, (double)g.M, a.gamma, a.beta, a.eps,
-        a.save_mean, a.save_var, w.coef);
+        a.save_mean, a.save_var, w.coef,
+        RunUpd{a.running_mean, a.running_var, a.momentum,
+               (float)(g.M / (double)(g.M - 1))});
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -946,24 +983,21 @@ cudaError_t forward_twophase(const Geom& g, const FwdArgs& a, const Workspace& w
     }
 }
 
+// The reduction pass of the backward: per-block (S1, S2) partials in w.part,
+// K per channel.
 template <int DT, int ACT, int MODE>
-static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Workspace& w,
-                                     cudaStream_t s, int sms) {
+static cudaError_t bwd_reduce_launch(const Geom& g, const void* src, const void* dzv,
+                                     const BwdIn& in, const Workspace& w, cudaStream_t s,
+                                     int sms, int64_t& K) {
     using T = typename Storage<DT>::T;
-    const T* z = static_cast<const T*>(a.src);
-    T* dz = static_cast<T*>(a.dz);
-    const float p = a.act_param;
-    const float inv_p = ACT == kIdent ? 1.f : 1.f / p;
-    const BwdIn in{a.gamma, a.beta, a.save_mean, a.save_var, a.eps, p, inv_p};
-    int64_t K;
-    const bool rows = rows_vectorised(g);
-    const RowGrid rg = rows ? row_grid(g, sms) : RowGrid{};
-    if (rows) {
+    const T* z = static_cast<const T*>(src);
+    const T* dz = static_cast<const T*>(dzv);
+    if (rows_vectorised(g)) {
+        const RowGrid rg = row_grid(g, sms);
         k_tp_reduce_rows<DT, ACT, MODE><<<dim3(rg.RB, rg.GY), kRowThreads, 0, s>>>(
-            static_cast<const uint4*>(a.src), static_cast<const uint4*>(a.dz), g.R, rg.VC, rg.RB,
+            static_cast<const uint4*>(src), static_cast<const uint4*>(dzv), g.R, rg.VC, rg.RB,
             g.C, in, w.part);
         K = rg.RB;
-        count_launches(1);
     } else if (g.layout == kNHWC) {
         const int RB = nhwc_row_blocks(g.R);
         const int W = g.C < 256 ? (int)g.C : 256;
@@ -971,14 +1005,12 @@ static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Work
         k_tp_reduce_nhwc<DT, ACT, MODE><<<grid, kTpRowThreads, 0, s>>>(z, dz, g.R, g.C, RB, in,
                                                                        w.part);
         K = RB;
-        count_launches(1);
     } else if (const int gq = unit_planes(g)) {
         const int64_t units = g.N * g.C / gq;
         k_tp_reduce_units<DT, ACT, MODE><<<(unsigned)((units + 255) / 256), 256, 0, s>>>(
-            static_cast<const uint4*>(a.src), static_cast<const uint4*>(a.dz), units,
+            static_cast<const uint4*>(src), static_cast<const uint4*>(dzv), units,
             (int)(gq * g.HW * g.esize / 16), (int)g.HW, g.C, in, w.part);
         K = g.N;
-        count_launches(1);
     } else {
         const int64_t planes = g.N * g.C;
         static std::atomic<int> occ{0};
@@ -986,21 +1018,25 @@ static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Work
         k_tp_reduce_nchw<DT, ACT, MODE><<<grid_for(planes, 8, sms * per_sm), 256, 0, s>>>(
             z, dz, planes, g.C, g.HW, in, w.part);
         K = g.N;
-        count_launches(1);
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    k_tp_finalize_bwd<MODE><<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
-        w.part, g.C, K, (double)g.M, in, a.dgamma, a.dbeta, w.coef, w.ctl);
     count_launches(1);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if (rows) {
+    return cudaGetLastError();
+}
+
+// The backward's elementwise pass: dx over dz from the records in w.coef.
+template <int DT, int ACT, int MODE>
+static cudaError_t bwd_apply_launch(const Geom& g, const void* src, void* dzv,
+                                    const Workspace& w, float p, float inv_p, cudaStream_t s,
+                                    int sms) {
+    using T = typename Storage<DT>::T;
+    const T* z = static_cast<const T*>(src);
+    T* dz = static_cast<T*>(dzv);
+    if (rows_vectorised(g)) {
         auto kern = k_tp_apply_bwd_rows<DT, ACT, MODE>;
         static std::atomic<int> occ{0};
         const RowGrid ag = apply_row_grid(g, sms * ctas_per_sm(kern, kApplyThreads, occ));
         kern<<<dim3(ag.RB, ag.GY), kApplyThreads, 0, s>>>(
-            static_cast<const uint4*>(a.src), static_cast<uint4*>(a.dz), g.R, ag.VC, ag.RB, g.C,
+            static_cast<const uint4*>(src), static_cast<uint4*>(dzv), g.R, ag.VC, ag.RB, g.C,
             w.coef, p, inv_p);
     } else if (g.layout == kNHWC) {
         k_tp_apply_bwd<DT, ACT, kNHWC, MODE><<<grid_for(g.E, 256, sms * 8), 256, 0, s>>>(
@@ -1013,6 +1049,23 @@ static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Work
     }
     count_launches(1);
     return cudaGetLastError();
+}
+
+template <int DT, int ACT, int MODE>
+static cudaError_t bwd_twophase_mode(const Geom& g, const BwdArgs& a, const Workspace& w,
+                                     cudaStream_t s, int sms) {
+    const float p = a.act_param;
+    const float inv_p = ACT == kIdent ? 1.f : 1.f / p;
+    const BwdIn in{a.gamma, a.beta, a.save_mean, a.save_var, a.eps, p, inv_p};
+    int64_t K = 0;
+    cudaError_t e = bwd_reduce_launch<DT, ACT, MODE>(g, a.src, a.dz, in, w, s, sms, K);
+    if (e != cudaSuccess) return e;
+    k_tp_finalize_bwd<MODE><<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
+        w.part, g.C, K, (double)g.M, in, a.dgamma, a.dbeta, w.coef, w.ctl);
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return bwd_apply_launch<DT, ACT, MODE>(g, a.src, a.dz, w, p, inv_p, s, sms);
 }
 
 template <int DT, int ACT>
@@ -1042,6 +1095,203 @@ cudaError_t backward_twophase(const Geom& g, const BwdArgs& a, const Workspace& 
     case kBF16: return bwd_twophase_dt<kBF16>(g, a, w, s, sms);
     default: return bwd_twophase_dt<kF16>(g, a, w, s, sms);
     }
+}
+
+// ------------------------------------------------------------ INPLACE-ABNsync
+// The layer's statistics over a batch split along N across GPUs: each GPU
+// reduces its shard to one record per channel, the caller gathers the
+// records of all GPUs, and each GPU combines them in rank order (fp64) and
+// applies the result to its shard.  Records are 3 doubles per channel:
+// forward (n, mean, M2), backward (n, sum dy, sum dy*xhat).
+
+// This GPU's forward record: the K block partials combined as
+// k_tp_finalize_fwd does.
+__global__ void __launch_bounds__(256)
+k_sync_record_fwd(const double2* __restrict__ part, int layout, int64_t C, int64_t K,
+                  int64_t R, int RB, int64_t HW, double M, double* __restrict__ rec) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t c = gw; c < C; c += nw) {
+        const double r = part[c].x;
+        double s1 = 0.0, s2 = 0.0;
+        for (int64_t k = lane; k < K; k += 32) {
+            const double2 pk = part[k * C + c];
+            const double d = pk.x - r;
+            const double w = partial_count(layout, k, R, RB, HW) * d;
+            s1 += w;
+            s2 += pk.y + w * d;
+        }
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        if (lane == 0) {
+            rec[c * 3] = M;
+            rec[c * 3 + 1] = r + s1 / M;
+            rec[c * 3 + 2] = fmax(s2 - s1 * (s1 / M), 0.0);
+        }
+    }
+}
+
+// The whole batch's statistics from the gathered forward records, one pass in
+// rank order around rank 0's mean r:
+//   Mt = sum n_k,  s1 = sum n_k (mean_k - r),  s2 = sum M2_k + n_k (mean_k - r)^2,
+//   mean = r + s1/Mt,  var = (s2 - s1^2/Mt)/Mt;
+// then the forward's apply coefficients.
+__global__ void __launch_bounds__(256)
+k_sync_finalize_fwd(const double* __restrict__ gathered, int world, int64_t C,
+                    const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                    float* __restrict__ save_mean, float* __restrict__ save_var,
+                    float4* __restrict__ coef, float* __restrict__ rmean,
+                    float* __restrict__ rvar, float momentum) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < C; c += stride) {
+        const double r = gathered[c * 3 + 1];
+        double n = 0.0, s1 = 0.0, s2 = 0.0;
+        for (int k = 0; k < world; ++k) {
+            const double* q = gathered + ((int64_t)k * C + c) * 3;
+            const double d = q[1] - r;
+            n += q[0];
+            s1 += q[0] * d;
+            s2 += q[2] + q[0] * d * d;
+        }
+        const double mean = r + s1 / n;
+        const double var = fmax((s2 - s1 * (s1 / n)) / n, 0.0);
+        // the running statistics' count is the whole batch's
+        fwd_coef_write(c, C, mean, var, gamma, beta, eps, save_mean, save_var, coef,
+                       RunUpd{rmean, rvar, momentum, (float)(n / (n - 1.0))});
+    }
+}
+
+// This GPU's backward record: the K block partials summed per channel.
+__global__ void __launch_bounds__(256)
+k_sync_record_bwd(const double2* __restrict__ part, int64_t C, int64_t K, double M,
+                  double* __restrict__ rec) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t c = gw; c < C; c += nw) {
+        double s1 = 0.0, s2 = 0.0;
+        for (int64_t k = lane; k < K; k += 32) {
+            const double2 pk = part[k * C + c];
+            s1 += pk.x;
+            s2 += pk.y;
+        }
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        if (lane == 0) {
+            rec[c * 3] = M;
+            rec[c * 3 + 1] = s1;
+            rec[c * 3 + 2] = s2;
+        }
+    }
+}
+
+// The whole batch's sums from the gathered backward records (rank order),
+// then the parameter gradients and the backward's apply coefficients.
+template <int MODE>
+__global__ void __launch_bounds__(256)
+k_sync_finalize_bwd(const double* __restrict__ gathered, int world, int64_t C, const BwdIn in,
+                    float* __restrict__ dgamma, float* __restrict__ dbeta,
+                    float4* __restrict__ coef, Control* __restrict__ ctl) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < C; c += stride) {
+        double n = 0.0, s1 = 0.0, s2 = 0.0;
+        for (int k = 0; k < world; ++k) {
+            const double* q = gathered + ((int64_t)k * C + c) * 3;
+            n += q[0];
+            s1 += q[1];
+            s2 += q[2];
+        }
+        bwd_coef_write<MODE>(c, C, s1, s2, n, in, dgamma, dbeta, coef, ctl);
+    }
+}
+
+template <int DT>
+static cudaError_t sync_fwd_stats_dt(const Geom& g, const void* x, double* rec,
+                                     const Workspace& w, cudaStream_t s, int sms) {
+    int64_t K = 0;
+    int RB = 1;
+    cudaError_t e = fwd_stats_launch<DT>(g, x, w, s, sms, K, RB);
+    if (e != cudaSuccess) return e;
+    k_sync_record_fwd<<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(
+        w.part, g.layout, g.C, K, g.R, RB, g.HW, (double)g.M, rec);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t sync_forward_stats(const Geom& g, const void* x, double* rec, const Workspace& w,
+                               cudaStream_t s, int sms) {
+    switch (g.dtype) {
+    case kF32: return sync_fwd_stats_dt<kF32>(g, x, rec, w, s, sms);
+    case kBF16: return sync_fwd_stats_dt<kBF16>(g, x, rec, w, s, sms);
+    default: return sync_fwd_stats_dt<kF16>(g, x, rec, w, s, sms);
+    }
+}
+
+cudaError_t sync_forward_apply(const Geom& g, const FwdArgs& a, const double* gathered,
+                               int world, const Workspace& w, cudaStream_t s, int sms) {
+    k_sync_finalize_fwd<<<(unsigned)((g.C + 255) / 256), 256, 0, s>>>(
+        gathered, world, g.C, a.gamma, a.beta, a.eps, a.save_mean, a.save_var, w.coef,
+        a.running_mean, a.running_var, a.momentum);
+    count_launches(1);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return forward_apply_pass(g, a, w.coef, s, sms);
+}
+
+template <int DT, int ACT>
+static cudaError_t sync_bwd_act(const Geom& g, const BwdArgs& a, double* rec,
+                                const double* gathered, int world, const Workspace& w,
+                                cudaStream_t s, int sms) {
+    const float p = a.act_param;
+    const float inv_p = ACT == kIdent ? 1.f : 1.f / p;
+    const BwdIn in{a.gamma, a.beta, nullptr, a.save_var, a.eps, p, inv_p};
+    if (rec != nullptr) {
+        int64_t K = 0;
+        cudaError_t e = bwd_reduce_launch<DT, ACT, kModeBwdZ>(g, a.src, a.dz, in, w, s, sms, K);
+        if (e != cudaSuccess) return e;
+        k_sync_record_bwd<<<grid_for(g.C, 8, sms * 16), 256, 0, s>>>(w.part, g.C, K,
+                                                                      (double)g.M, rec);
+        count_launches(1);
+        return cudaGetLastError();
+    }
+    k_sync_finalize_bwd<kModeBwdZ><<<(unsigned)((g.C + 255) / 256), 256, 0, s>>>(
+        gathered, world, g.C, in, a.dgamma, a.dbeta, w.coef, w.ctl);
+    count_launches(1);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return bwd_apply_launch<DT, ACT, kModeBwdZ>(g, a.src, a.dz, w, p, inv_p, s, sms);
+}
+
+template <int DT>
+static cudaError_t sync_bwd_dt(const Geom& g, const BwdArgs& a, double* rec,
+                               const double* gathered, int world, const Workspace& w,
+                               cudaStream_t s, int sms) {
+    switch (a.act) {
+    case kLeaky: return sync_bwd_act<DT, kLeaky>(g, a, rec, gathered, world, w, s, sms);
+    case kElu: return sync_bwd_act<DT, kElu>(g, a, rec, gathered, world, w, s, sms);
+    default: return sync_bwd_act<DT, kIdent>(g, a, rec, gathered, world, w, s, sms);
+    }
+}
+
+static cudaError_t sync_bwd(const Geom& g, const BwdArgs& a, double* rec,
+                            const double* gathered, int world, const Workspace& w,
+                            cudaStream_t s, int sms) {
+    switch (g.dtype) {
+    case kF32: return sync_bwd_dt<kF32>(g, a, rec, gathered, world, w, s, sms);
+    case kBF16: return sync_bwd_dt<kBF16>(g, a, rec, gathered, world, w, s, sms);
+    default: return sync_bwd_dt<kF16>(g, a, rec, gathered, world, w, s, sms);
+    }
+}
+
+cudaError_t sync_backward_stats(const Geom& g, const BwdArgs& a, double* rec,
+                                const Workspace& w, cudaStream_t s, int sms) {
+    return sync_bwd(g, a, rec, nullptr, 0, w, s, sms);
+}
+
+cudaError_t sync_backward_apply(const Geom& g, const BwdArgs& a, const double* gathered,
+                                int world, const Workspace& w, cudaStream_t s, int sms) {
+    return sync_bwd(g, a, nullptr, gathered, world, w, s, sms);
 }
 
 cudaError_t running_update(int64_t C, int64_t count, const float* mean, const float* var,

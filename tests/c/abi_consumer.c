@@ -77,6 +77,23 @@ int main(void) {
     printf("recompute_null_xhat %d\n",
            (int)iabn_checkpoint_recompute(&trunk, NULL, dummy, dummy, dummy,
                                           IABN_ACT_LEAKY_RELU, 0.01f, NULL));
+    printf("forward_running_null_rmean %d\n",
+           (int)iabn_forward_with_running_stats(&trunk, dummy, dummy, dummy, 1e-5f,
+                                                IABN_ACT_LEAKY_RELU, 0.01f, dummy, dummy, NULL,
+                                                dummy, 0.1f, NULL, 0, NULL));
+    printf("sync_forward_stats_null_stats %d\n",
+           (int)iabn_sync_forward_stats(&trunk, dummy, NULL, dummy, 1 << 30, NULL));
+    printf("sync_forward_apply_bad_world %d\n",
+           (int)iabn_sync_forward_apply(&trunk, dummy, (const double*)dummy, 0, dummy, dummy,
+                                        1e-5f, IABN_ACT_LEAKY_RELU, 0.01f, dummy, dummy, dummy,
+                                        (size_t)1 << 30, NULL));
+    printf("sync_backward_stats_bad_act %d\n",
+           (int)iabn_sync_backward_stats(&trunk, dummy, dummy, dummy, dummy, 7, 0.01f,
+                                         (double*)dummy, dummy, (size_t)1 << 30, NULL));
+    printf("sync_backward_apply_null_gathered %d\n",
+           (int)iabn_sync_backward_apply(&trunk, dummy, dummy + 2, NULL, 2, dummy, dummy, dummy,
+                                         1e-5f, IABN_ACT_LEAKY_RELU, 0.01f, dummy, dummy, dummy,
+                                         (size_t)1 << 30, NULL));
     printf("running_bad_count %d\n",
            (int)iabn_update_running_stats(256, 1, dummy, dummy, dummy, dummy, 0.1f, NULL));
     printf("status_null_ws %d\n", (int)iabn_get_device_status(NULL, NULL));

@@ -62,7 +62,10 @@ def test_c_consumer_matches_the_binding(tmp_path, compiler, flags, monkeypatch):
     assert int(got["describe_bad_call"]) == iabn.IABN_ERR_INVALID_ARG
     for k in ("forward_standard_null_z", "backward_standard_null_mean",
               "forward_checkpoint_bad_eps", "backward_checkpoint_bad_desc",
-              "recompute_null_xhat"):
+              "recompute_null_xhat", "sync_forward_stats_null_stats",
+              "forward_running_null_rmean",
+              "sync_forward_apply_bad_world", "sync_backward_stats_bad_act",
+              "sync_backward_apply_null_gathered"):
         assert int(got[k]) == iabn.IABN_ERR_INVALID_ARG, k
     assert int(got["forward_null_x"]) == iabn.IABN_ERR_INVALID_ARG
     assert int(got["backward_bad_desc"]) == iabn.IABN_ERR_INVALID_ARG

@@ -242,3 +242,39 @@ def test_tmem_stash_bitwise(case, monkeypatch):
         np.testing.assert_array_equal(a, b)
     monkeypatch.setenv("IABN_TMEM_STASH", "1")
     check_layer(inp, oracle_expect(inp), "resident", running=False)
+
+
+FUSED_RUNNING = [
+    wl.spec(0),
+    wl.LayerSpec("fused_running_nhwc", 8, 64, 28, 28, wl.NHWC, wl.BF16, wl.LEAKY_RELU, 0.01,
+                 seed=20180640),
+    wl.LayerSpec("fused_running_nchw", 6, 32, 7, 7, wl.NCHW, wl.F16, wl.ELU, 1.0,
+                 seed=20180641),
+]
+
+
+@pytest.mark.parametrize("plan", PLANS)
+@pytest.mark.parametrize("sp", FUSED_RUNNING, ids=lambda s: s.name)
+def test_forward_with_running_stats(sp, plan):
+    """The forward that updates the running statistics in its own finalize
+    gives the bits of iabn_forward followed by iabn_update_running_stats, and
+    the oracle's running update."""
+    import place_batchnorm_activation_b200 as iabn
+    inp = wl.draw(sp)
+    exp = oracle_expect(inp)
+    with forced_plan(plan):
+        a, b = GpuLayer(inp), GpuLayer(inp)
+        a.forward()
+        a.running()
+        iabn.forward_with_running_stats(b.x, b.gamma, b.beta, b.mean, b.var, b.rmean, b.rvar,
+                                        b.ws, shape=sp.shape, layout=sp.layout, eps=sp.eps,
+                                        act=sp.act, act_param=sp.act_param,
+                                        momentum=sp.momentum)
+        b.check_guards("forward with running statistics")
+    torch.cuda.synchronize()
+    for name in ("x", "mean", "var", "rmean", "rvar"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    tol = TOL[sp.dtype]
+    compare(b.rmean.cpu().numpy(), exp["running_mean"], tol, f"{sp.name} fused running_mean")
+    compare(b.rvar.cpu().numpy(), exp["running_var"], tol, f"{sp.name} fused running_var")
+    assert b.status() == 0
