@@ -39,15 +39,16 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # DRAM bytes per launch (dram__bytes_read.sum, dram__bytes_write.sum) of the
 # resident kernels on the ResNet-trunk layer, from one ncu capture:
 #   python bench.py --profile 1 --steps 1 --warmup 1
-#   ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum \
+#   ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,\
+#   lts__t_sector_hit_rate.pct,dram__throughput.avg.pct_of_peak_sustained_elapsed \
 #       --clock-control none -k regex:k_resident -s 2 -c 2 --csv \
 #       python bench.py --profile 1 --steps 1 --warmup 1
 # Reported only while the CUDA sources hash to the value they were captured
 # on; otherwise "traffic" and "dram_bytes" are null.
 NCU_TRAFFIC = {
-    "sources_sha256": "12dc261b5b714a43a82074d78278cdff307fea806943802f38b1400834dc3ec7",
-    "backward": {"read": 287629824, "write": 37336064},
-    "forward": {"read": 110013440, "write": 22978560},
+    "sources_sha256": "f534cde10cf83cdfe82c1e3a7722bbac2cb49a369b04e090b922d00fb13f9700",
+    "backward": {"read": 287367936, "write": 33791744},
+    "forward": {"read": 109641728, "write": 22854912},
 }
 # the resident kernels' phase trace in the workspace (IABN_TRACE=1): up to 256
 # CTAs x 16 slots of 8 bytes, right after the 256-byte control block
@@ -348,39 +349,75 @@ class _Null:
 
 
 def e2e_steps(layer, steps, warmup):
-    """Through the public API with host buffers: pinned host x, dz -> device,
-    forward, backward, running stats, z and dx (and dgamma, dbeta) -> host.
-    Returns per-step ms and bytes moved each way."""
+    """Through the public API with host buffers, every step: pinned host x and
+    dz -> device, the forward (with the running-statistics update) and the
+    backward, z and dx (and dgamma, dbeta) -> host.  Copies and compute run on
+    three streams over two device buffer sets, so step i+1's host-to-device
+    copies overlap step i's kernels and device-to-host copies (PCIe carries
+    both directions at once), and z goes back while the backward reads it.
+    Returns per-step ms (the whole run's device time over the steps) and the
+    bytes moved each way per step."""
     import torch
+    sp = layer.sp
     hx = layer.x0.cpu().pin_memory()
     hdz = layer.dz0.cpu().pin_memory()
     hz = torch.empty_like(hx).pin_memory()
     hdx = torch.empty_like(hdz).pin_memory()
     hg = torch.empty_like(layer.dgamma, device="cpu").pin_memory()
     hb = torch.empty_like(layer.dbeta, device="cpu").pin_memory()
+    dev = layer.x.device
+    slots = [dict(x=layer.x, dz=layer.dz, dg=layer.dgamma, db=layer.dbeta),
+             dict(x=torch.empty_like(layer.x), dz=torch.empty_like(layer.dz),
+                  dg=torch.empty_like(layer.dgamma), db=torch.empty_like(layer.dbeta))]
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    freed = [None, None]   # event: the slot's device-to-host copies are done
+    kw = dict(shape=sp.shape, layout=sp.layout, eps=sp.eps, act=sp.act, act_param=sp.act_param)
 
-    def step():
-        layer.x.copy_(hx, non_blocking=True)
-        layer.dz.copy_(hdz, non_blocking=True)
-        layer.fwd_train()
-        layer.bwd()
-        hz.copy_(layer.x, non_blocking=True)
-        hdx.copy_(layer.dz, non_blocking=True)
-        hg.copy_(layer.dgamma, non_blocking=True)
-        hb.copy_(layer.dbeta, non_blocking=True)
+    def step(i):
+        k = slots[i % 2]
+        with torch.cuda.stream(s_in):
+            if freed[i % 2] is not None:
+                s_in.wait_event(freed[i % 2])
+            k["x"].copy_(hx, non_blocking=True)
+            x_in = ev()
+            x_in.record(s_in)
+            k["dz"].copy_(hdz, non_blocking=True)
+            dz_in = ev()
+            dz_in.record(s_in)
+        s_run.wait_event(x_in)
+        layer.iabn.forward_with_running_stats(k["x"], layer.gamma, layer.beta, layer.mean,
+                                              layer.var, layer.rmean, layer.rvar, layer.ws,
+                                              momentum=sp.momentum, stream=s_run, **kw)
+        fwd_done = ev()
+        fwd_done.record(s_run)
+        s_run.wait_event(dz_in)
+        layer.iabn.backward(k["x"], k["dz"], layer.gamma, layer.beta, layer.var, k["dg"],
+                            k["db"], layer.ws, stream=s_run, **kw)
+        bwd_done = ev()
+        bwd_done.record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(fwd_done)
+            hz.copy_(k["x"], non_blocking=True)      # z, while the backward reads it
+            s_out.wait_event(bwd_done)
+            hdx.copy_(k["dz"], non_blocking=True)
+            hg.copy_(k["dg"], non_blocking=True)
+            hb.copy_(k["db"], non_blocking=True)
+            freed[i % 2] = ev()
+            freed[i % 2].record(s_out)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
-    times = []
-    for _ in range(steps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        step()
-        b.record()
-        times.append((a, b))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    for i in range(warmup, warmup + steps):
+        step(i)
+    s_in.wait_stream(s_out)
+    s_in.wait_stream(s_run)
+    t1.record(s_in)
     torch.cuda.synchronize()
-    ms = [a.elapsed_time(b) for a, b in times]
+    ms = [t0.elapsed_time(t1) / steps] * steps
     h2d = hx.numel() * hx.element_size() + hdz.numel() * hdz.element_size()
     d2h = (hz.numel() * hz.element_size() + hdx.numel() * hdx.element_size()
            + hg.numel() * 4 + hb.numel() * 4)
@@ -654,6 +691,55 @@ def bench_twophase(flush, steps, warmup, hbm_peak, device):
             "frac_hbm_peak": round(gbs / hbm_peak, 4),
             "launches_per_step": launches / max(1, steps),
             "plan": "IABN_FORCE_PLAN=twophase"}
+
+
+def bench_sync(flush, steps, warmup, hbm_peak, device):
+    """INPLACE-ABNsync on the ResNet-trunk layer with one rank: the record
+    and apply calls of each direction through the C ABI, with the GPU's own
+    record as the gathered array (with more GPUs an all-gather of 24*C bytes
+    per GPU sits between the two calls); L2 flushed before each direction,
+    x and dz restored between steps, outside the timed events."""
+    import torch
+    import workloads as wl
+    sp = wl.spec(1)
+    L = Layer(sp, sp.seed, device)
+    iabn = L.iabn
+    rec = torch.empty(sp.c * 3, dtype=torch.float64, device=device)
+    kw = dict(shape=sp.shape, layout=sp.layout)
+    act = dict(eps=sp.eps, act=sp.act, act_param=sp.act_param)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    recs = []
+    l0 = iabn.iabn_kernel_launches()
+    for i in range(warmup + steps):
+        L.restore()
+        r = [ev() for _ in range(4)]
+        flush.zero_()
+        r[0].record()
+        iabn.sync_forward_stats(L.x, rec, L.ws, **kw)
+        iabn.sync_forward_apply(L.x, rec.view(1, -1), L.gamma, L.beta, L.mean, L.var, L.ws,
+                                **kw, **act)
+        r[1].record()
+        flush.zero_()
+        r[2].record()
+        iabn.sync_backward_stats(L.x, L.dz, L.gamma, L.beta, rec, L.ws, **kw, act=sp.act,
+                                 act_param=sp.act_param)
+        iabn.sync_backward_apply(L.x, L.dz, rec.view(1, -1), L.gamma, L.beta, L.var, L.dgamma,
+                                 L.dbeta, L.ws, **kw, **act)
+        r[3].record()
+        if i >= warmup:
+            recs.append(r)
+    torch.cuda.synchronize()
+    launches = (iabn.iabn_kernel_launches() - l0) / (warmup + steps)
+    tf = statistics.median(r[0].elapsed_time(r[1]) for r in recs)
+    tb = statistics.median(r[2].elapsed_time(r[3]) for r in recs)
+    gbs = L.bytes / ((tf + tb) * 1e-3) / 1e9
+    del L
+    torch.cuda.empty_cache()
+    return {"fwd_us": round(tf * 1e3, 2), "bwd_us": round(tb * 1e3, 2), "gbs": round(gbs, 1),
+            "frac_hbm_peak": round(gbs / hbm_peak, 4), "launches_per_step": launches,
+            "world": 1,
+            "plan": "record call (two-phase statistics / reduce kernel + record kernel), "
+                    "apply call (rank-order combine + elementwise pass), per direction"}
 
 
 # ------------------------------------------------------------ CPU (oracle)
@@ -999,7 +1085,7 @@ def main():
     d_ms = reduce_max(df + db + statistics.mean(u), world, device)
 
     # e2e through host buffers
-    e_ms, h2d, d2h = e2e_steps(layer, max(3, args.steps // 10), 2)
+    e_ms, h2d, d2h = e2e_steps(layer, max(5, args.steps // 5), 2)
     e_max = reduce_max(statistics.mean(e_ms), world, device)
     e2e_value = whole_job_gbs(layer.bytes, world, e_max)
 
@@ -1016,6 +1102,11 @@ def main():
                                                             hbm_peak, device)
         except Exception as e:
             extra["twophase_resnet_trunk"] = {"error": f"{type(e).__name__}: {e}"}
+        try:
+            extra["sync_resnet_trunk"] = bench_sync(flush, max(5, args.steps // 5), 3, hbm_peak,
+                                                    device)
+        except Exception as e:
+            extra["sync_resnet_trunk"] = {"error": f"{type(e).__name__}: {e}"}
         try:
             extra["layers_vs_standard"] = bench_layer_variants(flush, max(5, args.steps // 5), 3,
                                                                device)
@@ -1072,7 +1163,10 @@ def main():
                              "dram_bytes": ncu_dram("forward"),
                              "algorithmic_bytes_per_launch": 2 * sp.numel * sp.itemsize},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e_max, 3)},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e_max, 3),
+                    "how": "public API, pinned host buffers; host-to-device copies, kernels "
+                           "and device-to-host copies on three streams over two device "
+                           "buffer sets (step i+1's copies overlap step i)"},
             "gpu_launches": int(launches),
             "clocks": sampler.summary(),
             "timed_wall_s": round(wall, 4),
