@@ -403,11 +403,20 @@ iabn_status iabn_describe_plan(const iabn_desc* d, int32_t call, int32_t sm_coun
  *     GPU (other streams, other host threads) race and give wrong results.
  *     Each call zeroes the array's control block on `stream` before its
  *     kernels, so device-side conditions of one call (a bounded wait that ran
- *     out) are not carried into the next and cannot be read back. */
+ *     out) are not carried into the next; iabn_get_static_ws_status reads
+ *     them after the call. */
 iabn_status iabn_forward_static_ws(const iabn_desc* d, void* x_inout,
                                    const float* gamma, const float* beta, float eps,
                                    int32_t act, float act_param,
                                    float* save_mean, float* save_var, void* stream);
+
+/* The device status of the iabn_forward_static_ws calls on the current
+ * device since its last call or the last read: synchronises `stream`, then
+ * reads and clears the status word of the library's own scratch, as
+ * iabn_get_device_status does for a caller's workspace (same return values;
+ * IABN_OK before any such call).  Each iabn_forward_static_ws call starts
+ * from a cleared status, so read it after the call that matters. */
+iabn_status iabn_get_static_ws_status(void* stream);
 
 #ifdef __cplusplus
 }

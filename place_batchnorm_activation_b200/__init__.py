@@ -53,7 +53,8 @@ IABN_ACT_LEAKY_RELU, IABN_ACT_ELU, IABN_ACT_IDENTITY = 0, 1, 2
 EXPORTS = ("iabn_workspace_size", "iabn_forward", "iabn_forward_with_running_stats",
            "iabn_backward",
            "iabn_update_running_stats", "iabn_get_device_status", "iabn_kernel_launches",
-           "iabn_forward_static_ws", "iabn_describe_plan", "iabn_inference",
+           "iabn_forward_static_ws", "iabn_get_static_ws_status", "iabn_describe_plan",
+           "iabn_inference",
            "iabn_forward_standard", "iabn_backward_standard", "iabn_forward_checkpoint",
            "iabn_backward_checkpoint", "iabn_checkpoint_recompute",
            "iabn_sync_forward_stats", "iabn_sync_forward_apply", "iabn_sync_backward_stats",
@@ -139,6 +140,8 @@ def lib() -> ctypes.CDLL:
             L.iabn_kernel_launches.restype = ctypes.c_uint64
             L.iabn_forward_static_ws.argtypes = [pd, vp, vp, vp, f32, i32, f32, vp, vp, vp]
             L.iabn_forward_static_ws.restype = i32
+            L.iabn_get_static_ws_status.argtypes = [vp]
+            L.iabn_get_static_ws_status.restype = i32
             L.iabn_describe_plan.argtypes = [pd, i32, i32, i32, ctypes.POINTER(IabnPlanInfo)]
             L.iabn_describe_plan.restype = i32
             L.iabn_sync_forward_stats.argtypes = [pd, vp, vp, vp, ctypes.c_size_t, vp]
@@ -257,6 +260,12 @@ def iabn_forward_static_ws(desc, x_inout, gamma, beta, eps, act, act_param, save
     argument) for callers that cannot allocate device memory."""
     return int(lib().iabn_forward_static_ws(ctypes.byref(desc), x_inout, gamma, beta, eps, act,
                                             act_param, save_mean, save_var, stream))
+
+
+def iabn_get_static_ws_status(stream) -> int:
+    """Reads and clears the status word of iabn_forward_static_ws's scratch
+    on the current device (synchronises the stream)."""
+    return int(lib().iabn_get_static_ws_status(stream))
 
 
 def iabn_describe_plan(desc, call, sm_count, smem_optin, info) -> int:
@@ -561,6 +570,12 @@ def backward_sync(z, dz, gamma, beta, save_var, dgamma, dbeta, stats, workspace,
                         shape=shape, layout=layout, eps=eps, act=act, act_param=act_param,
                         stream=stream)
     return gathered
+
+
+def get_static_ws_status(stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the status of the
+    iabn_forward_static_ws calls on the current device."""
+    return iabn_get_static_ws_status(_stream_ptr(stream))
 
 
 def get_device_status(workspace, stream=None) -> int:

@@ -78,3 +78,12 @@ extern "C" iabn_status iabn_forward_static_ws(const iabn_desc* d, void* x_inout,
     return iabn_forward(d, x_inout, gamma, beta, eps, act, act_param, save_mean, save_var, ws,
                         kStaticWsBytes, stream);
 }
+
+extern "C" iabn_status iabn_get_static_ws_status(void* stream) {
+    void* ws = nullptr;
+    if (static_ws_address(&ws) != cudaSuccess) {
+        cudaGetLastError();
+        return IABN_ERR_CUDA;
+    }
+    return iabn_get_device_status(ws, stream);
+}

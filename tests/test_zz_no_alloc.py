@@ -92,3 +92,30 @@ def test_static_workspace_rejects_oversized_descriptor():
                                      g.data_ptr(), g.data_ptr(), 1e-5, 0, 0.01, g.data_ptr(),
                                      g.data_ptr(), None)
     assert st == iabn.IABN_ERR_INVALID_ARG
+
+
+def test_static_ws_status_reports_a_timed_out_wait(monkeypatch):
+    """A bounded wait of the resident kernel made to run out (one CTA waits
+    on a word nothing sets; the others' barrier budget is 20 ms) inside
+    iabn_forward_static_ws: the call returns IABN_OK (the condition is found
+    on the device), iabn_get_static_ws_status reports IABN_ERR_TIMEOUT once
+    and clears it, and the next call is correct."""
+    sp = wl.LayerSpec("static_timeout", 8, 256, 14, 14, wl.NHWC, wl.BF16, wl.LEAKY_RELU, 0.01,
+                      seed=34)
+    inp = wl.draw(sp)
+    monkeypatch.setenv("IABN_FORCE_PLAN", "resident")
+    assert iabn.get_static_ws_status() == 0
+    monkeypatch.setenv("IABN_BARRIER_BUDGET_NS", str(20_000_000))
+    monkeypatch.setenv("IABN_TEST_STALL_CTA", "3")
+    _run(sp, inp, True)
+    monkeypatch.delenv("IABN_TEST_STALL_CTA")
+    monkeypatch.delenv("IABN_BARRIER_BUDGET_NS")
+    assert iabn.get_static_ws_status() == 6      # IABN_ERR_TIMEOUT
+    assert iabn.get_static_ws_status() == 0      # the read cleared it
+    z1, m1, v1 = _run(sp, inp, True)
+    z2, m2, v2 = _run(sp, inp, False)
+    assert iabn.get_static_ws_status() == 0
+    tol = TOL[sp.dtype]
+    compare(z1, z2, sp.dtype, "static z after a timed-out call")
+    compare(m1, m2, tol, "static mean after a timed-out call")
+    compare(v1, v2, tol, "static var after a timed-out call")
