@@ -46,9 +46,9 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # Reported only while the resident kernels' sources (KERNEL_SOURCES) hash to the value
 # they were captured on; otherwise "traffic" and "dram_bytes" are null.
 NCU_TRAFFIC = {
-    "sources_sha256": "79a2f0dcecaa735439c5b400a08e7a214bc13e47eba0b5eff3ca855e4a9a19aa",
-    "backward": {"read": 287367936, "write": 33791744},
-    "forward": {"read": 109641728, "write": 22854912},
+    "sources_sha256": "d386d0932a0a3de7700da3720cc3a827b8bec8d2ad039a85f11e125d2a6d2103",
+    "backward": {"read": 272316416, "write": 32016640},
+    "forward": {"read": 102926848, "write": 20714496},
 }
 # the resident kernels' phase trace in the workspace (IABN_TRACE=1): up to 256
 # CTAs x 16 slots of 8 bytes, right after the 256-byte control block

@@ -28,9 +28,10 @@
 //            per channel, fixed order), a second grid barrier.
 //   phase B  tiles n-1..0: resident tiles first, then the streamed ones -- the
 //            most recently read first: the last one of each ring slot is still
-//            in the slot, the others are read back from L2.  The consumers
-//            write their results straight to global memory with 128-bit
-//            stores; the producer refills each freed ring slot.
+//            in the slot, the others are read back from L2 -- and then the rows
+//            kept in Tensor Memory.  The consumers write their results
+//            straight to global memory with 128-bit stores; the producer
+//            refills each freed ring slot.
 //
 // Method: "In-Place Activated BatchNorm for Memory-Optimized Training of
 // DNNs" (paperlayer.ai summary), section 3: "Batch Normalization Review",
@@ -1521,8 +1522,30 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
             }
         };
         acct_start();
+        for (int t = n - 1; t >= nring; --t) {
+            const int s = ring + (t - nring);
+            apply_tile(t, s, 0, INT_MAX);
+            release(&done[s]);
+        }
+        acct_work();
+        for (int j = 0; j < nB; ++j) {
+            const int t = thi - 1 - j;
+            const int s = t % ring;
+            // a tile still in its slot from phase A needs no wait
+            if (!ring_resident(t) && !cwait(s)) break;
+            acct_wait();
+            // skip the stashed rows: ordinals [js, js + Jc)
+            const int qlo = stash && sfirst ? Jc - t * tile_ord : 0;
+            const int qhi = stash && !sfirst ? js - t * tile_ord : INT_MAX;
+            apply_tile(t, s, qlo, qhi);
+            acct_comp();
+            release(&done[s]);
+            acct_work();
+        }
+        // the stashed rows last: their results are written after every read
+        // of phase B, so their new L2 lines evict nothing phase B still reads
         if (scp) {
-            // the stashed row groups first, RB at a time (four vectors per
+            // the stashed row groups, RB at a time (four vectors per
             // tensor): this thread's column k of group i is at TMEM column
             // 8*(NT*(i*CPT + k) + tensor) + 4*(warp/4)
             unsigned char* grow = a.dst + u0 * P.unit_bytes;
@@ -1549,7 +1572,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 }
             }
         } else if (stash && active) {
-            // the stashed rows first: no wait for any tile
+            // the stashed rows (no wait for any tile)
             unsigned char* grow = a.dst + u0 * P.unit_bytes;
             unsigned char* grow2 = CKPT ? a.dst2 + u0 * P.unit_bytes : nullptr;
             for (int i0 = 0; i0 < Jc; i0 += RB) {
@@ -1576,26 +1599,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 }
             }
         }
-        for (int t = n - 1; t >= nring; --t) {
-            const int s = ring + (t - nring);
-            apply_tile(t, s, 0, INT_MAX);
-            release(&done[s]);
-        }
         acct_work();
-        for (int j = 0; j < nB; ++j) {
-            const int t = thi - 1 - j;
-            const int s = t % ring;
-            // a tile still in its slot from phase A needs no wait
-            if (!ring_resident(t) && !cwait(s)) break;
-            acct_wait();
-            // skip the stashed rows: ordinals [js, js + Jc)
-            const int qlo = stash && sfirst ? Jc - t * tile_ord : 0;
-            const int qhi = stash && !sfirst ? js - t * tile_ord : INT_MAX;
-            apply_tile(t, s, qlo, qhi);
-            acct_comp();
-            release(&done[s]);
-            acct_work();
-        }
         acct_flush(11);
     }
 
