@@ -172,9 +172,18 @@ __device__ __forceinline__ void src_affine(float g, float b, float mean, float v
 
 // ------------------------------------------------------------ small helpers
 
-// 16-byte global load, streaming (evict-first) cache hint.  asm volatile keeps
-// a batch of these in program order, so a batch is in flight before its values
-// are used.
+// 16-byte global loads.  asm volatile keeps a batch of these in program
+// order, so a batch is in flight before its values are used.
+//   ldg_cg: cached in L2 only, normal eviction priority, so a later pass over
+//           the same data can still find it there;
+//   ldg_cs: streaming (evict-first).
+__device__ __forceinline__ uint4 ldg_cg(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint4 ldg_cs(const void* p) {
     uint4 v;
     asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"

@@ -52,6 +52,9 @@ struct AffArgs {
     const float* rmean;
     const float* rvar;
     float eps, p;
+    // rows launch, second pass over x (kCoefGiven): the statistics pass's row
+    // segments [b*R/nseg, (b+1)*R/nseg); 0: grid-stride walk
+    int nseg;
 };
 
 // Coefficients of one channel: y = (a - m)*sc + b (fp32 storage) or
@@ -105,7 +108,7 @@ constexpr int kAffUnroll = 4;
 
 // NHWC rows: thread -> (column, row phase); its column's channels' coefficients
 // in registers; kAffUnroll rows' loads in flight.
-template <int DT, int ACT, int SRC, bool CKPT>
+template <int DT, int ACT, int SRC, bool CKPT, bool REV>
 __global__ void __launch_bounds__(kAffThreads) k_aff_rows(const AffArgs a) {
     constexpr int VE = Vec<DT>::N;   // elements per 16-byte vector
     const int W = a.VC < kAffThreads ? a.VC : kAffThreads;
@@ -120,6 +123,36 @@ __global__ void __launch_bounds__(kAffThreads) k_aff_rows(const AffArgs a) {
     const uint4* src = reinterpret_cast<const uint4*>(a.src) + col;
     uint4* dst = reinterpret_cast<uint4*>(a.dst) + col;
     uint4* dst2 = CKPT ? reinterpret_cast<uint4*>(a.dst2) + col : nullptr;
+    auto one = [&](const uint4& v, int64_t r) {
+        float f[VE], o[VE], o2[VE];
+        Vec<DT>::unpack(v, f);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) apply_elem<DT, ACT, CKPT>(f[e], k[e], a.p, o[e], o2[e]);
+        __stcs(dst + r * a.VC, Vec<DT>::pack(o));
+        if (CKPT) __stcs(dst2 + r * a.VC, Vec<DT>::pack(o2));
+    };
+    if (REV) {
+        // The second pass over x, right after the statistics pass read it
+        // segment by segment, front to back: the J blocks of segment b share
+        // its rows (row phases j*RPB + phase) and walk them last first, so
+        // the rows L2 still holds from that pass come first.
+        const int J = (int)gridDim.x / a.nseg;
+        const int b = (int)blockIdx.x / J, j = (int)blockIdx.x % J;
+        const int64_t s0 = (int64_t)b * a.R / a.nseg, s1 = ((int64_t)b + 1) * a.R / a.nseg;
+        const int64_t stride = (int64_t)J * RPB;
+        const int64_t first = s0 + (int64_t)j * RPB + phase;
+        if (first >= s1) return;
+        int64_t r = first + (s1 - 1 - first) / stride * stride;   // this thread's last row
+        for (; r - (kAffUnroll - 1) * stride >= first; r -= kAffUnroll * stride) {
+            uint4 v[kAffUnroll];
+#pragma unroll
+            for (int u = 0; u < kAffUnroll; ++u) v[u] = __ldcs(src + (r - u * stride) * a.VC);
+#pragma unroll
+            for (int u = 0; u < kAffUnroll; ++u) one(v[u], r - u * stride);
+        }
+        for (; r >= first; r -= stride) one(__ldcs(src + r * a.VC), r);
+        return;
+    }
     const int64_t rstep = (int64_t)gridDim.x * RPB;
     for (int64_t r0 = (int64_t)blockIdx.x * RPB + phase; r0 < a.R; r0 += rstep * kAffUnroll) {
         uint4 v[kAffUnroll];
@@ -236,17 +269,26 @@ cudaError_t launch_aff(const Geom& g, AffArgs a, int sms, cudaStream_t s) {
     const int64_t rby = g.C * g.esize;
     if (g.layout == kNHWC && rby % 16 == 0 && rby / 16 <= (int64_t)1 << 30) {
         a.VC = (int)(rby / 16);
-        auto kern = k_aff_rows<DT, ACT, SRC, CKPT>;
-        static std::atomic<int> occ{0};
+        // the segment walk only for a second pass over x (kCoefGiven)
+        const bool rev = SRC == kCoefGiven && a.nseg > 0;
+        auto kern = rev ? k_aff_rows<DT, ACT, SRC, CKPT, SRC == kCoefGiven>
+                        : k_aff_rows<DT, ACT, SRC, CKPT, false>;
+        static std::atomic<int> occ{0}, occ_rev{0};
         const int W = a.VC < kAffThreads ? a.VC : kAffThreads;
         const int64_t gy = (a.VC + W - 1) / W;
         if (gy > 65535) return cudaErrorNotSupported;
         const int64_t RPB = kAffThreads / W;
-        const int64_t want = (int64_t)sms * blocks_per_sm(kern, 0, occ);
+        const int64_t want = (int64_t)sms * blocks_per_sm(kern, 0, rev ? occ_rev : occ);
         int64_t gx = (want + gy - 1) / gy;
         const int64_t need = (g.R + RPB - 1) / RPB;
         if (gx > need) gx = need;
         if (gx < 1) gx = 1;
+        if (rev) {
+            // J blocks per segment, at least one
+            int64_t J = gx / a.nseg;
+            if (J < 1) J = 1;
+            gx = J * a.nseg;
+        }
         kern<<<dim3((unsigned)gx, (unsigned)gy), kAffThreads, 0, s>>>(a);
     } else {
         const size_t smem = g.C <= kAffSmemChannels ? (size_t)g.C * sizeof(Coef) : 0;
@@ -327,13 +369,14 @@ cudaError_t recompute_pass(const Geom& g, const void* xhat, void* z, const float
 }
 
 cudaError_t forward_apply_pass(const Geom& g, const FwdArgs& f, const float4* coef,
-                               cudaStream_t s, int sms) {
+                               cudaStream_t s, int sms, int nseg) {
     AffArgs a = {};
     a.src = static_cast<const unsigned char*>(f.x);
     a.dst = static_cast<unsigned char*>(f.dst);
     a.dst2 = static_cast<unsigned char*>(f.dst2);
     a.coef = coef;
     a.p = f.act_param;
+    a.nseg = nseg;
     if (f.mode == kModeFwdCkpt) return launch_aff_dt<kCoefGiven, true>(g, a, f.act, sms, s);
     return launch_aff_dt<kCoefGiven, false>(g, a, f.act, sms, s);
 }

@@ -101,7 +101,7 @@ cudaError_t recompute_pass(const Geom& g, const void* xhat, void* z, const float
                            const float* beta, int act, float act_param, cudaStream_t s,
                            int sms);
 cudaError_t forward_apply_pass(const Geom& g, const FwdArgs& f, const float4* coef,
-                               cudaStream_t s, int sms);
+                               cudaStream_t s, int sms, int nseg = 0);
 // INPLACE-ABNsync (iabn_twophase.cu): this GPU's per-channel record (3
 // doubles per channel), and the apply from the records of all GPUs
 // ([world][C][3], rank order).

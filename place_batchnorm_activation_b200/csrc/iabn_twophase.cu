@@ -387,10 +387,13 @@ struct RowTile {
 // own first value K of each channel, turns them into (mean, M2) in fp64, and
 // the block's row phases combine around phase 0's mean in phase order; one
 // (mean, M2) partial per (row block, channel).
-template <int DT>
+template <int DT, bool KEEP>
 __global__ void __launch_bounds__(kRowThreads, 1)
 k_tp_stats_rows(const uint4* __restrict__ x, int64_t R, int VC, int RB, int64_t C,
                 double2* __restrict__ part) {
+    // KEEP: x is read again by the apply pass over these row segments, last
+    // rows first; load it with normal L2 priority (else streaming)
+    auto ld = [](const uint4* p) { return KEEP ? ldg_cg(p) : ldg_cs(p); };
     constexpr int VE = Vec<DT>::N;
     const RowTile<> rt(VC, R, RB);
     const int64_t n = rt.count();
@@ -415,11 +418,11 @@ k_tp_stats_rows(const uint4* __restrict__ x, int64_t R, int VC, int RB, int64_t 
         for (; r + (kStatsBatch - 1) * step < rt.r1; r += kStatsBatch * step) {
             uint4 v[kStatsBatch];
 #pragma unroll
-            for (int k = 0; k < kStatsBatch; ++k) v[k] = ldg_cs(src + (r + k * step) * VC);
+            for (int k = 0; k < kStatsBatch; ++k) v[k] = ld(src + (r + k * step) * VC);
 #pragma unroll
             for (int k = 0; k < kStatsBatch; ++k) add(v[k]);
         }
-        for (; r < rt.r1; r += step) add(ldg_cs(src + r * VC));
+        for (; r < rt.r1; r += step) add(ld(src + r * VC));
     }
     // combine the row phases of each column, one channel of the vector at a
     // time (unrolled: the per-channel registers must not be indexed at run time)
@@ -487,13 +490,13 @@ k_tp_reduce_rows(const uint4* __restrict__ z, const uint4* __restrict__ dz, int6
             uint4 vz[B], vd[B];
 #pragma unroll
             for (int k = 0; k < B; ++k) {
-                vz[k] = ldg_cs(pz + (r + k * step) * VC);
-                vd[k] = ldg_cs(pd + (r + k * step) * VC);
+                vz[k] = ldg_cg(pz + (r + k * step) * VC);
+                vd[k] = ldg_cg(pd + (r + k * step) * VC);
             }
 #pragma unroll
             for (int k = 0; k < B; ++k) add(vz[k], vd[k]);
         }
-        for (; r < rt.r1; r += step) add(ldg_cs(pz + r * VC), ldg_cs(pd + r * VC));
+        for (; r < rt.r1; r += step) add(ldg_cg(pz + r * VC), ldg_cg(pd + r * VC));
     }
     __shared__ float2 sm[kRowThreads];
 #pragma unroll
@@ -868,6 +871,16 @@ struct RowGrid {
     int RB, GY, VC;
 };
 
+// Whether the forward's apply pass walks the statistics pass's row segments
+// last row first.  L2 keeps the most recently read ~80 MB of a streamed
+// tensor, so a tensor larger than that is found there only in that order; a
+// smaller one is found there whole, and the plain grid-stride walk is faster
+// (same-box A/B: ResNet trunk 102.8 MB fwd 71.6 -> 69.6 us, the 51.4 MB
+// sweep layer 50.2 -> 48.3 us, but the 6.4 MB layer 31.4 -> 35.4 us).
+static bool reverse_segments(const Geom& g) {
+    return rows_vectorised(g) && g.E * g.esize > ((int64_t)32 << 20);
+}
+
 // NCHW small planes: g whole planes per 16-byte aligned unit (0: not used).
 static int unit_planes(const Geom& g) {
     if (g.layout != kNCHW) return 0;
@@ -928,8 +941,12 @@ static cudaError_t fwd_stats_launch(const Geom& g, const void* xv, const Workspa
     if (rows_vectorised(g)) {
         const RowGrid rg = row_grid(g, sms);
         RB = rg.RB;
-        k_tp_stats_rows<DT><<<dim3(rg.RB, rg.GY), kRowThreads, 0, s>>>(
-            static_cast<const uint4*>(xv), g.R, rg.VC, rg.RB, g.C, w.part);
+        if (reverse_segments(g))
+            k_tp_stats_rows<DT, true><<<dim3(rg.RB, rg.GY), kRowThreads, 0, s>>>(
+                static_cast<const uint4*>(xv), g.R, rg.VC, rg.RB, g.C, w.part);
+        else
+            k_tp_stats_rows<DT, false><<<dim3(rg.RB, rg.GY), kRowThreads, 0, s>>>(
+                static_cast<const uint4*>(xv), g.R, rg.VC, rg.RB, g.C, w.part);
         K = RB;
     } else if (g.layout == kNHWC) {
         RB = nhwc_row_blocks(g.R);
@@ -970,8 +987,10 @@ static cudaError_t fwd_twophase_dt(const Geom& g, const FwdArgs& a, const Worksp
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // the elementwise pass with fixed channels per thread (iabn_elementwise.cu)
-    return forward_apply_pass(g, a, w.coef, s, sms);
+    // the elementwise pass with fixed channels per thread (iabn_elementwise.cu);
+    // a tensor too large to stay whole in L2 is walked over the statistics
+    // pass's row segments, each last row first (see reverse_segments)
+    return forward_apply_pass(g, a, w.coef, s, sms, reverse_segments(g) ? RB : 0);
 }
 
 cudaError_t forward_twophase(const Geom& g, const FwdArgs& a, const Workspace& w,
@@ -1236,7 +1255,8 @@ cudaError_t sync_forward_apply(const Geom& g, const FwdArgs& a, const double* ga
     count_launches(1);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return forward_apply_pass(g, a, w.coef, s, sms);
+    return forward_apply_pass(g, a, w.coef, s, sms,
+                              reverse_segments(g) ? row_grid(g, sms).RB : 0);
 }
 
 template <int DT, int ACT>
