@@ -46,7 +46,7 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # Reported only while the resident kernels' sources (KERNEL_SOURCES) hash to the value
 # they were captured on; otherwise "traffic" and "dram_bytes" are null.
 NCU_TRAFFIC = {
-    "sources_sha256": "3eaa9fcfeac01ae5be9f9cf2f59f9507a3373a9f86af3c410cca41df25b8566d",
+    "sources_sha256": "3db2e47fe0bdf04726f6f2bac042f1a36425e279699104ed1642591d1018f2d3",
     "backward": {"read": 272316416, "write": 32016640},
     "forward": {"read": 102926848, "write": 20714496},
 }
