@@ -87,7 +87,7 @@ int layer_mode(int layer, int dir) {
 // device cannot hold the tiles.
 bool make_plan(const Geom& g, int mode, const DeviceLimits& dl, ResPlan& P, int& cpt) {
     if (dl.sms <= 0 || dl.smem_optin <= 0) return false;
-    const int dir = mode == kModeFwd || mode == kModeFwdCkpt ? 0 : 1;
+    const int dir = mode_dir(mode);
     // coefficient records per channel in phase B
     const int nrec = mode == kModeBwdX || mode == kModeBwdXhat ? 2 : 1;
     const int s = g.esize;
@@ -137,13 +137,25 @@ bool make_plan(const Geom& g, int mode, const DeviceLimits& dl, ResPlan& P, int&
         P.unit_bytes = (int)(gq * pb);
         P.units = g.N * g.C / gq;
         int tu = target / P.unit_bytes;
-        P.tile_units = tu < 1 ? 1 : tu;
+        if (tu < 1) tu = 1;
         P.g = gq;
-        // lanes per plane: one for small planes (no shuffles; the CTA's 256
-        // threads take 256 planes at once), else enough for ~8 elements each
+        // lanes per plane: one for small planes (no shuffles), else enough for
+        // ~8 elements each
         int L = 1;
         if (g.HW > 64)
             while (L < 32 && L * 8 < g.HW) L *= 2;
+        if (dir == 0) {
+            // the forward's 480 consumer threads: more lanes while a tile holds
+            // fewer planes than they take at once (nc / L), so none is idle,
+            // and a tile of whole rounds of nc / L planes where the target
+            // size holds one
+            const int nc = res_consumers(kNCHW, 0);
+            while (L < 32 && nc / L > (int64_t)tu * gq) L *= 2;
+            const int gp = nc / L;
+            const int m = gp / gcd_int(gp, gq);
+            if (tu >= m) tu = tu / m * m;
+        }
+        P.tile_units = tu;
         P.L = L;
         P.VC = 1;
         P.RP = 1;
@@ -241,7 +253,7 @@ bool resident_shape(const Geom& g, int layer, int dir, int sms, int smem_optin,
         return false;
     const bool nhwc = g.layout == kNHWC;
     out.grid = P.G;
-    out.threads = kResThreads;
+    out.threads = res_threads(g.layout, mode_dir(layer_mode(layer, dir)));
     out.smem_bytes = P.smem_bytes;
     out.tile_bytes = P.tile_bytes;
     out.slots = P.nslots;

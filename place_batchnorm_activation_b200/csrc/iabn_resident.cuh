@@ -6,8 +6,10 @@
 // NCHW: groups of g whole planes, g chosen so every unit starts on a 16-byte
 // boundary) and streams it through shared-memory slots with the bulk-copy
 // engine.  One producer warp issues every bulk load; eight consumer warps
-// compute and store; one copier warp moves stashed rows from the landed
-// slots into Tensor Memory (see the TMEM stash below).  Slots are handed over with mbarriers (full: data
+// compute and store (fifteen in the NCHW forward); one copier warp moves
+// stashed rows from the landed slots into Tensor Memory (see the TMEM stash
+// below; the NCHW forward, which stashes nothing, has none).  Slots are
+// handed over with mbarriers (full: data
 // landed; empty: consumers done with a phase A tile; done: consumers done
 // with a phase B tile, so the slot may be refilled), so no consumer waits on
 // a CTA-wide barrier per tile.
@@ -48,9 +50,24 @@
 
 namespace iabn {
 
-constexpr int kConsumers = 256;                  // consumer threads (8 warps)
+constexpr int kConsumers = 256;                  // NHWC consumer threads (8 warps)
 constexpr int kConsumerWarps = kConsumers / 32;
 constexpr int kResThreads = kConsumers + 64;     // + one producer warp + one copier warp
+// The NCHW forward keeps nothing in Tensor Memory, so it has no copier warp,
+// and its plane loops fit in 128 registers a thread without spilling: 15
+// consumer warps and the producer, four warps on each scheduler (each
+// scheduler owns a quarter of the register file).  (The NCHW backward keeps
+// the 8 + 2 layout: at 128 registers its phase B ran slower.)
+constexpr int kConsumersNchwFwd = 480;
+__host__ __device__ constexpr int mode_dir(int mode) {
+    return mode == kModeFwd || mode == kModeFwdCkpt ? 0 : 1;
+}
+__host__ __device__ constexpr int res_consumers(int layout, int dir) {
+    return layout == kNCHW && dir == 0 ? kConsumersNchwFwd : kConsumers;
+}
+__host__ __device__ constexpr int res_threads(int layout, int dir) {
+    return layout == kNCHW && dir == 0 ? kConsumersNchwFwd + 32 : kResThreads;
+}
 constexpr int kMaxSlots = 32;
 constexpr int kBarBytes = 4 * kMaxSlots * 8;     // full[], empty[], done[], cpdone[] mbarriers
 
@@ -204,13 +221,25 @@ __device__ __forceinline__ float2 act_forward2(float2 y, float p, bool slope_le1
         return slope_le1 ? f2(fmaxf(y.x, t.x), fmaxf(y.y, t.y))
                          : f2(fminf(y.x, t.x), fminf(y.y, t.y));
     }
-    if (ACT == kElu) return f2(act_forward<kElu, DT>(y.x, p), act_forward<kElu, DT>(y.y, p));
+    if (ACT == kElu) {
+        if (DT == kF32) return f2(act_forward<kElu, DT>(y.x, p), act_forward<kElu, DT>(y.y, p));
+        // 16-bit storage: e = p*(exp(min(y, 0)) - 1) is exactly 0 for y >= 0
+        // (the exponential of +0 is exactly 1), so max(y, 0) + e is act_forward's
+        // select, on pairs and without a comparison
+        const float2 e = __fmul2_rn(f2(p, p), __fadd2_rn(f2(__expf(fminf(y.x, 0.f)),
+                                                            __expf(fminf(y.y, 0.f))),
+                                                         f2(-1.f, -1.f)));
+        return __fadd2_rn(f2(fmaxf(y.x, 0.f), fmaxf(y.y, 0.f)), e);
+    }
     return y;
 }
 
 template <int DT, int ACT, int LAYOUT, int CPT, int MODE>
-__global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
-    constexpr int DIR = MODE == kModeFwd || MODE == kModeFwdCkpt ? 0 : 1;
+__global__ void __launch_bounds__(res_threads(LAYOUT, mode_dir(MODE)), 1)
+    k_resident(const ResArgs a) {
+    constexpr int DIR = mode_dir(MODE);
+    constexpr int NC = res_consumers(LAYOUT, DIR);   // consumer threads
+    constexpr int CW = NC / 32;                      // consumer warps
     // checkpointing forward: a second output (z) besides xhat
     constexpr bool CKPT = MODE == kModeFwdCkpt;
     // backward from a stored x or xhat: y is recomputed by a scale and shift
@@ -231,16 +260,16 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     // gamma, beta (and, backward, the saved variance and, standard backward,
     // the saved mean) of the first channel each consumer half-warp finalizes,
     // fetched while phase A streams
-    __shared__ float s_par[kConsumerWarps][2][4];
+    __shared__ float s_par[CW][2][4];
 
     const ResPlan& P = a.P;
     unsigned char* scratch = smem + kBarBytes;
     unsigned char* slots = scratch + P.scratch_bytes;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const bool consumer = warp < kConsumerWarps;
-    const bool producer = warp == kConsumerWarps;
-    const bool copier = warp == kConsumerWarps + 1;
+    const bool consumer = warp < CW;
+    const bool producer = warp == CW;
+    const bool copier = warp == CW + 1;
     const int b = blockIdx.x;
     const int G = P.G;
     // Phase trace: 0 start, 1 phase A done, 2 merged, 3 barrier 1, 4 finalize,
@@ -322,8 +351,8 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     if (tid == 0) {
         for (int s = 0; s < P.nslots; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-            mbar_init(&done[s], kConsumerWarps);
+            mbar_init(&empty[s], CW);
+            mbar_init(&done[s], CW);
             mbar_init(&cpdone[s], 1);
         }
         mbar_init_fence();
@@ -473,7 +502,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         } else {
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
-                col[k] = tid + k * kConsumers;
+                col[k] = tid + k * NC;
                 colok[k] = consumer && col[k] < VC;
             }
         }
@@ -511,7 +540,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     const int tile_ord = P.tile_units / RP;   // row ordinals per tile and thread (NHWC)
     // NCHW mapping: groups of L lanes per plane.
     const int L = P.L;
-    const int GP = kConsumers / L;
+    const int GP = NC / L;
     const int grp = tid / L, glane = tid % L;
     const int HW = (int)a.HW;
     const int pbytes = HW * (int)sizeof(typename Storage<DT>::T);
@@ -1064,7 +1093,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
         // Channel pairs go to warp 0 of every CTA first, then warp 1, ...: the
         // scattered partial loads spread over as many SMs as there are pairs.
         const int hl = lane & 15, half = lane >> 4;
-        const int64_t nw = (int64_t)G * kConsumerWarps;
+        const int64_t nw = (int64_t)G * CW;
         bool first = true;
         for (int64_t cpair = (int64_t)warp * G + b; cpair * 2 < a.C;
              cpair += nw, first = false) {
@@ -1203,7 +1232,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
     float4* scoef = reinterpret_cast<float4*>(scratch);
     if (LAYOUT == kNCHW && P.ncoef > 0) {
         if (consumer && !failed())
-            for (int i = tid; i < P.ncoef; i += kConsumers) {
+            for (int i = tid; i < P.ncoef; i += NC) {
                 const int64_t c = ch0 + i;
                 const int64_t cm = c >= a.C ? c - a.C : c;
                 scoef[i] = a.coef[cm];
@@ -1428,10 +1457,10 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 };
                 unsigned char* gt = a.dst + t_u0(t) * P.unit_bytes;
                 unsigned char* gt2 = CKPT ? a.dst2 + t_u0(t) * P.unit_bytes : nullptr;
-                // This thread's vectors v = tid + kConsumers*j start ES elements
+                // This thread's vectors v = tid + NC*j start ES elements
                 // apart: its plane offset `off` and window index `c` advance by
                 // fixed steps (dq planes + dr elements), no division per vector.
-                constexpr uint32_t ES = (uint32_t)kConsumers * EPV;
+                constexpr uint32_t ES = (uint32_t)NC * EPV;
                 const uint32_t dq = ES / hw, dr = ES - dq * hw, dqc = dq % C32;
                 uint32_t c, off;
                 {
@@ -1480,10 +1509,34 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                         // planes at least a vector long: two coefficient sets at
                         // most, chosen per element without branches
                         const Rec2 q0 = coef_at(cc), q1 = coef_at(cc + 1u == C32 ? 0u : cc + 1u);
+                        if (DIR == 0 && !CKPT) {
+                            // the forward: both channels' affine results on
+                            // pairs, then one select per element (not one per
+                            // coefficient) and the activation on pairs
+                            const float4 &a0 = q0.a, &a1 = q1.a;
 #pragma unroll
-                        for (int k = 0; k < EPV; ++k) {
-                            const bool first = (uint32_t)k < rem;
-                            rewrite_elem(k, first ? q0 : q1);
+                            for (int k = 0; k < EPV; k += 2) {
+                                const float2 x = f2(xz[k], xz[k + 1]);
+                                const float2 y0 =
+                                    DT == kF32 ? __ffma2_rn(__fadd2_rn(x, f2(-a0.x, -a0.x)),
+                                                            f2(a0.y, a0.y), f2(a0.z, a0.z))
+                                               : __ffma2_rn(x, f2(a0.y, a0.y), f2(a0.w, a0.w));
+                                const float2 y1 =
+                                    DT == kF32 ? __ffma2_rn(__fadd2_rn(x, f2(-a1.x, -a1.x)),
+                                                            f2(a1.y, a1.y), f2(a1.z, a1.z))
+                                               : __ffma2_rn(x, f2(a1.y, a1.y), f2(a1.w, a1.w));
+                                const float2 y = f2((uint32_t)k < rem ? y0.x : y1.x,
+                                                    (uint32_t)k + 1u < rem ? y0.y : y1.y);
+                                const float2 z = act_forward2<ACT, DT>(y, p, le1);
+                                xz[k] = z.x;
+                                xz[k + 1] = z.y;
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < EPV; ++k) {
+                                const bool first = (uint32_t)k < rem;
+                                rewrite_elem(k, first ? q0 : q1);
+                            }
                         }
                     } else {
                         Rec2 q = coef_at(cc);
@@ -1510,7 +1563,7 @@ __global__ void __launch_bounds__(kResThreads, 1) k_resident(const ResArgs a) {
                 };
                 // one vector at a time (a two-vector interleave measured slower:
                 // many-channel 40.5 / 60.3 us against 36.9 / 55.3)
-                for (int v = tid; v < nvec; v += kConsumers) {
+                for (int v = tid; v < nvec; v += NC) {
                     const uint4 vz = lds128(sbv + (uint32_t)v * 16u);
                     const uint4 vd =
                         DIR == 1 ? lds128(sbv + (uint32_t)P.half_bytes + (uint32_t)v * 16u) : vz;
@@ -1652,7 +1705,7 @@ cudaError_t launch_resident_one(const ResArgs& a, int smem_optin, cudaStream_t s
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)a.P.G);
-    cfg.blockDim = dim3(kResThreads);
+    cfg.blockDim = dim3(res_threads(LAYOUT, mode_dir(MODE)));
     cfg.dynamicSmemBytes = (size_t)a.P.smem_bytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

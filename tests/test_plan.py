@@ -56,7 +56,10 @@ def check_resident(info, shape, layout, dtype, call, sm_count, smem_optin):
     n, c, h, w = shape
     s = esize(dtype)
     nt = 1 if call % 2 == 0 else 2           # tensors streamed: x; or z (x, xhat) and dz
-    assert info["launches"] == 1 and info["threads"] == 320
+    # 8 consumer warps, a producer and a copier; the NCHW forward (no Tensor
+    # Memory stash): 15 consumer warps and a producer
+    threads = 512 if layout == wl.NCHW and call % 2 == 0 else 320
+    assert info["launches"] == 1 and info["threads"] == threads
     units = n * h * w if layout == wl.NHWC else n * c // info["planes_per_unit"]
     assert 1 <= info["grid"] <= min(sm_count, 256, units)
     assert 0 < info["smem_bytes"] <= smem_optin - 1024
@@ -152,6 +155,21 @@ def test_benchmark_workloads_take_the_resident_plan():
     for direction, rows in ((0, 64), (1, 32)):
         info = iabn.describe_plan(trunk.shape, trunk.layout, trunk.dtype, direction, **B200)
         assert (info["stash_rows"], info["stash_copy_engine"], info["row_phases"]) == (rows, 1, 8)
+
+
+def test_nchw_forward_tiles_hold_whole_rounds_of_planes():
+    """NCHW forward tiles hold a whole number of the planes its 480 consumer
+    threads take at once (480 / lanes per plane) where the tile size target
+    allows: the many-channel layer (7x7 fp16 planes, 8 planes per 16-byte
+    aligned unit of 784 bytes) forward 60 units (480 planes, one lane each);
+    the backward keeps 256 consumer threads and the plain target, 31 units."""
+    mc = wl.spec(3)
+    fwd = iabn.describe_plan(mc.shape, mc.layout, mc.dtype, 0, **B200)
+    bwd = iabn.describe_plan(mc.shape, mc.layout, mc.dtype, 1, **B200)
+    assert fwd["plan"] == bwd["plan"] == "resident"
+    assert fwd["planes_per_unit"] == bwd["planes_per_unit"] == 8
+    assert fwd["tile_bytes"] == 60 * 784 and bwd["tile_bytes"] == 31 * 784
+    assert (fwd["threads"], bwd["threads"]) == (512, 320)
 
 
 def test_small_shared_memory_declines_the_resident_plan():
