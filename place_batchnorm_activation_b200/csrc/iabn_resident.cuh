@@ -1531,6 +1531,25 @@ __global__ void __launch_bounds__(res_threads(LAYOUT, mode_dir(MODE)), 1)
                                 xz[k] = z.x;
                                 xz[k + 1] = z.y;
                             }
+                        } else if (DIR == 1 && !SRCV) {
+                            // the in-place backward: dx with both channels'
+                            // coefficients on pairs, then one select per element
+                            const float4 &a0 = q0.a, &a1 = q1.a;
+#pragma unroll
+                            for (int k = 0; k < EPV; k += 2) {
+                                float y0, d0, y1, d1;
+                                act_backward<ACT, DT>(xz[k], xd[k], p, inv_p, y0, d0);
+                                act_backward<ACT, DT>(xz[k + 1], xd[k + 1], p, inv_p, y1, d1);
+                                const float2 y = f2(y0, y1), dy = f2(d0, d1);
+                                const float2 r0 = __ffma2_rn(f2(a0.x, a0.x), dy,
+                                                             __ffma2_rn(f2(a0.y, a0.y), y,
+                                                                        f2(a0.z, a0.z)));
+                                const float2 r1 = __ffma2_rn(f2(a1.x, a1.x), dy,
+                                                             __ffma2_rn(f2(a1.y, a1.y), y,
+                                                                        f2(a1.z, a1.z)));
+                                xz[k] = (uint32_t)k < rem ? r0.x : r1.x;
+                                xz[k + 1] = (uint32_t)k + 1u < rem ? r0.y : r1.y;
+                            }
                         } else {
 #pragma unroll
                             for (int k = 0; k < EPV; ++k) {
