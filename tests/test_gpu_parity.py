@@ -148,6 +148,13 @@ EDGE = [
     (8, 4104, 3, 3, wl.NHWC, wl.F16, wl.LEAKY_RELU, 0.01),
     (2, 1024, 1, 1, wl.NHWC, wl.BF16, wl.IDENTITY, 0.0),
     (64, 40, 3, 3, wl.NCHW, wl.F16, wl.ELU, 1.0),
+    # NCHW forwards whose small planes get two or four lanes each (tiles of
+    # 240 or 120 planes for the 480 consumer threads), several ragged tiles
+    # per CTA, and one whose tile is rounded to whole rounds of planes
+    (128, 512, 7, 7, wl.NCHW, wl.F32, wl.ELU, 1.0),
+    (512, 128, 8, 8, wl.NCHW, wl.BF16, wl.LEAKY_RELU, 0.01),
+    (640, 60, 8, 8, wl.NCHW, wl.F32, wl.IDENTITY, 0.0),
+    (768, 96, 6, 6, wl.NCHW, wl.F16, wl.ELU, 1.0),
 ]
 
 
