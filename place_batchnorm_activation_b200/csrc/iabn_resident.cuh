@@ -1404,11 +1404,15 @@ __global__ void __launch_bounds__(res_threads(LAYOUT, mode_dir(MODE)), 1)
                 const uint32_t hb = DIR == 0 ? 0u : (uint32_t)P.half_bytes;
                 unsigned char* gtile = a.dst + t_u0(t) * P.unit_bytes;
                 unsigned char* gtile2 = CKPT ? a.dst2 + t_u0(t) * P.unit_bytes : nullptr;
-                // rows in batches of RB: loads, then math, then stores
-                for (int i0 = max(qlo, 0); i0 < m; i0 += RB) {
-                    uint4 vz[RB][CPT], vd[RB][CPT], vo[RB][CPT];
+                // The backward with one column per thread takes its rows one at
+                // a time here: batches of 2 or 4 rows measured 2-4 us slower on
+                // the large layers.
+                constexpr int RBB = DIR == 1 && CPT == 1 ? 1 : RB;
+                // rows in batches of RBB: loads, then math, then stores
+                for (int i0 = max(qlo, 0); i0 < m; i0 += RBB) {
+                    uint4 vz[RBB][CPT], vd[RBB][CPT], vo[RBB][CPT];
 #pragma unroll
-                    for (int u = 0; u < RB; ++u)
+                    for (int u = 0; u < RBB; ++u)
 #pragma unroll
                         for (int k = 0; k < CPT; ++k) {
                             if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
@@ -1417,11 +1421,11 @@ __global__ void __launch_bounds__(res_threads(LAYOUT, mode_dir(MODE)), 1)
                             if (DIR == 1) vd[u][k] = lds128(o + hb);
                         }
 #pragma unroll
-                    for (int u = 0; u < RB; ++u)
+                    for (int u = 0; u < RBB; ++u)
                         if (i0 + u < m) rewrite(vz[u], vd[u], vo[u]);
                     // results go straight to their place in global memory
 #pragma unroll
-                    for (int u = 0; u < RB; ++u)
+                    for (int u = 0; u < RBB; ++u)
 #pragma unroll
                         for (int k = 0; k < CPT; ++k) {
                             if (i0 + u >= m || (CPT > 1 && !colok[k])) continue;
