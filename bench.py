@@ -46,9 +46,9 @@ METRIC = "InPlace-ABN fwd+bwd GB/s and % of B200 HBM roofline per config; elemen
 # Reported only while the resident kernels' sources (KERNEL_SOURCES) hash to the value
 # they were captured on; otherwise "traffic" and "dram_bytes" are null.
 NCU_TRAFFIC = {
-    "sources_sha256": "77d264ef14b69c625c6db9e9d4aa80abb2c1a19bf68b1d185c3ba9d4c22aaad0",
-    "backward": {"read": 271959296, "write": 32890880},
-    "forward": {"read": 102943744, "write": 21438208},
+    "sources_sha256": "bbdc62027627e6b1321072c2715d14102e149c15a87bb35033754587b1702b6b",
+    "backward": {"read": 272967424, "write": 32150272},
+    "forward": {"read": 102939392, "write": 21014784},
 }
 # the resident kernels' phase trace in the workspace (IABN_TRACE=1): up to 256
 # CTAs x 16 slots of 8 bytes, right after the 256-byte control block
